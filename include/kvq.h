@@ -1,0 +1,196 @@
+/*
+ * kvq.h -- C ABI of the B200 (sm_100a) mixed-precision quantized KV cache.
+ *
+ * What it computes (sources are web pages, cited by title and section):
+ *  - "Kuantisasi KV cache mengganggu attention melalui key dan value
+ *    tersimpan" (nalar.dev), section "Error pada key masuk sebelum softmax":
+ *    decode attention s = q K^T * sm_scale, a = softmax(s), o = a V over the
+ *    stored (reconstructed) keys and values; section "Granularitas
+ *    kuantisasi menentukan nilai yang berbagi scale": a group of values
+ *    shares one scale and one zero point; section "Pertumbuhan cache
+ *    mengubah trade pada serving": the newest tokens stay at higher
+ *    precision while older ones are quantized, and dequantization can be
+ *    fused into the attention kernel or done into temporary storage.
+ *  - "Quantize What Counts: More for Keys, Less for Values" (summary of
+ *    arXiv 2502.15075), Methodologie / Belangrijkste Bijdragen / Resultaten:
+ *    more bits for keys than values (e.g. K4V2), key groups of 32 channels,
+ *    value groups of 64-128, optional rotation of keys only.
+ *
+ * Quantizer (per token, per group of contiguous channels; the pages print
+ * no formula, this is the min/max reading):
+ *    zero  = fp16 of min(x) rounded toward -inf
+ *    scale = fp16 of ((max(x) - zero) / (2^b - 1)), every step rounded up
+ *    code  = clamp(rint((x - zero) / scale), 0, 2^b - 1)   (ties to even)
+ *    x^    = code * scale + zero                           (one fp32 fma)
+ * so |x - x^| <= scale/2 (+ fp32 rounding) for every element.  Inputs must
+ * keep group minima >= -65504 and (max - zero)/(2^b - 1) <= 65504; NaN and
+ * Inf are not supported.
+ *
+ * Conventions for every entry point:
+ *  - Device buffers are owned by the caller; the library never allocates,
+ *    frees or synchronizes, and keeps no pointer after a call returns.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream).  Calls on one stream run in order.
+ *  - Return value: KVQ_OK, or a negative KVQ_ERR_* code.  Arguments are
+ *    checked on the host before anything is launched; on an error nothing
+ *    is enqueued.  KVQ_ERR_CUDA reports a failed launch.
+ *  - Lengths live on the device (int32).  The host passes an upper bound
+ *    (max_len / max_new) used to size the launch; device lengths above it
+ *    are clamped to it, and page-table entries outside [0, num_pages) are
+ *    treated as absent pages (their tokens are skipped, never read).
+ *
+ * Storage layout (P = page_size tokens, d = head_dim, per layer):
+ *    k_codes [num_pages][Hkv][P][d*k_bits/8]  token rows; channel j in bits
+ *            k_bits*(j mod (32/k_bits)) of little-endian 32-bit word
+ *            floor(j*k_bits/32)
+ *    k_meta  [num_pages][Hkv][P][d/k_group] x {uint16 scale, uint16 zero}
+ *            (IEEE binary16 bit patterns)
+ *    v_codes [num_pages][Hkv][d][P*v_bits/8]  channel rows; token slot t in
+ *            bits v_bits*(t mod (32/v_bits)) of word floor(t*v_bits/32)
+ *    v_meta  [num_pages][Hkv][P][d/v_group] x {uint16 scale, uint16 zero}
+ *    k_win, v_win [batch][Hkv][window][d] bf16 ring, slot = position % window
+ *    page_table [batch][max_pages_per_seq] int32 physical page ids
+ *  Position p of sequence b lives in page page_table[b][p / P], slot p % P,
+ *  when p < len - window, and in ring slot p % window otherwise.  All
+ *  buffers must be 16-byte aligned.
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* kvq_stream_t; /* same type as cudaStream_t */
+
+enum {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = -1,  /* null pointer, negative size, bad alignment */
+    KVQ_ERR_UNSUPPORTED = -2,  /* bits, head_dim, groups or GQA outside the supported set */
+    KVQ_ERR_WORKSPACE = -3,    /* workspace missing or smaller than kvq_decode_workspace_bytes */
+    KVQ_ERR_CUDA = -4          /* a CUDA call or launch failed */
+};
+
+enum { KVQ_F32 = 0, KVQ_BF16 = 1 }; /* element types of inputs */
+
+/* Problem statement of one layer's cache.
+ * head_dim        d, 64 or 128
+ * num_q_heads     Hq; num_kv_heads Hkv; Hq % Hkv == 0, 1 <= Hq/Hkv <= 8
+ *                 (query head h reads kv-head h / (Hq/Hkv))
+ * k_bits, v_bits  1, 2, 4 or 8 ("more for keys": k_bits >= v_bits is the
+ *                 intended use, not a requirement)
+ * k_group,v_group channels per group: 16, 32, 64 or 128, dividing d
+ * page_size       tokens per page: 64
+ * window          W >= 0 newest positions kept in bf16 (0 = none)
+ * rotate_keys     1 = keys are multiplied by (diag(rot_signs) H / sqrt(d))
+ *                 before quantization (H Sylvester Walsh-Hadamard) and the
+ *                 query is rotated the same way when scoring quantized
+ *                 positions; window keys stay unrotated.
+ * rot_signs       device int8 [d] of +1/-1, required when rotate_keys
+ */
+typedef struct kvq_layout {
+    int head_dim;
+    int num_q_heads;
+    int num_kv_heads;
+    int k_bits;
+    int v_bits;
+    int k_group;
+    int v_group;
+    int page_size;
+    int window;
+    int rotate_keys;
+    const int8_t* rot_signs;
+} kvq_layout;
+
+/* Device buffers of one layer's cache (layout in the file header). */
+typedef struct kvq_cache {
+    void* k_codes;
+    void* v_codes;
+    void* k_meta;
+    void* v_meta;
+    void* k_win;                 /* bf16; may be NULL when window == 0 */
+    void* v_win;
+    const int32_t* page_table;   /* device [batch][max_pages_per_seq] */
+    int batch;
+    int max_pages_per_seq;
+    int num_pages;               /* physical pages in k_codes/... */
+} kvq_cache;
+
+/* Message for a status code (static string, never NULL). */
+const char* kvq_status_string(int status);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int kvq_version(void);
+
+/* Bytes of ONE physical page of each array (all kv-heads of the page):
+ * codes plus fp16 metadata ("Pertumbuhan cache ...": memory = payload +
+ * metadata).  Any output pointer may be NULL. */
+int kvq_page_bytes(const kvq_layout* layout, size_t* k_codes, size_t* k_meta,
+                   size_t* v_codes, size_t* v_meta);
+
+/* Bytes of one window ring (k_win or v_win) for `batch` sequences. */
+int kvq_window_bytes(const kvq_layout* layout, int batch, size_t* bytes);
+
+/* Workspace that kvq_decode_attention needs for this batch and bound on
+ * lengths on the current device (split partials); 0 on invalid input. */
+size_t kvq_decode_workspace_bytes(const kvq_layout* layout, int batch, int max_len);
+
+/* Append new tokens and quantize what leaves the bf16 window.
+ * ("Granularitas kuantisasi ..." group quantizer; "Pertumbuhan cache ..."
+ * recent-token window; "Quantize What Counts" K/V bit split.)
+ * k_new, v_new  device [total_new][Hkv][d], in_dtype KVQ_BF16 or KVQ_F32,
+ *               rows of sequence b are cu_new[b] .. cu_new[b+1]-1
+ * cu_new        device int32 [batch+1], non-decreasing, cu_new[0] == 0
+ * lens          device int32 [batch], tokens already in the cache; NOT
+ *               updated here -- the caller advances it (lens += n) on the
+ *               same stream before the next call
+ * max_new       host bound on cu_new[b+1]-cu_new[b] (launch size)
+ * Positions [max(0, L-W), max(0, L+n-W)) are quantized into pages (read
+ * from the ring when older than L); positions [max(L, L+n-W), L+n) are
+ * written to the ring (fp32 input rounded to nearest-even bf16).  Pages
+ * must be mapped for every quantized position. */
+int kvq_quantize_append(const kvq_layout* layout, const kvq_cache* cache,
+                        const void* k_new, const void* v_new, int in_dtype,
+                        const int32_t* cu_new, const int32_t* lens, int max_new,
+                        kvq_stream_t stream);
+
+/* Decode attention of one query token per sequence over the cache, with
+ * dequantization fused into the kernel ("Pertumbuhan cache ..."), GQA and
+ * ragged lengths; split-K over the sequence, then a log-sum-exp combine.
+ * q         device [batch][Hq][d], q_dtype KVQ_BF16 or KVQ_F32
+ * lens      device int32 [batch] (cached tokens); max_len >= max(lens)
+ * sm_scale  score scale (1/sqrt(d) for standard attention)
+ * out       device fp32 [batch][Hq][d]; lse device fp32 [batch][Hq] (natural
+ *           log of sum exp(scores)) or NULL.  A sequence of length 0 gets
+ *           out = 0 and lse = -inf.
+ * workspace device, >= kvq_decode_workspace_bytes(layout, batch, max_len)
+ *           bytes, 256-byte aligned; its contents need no initialisation. */
+int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache,
+                         const void* q, int q_dtype, const int32_t* lens, int max_len,
+                         float sm_scale, float* out, float* lse,
+                         void* workspace, size_t workspace_bytes, kvq_stream_t stream);
+
+/* Reconstruct the cache to fp32 [batch][Hkv][max_len][d] (check path;
+ * "dequantization into temporary storage").  Quantized positions give
+ * code*scale+zero (keys in the rotated domain when rotate_keys), window
+ * positions give their bf16 values; positions >= lens[b] are not written. */
+int kvq_dequantize(const kvq_layout* layout, const kvq_cache* cache,
+                   const int32_t* lens, int max_len, float* k_out, float* v_out,
+                   kvq_stream_t stream);
+
+/* Rotate `rows` key rows [rows][Hkv... flattened][d] exactly as
+ * kvq_quantize_append does before quantizing them (check path for the
+ * key-only rotation of "Quantize What Counts", Resultaten).
+ * k       device [rows][d] (in_dtype KVQ_BF16 or KVQ_F32)
+ * out     device fp32 [rows][d] */
+int kvq_rotate_keys(const kvq_layout* layout, const void* k, int in_dtype, int rows,
+                    float* out, kvq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

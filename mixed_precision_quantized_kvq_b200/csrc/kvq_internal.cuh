@@ -1,0 +1,126 @@
+// Internal declarations of the kvq CUDA library (sm_100a).
+// Kernel parameter block, cache addressing and the launchers that the C-ABI
+// layer (kvq_api.cu) calls.  Nothing here is visible outside the library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int kPage = 64;          // tokens per page
+constexpr int kMaxGqa = 8;         // query heads per kv-head
+
+// Flat copy of kvq_layout + kvq_cache with the derived strides kernels use.
+struct Params {
+    int d, hq, hkv, g;             // head_dim, heads, gqa ratio
+    int kb, vb, kg, vg;            // bits and group sizes
+    int nkg, nvg;                  // groups per row
+    int W;                         // window
+    int rotate;
+    const int8_t* signs;
+    uint8_t* k_codes;
+    uint8_t* v_codes;
+    uint32_t* k_meta;              // {u16 scale, u16 zero} per group
+    uint32_t* v_meta;
+    __nv_bfloat16* k_win;
+    __nv_bfloat16* v_win;
+    const int32_t* page_table;
+    int batch, max_pages, num_pages;
+    int krow_bytes;                // d*kb/8
+    int vchan_bytes;               // page*vb/8
+};
+
+// ---- cache addressing (layout documented in kvq.h) ----------------------
+__device__ __forceinline__ uint8_t* k_code_row(const Params& p, int page, int h, int slot) {
+    return p.k_codes + ((size_t(page) * p.hkv + h) * kPage + slot) * p.krow_bytes;
+}
+__device__ __forceinline__ uint32_t* k_meta_row(const Params& p, int page, int h, int slot) {
+    return p.k_meta + ((size_t(page) * p.hkv + h) * kPage + slot) * p.nkg;
+}
+__device__ __forceinline__ uint8_t* v_code_chan(const Params& p, int page, int h, int j) {
+    return p.v_codes + ((size_t(page) * p.hkv + h) * p.d + j) * p.vchan_bytes;
+}
+__device__ __forceinline__ uint32_t* v_meta_row(const Params& p, int page, int h, int slot) {
+    return p.v_meta + ((size_t(page) * p.hkv + h) * kPage + slot) * p.nvg;
+}
+__device__ __forceinline__ size_t win_off(const Params& p, int b, int h, int pos) {
+    return ((size_t(b) * p.hkv + h) * p.W + (pos % p.W)) * p.d;
+}
+// physical page of logical page `lp` of sequence b, or -1 when absent
+__device__ __forceinline__ int phys_page(const Params& p, int b, int lp) {
+    if (lp < 0 || lp >= p.max_pages) return -1;
+    int pg = __ldg(p.page_table + size_t(b) * p.max_pages + lp);
+    return (pg >= 0 && pg < p.num_pages) ? pg : -1;
+}
+
+// meta word -> (scale, zero) as fp32
+__device__ __forceinline__ float2 meta_f2(uint32_t w) {
+    __half2 h = *reinterpret_cast<const __half2*>(&w);
+    return __half22float2(h);   // .x = scale, .y = zero
+}
+
+// ---- key-only rotation (Walsh-Hadamard), shared by append and decode ----
+template <int D>
+struct RotScale;
+template <>
+struct RotScale<64> { static constexpr float v = 0.125f; };
+template <>
+struct RotScale<128> { static constexpr float v = 0.0883883476483184405f; };  // 1/sqrt(128)
+
+// x holds channels lane*CPL .. lane*CPL+CPL-1.  Sylvester-ordered transform:
+// butterflies (a, b) -> (a + b, a - b) over strides 1, 2, ..., D/2.
+template <int D>
+__device__ __forceinline__ void rotate_warp(float (&x)[D / 32], const int8_t* signs, int lane) {
+    constexpr int CPL = D / 32;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) x[i] = __fmul_rn(x[i], (float)__ldg(signs + lane * CPL + i));
+#pragma unroll
+    for (int s = 1; s < CPL; s <<= 1) {
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            if (!(i & s)) {
+                float a = x[i], b = x[i + s];
+                x[i] = __fadd_rn(a, b);
+                x[i + s] = __fsub_rn(a, b);
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            float o = __shfl_xor_sync(0xffffffffu, x[i], m);
+            x[i] = (lane & m) ? __fsub_rn(o, x[i]) : __fadd_rn(x[i], o);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) x[i] = __fmul_rn(x[i], RotScale<D>::v);
+}
+
+// ---- launchers -----------------------------------------------------------
+struct DecodePlan {
+    int splits_q;       // splits over quantized pages
+    int pages_per_split;
+    int window_split;   // 1 if a separate split handles the bf16 window
+    int total_splits;
+};
+DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count);
+size_t decode_workspace_bytes(const Params& p, int batch, const DecodePlan& plan);
+
+cudaError_t launch_quantize_append(const Params& p, const void* k_new, const void* v_new,
+                                   int in_bf16, const int32_t* cu_new, const int32_t* lens,
+                                   int max_new, cudaStream_t s);
+cudaError_t launch_dequantize(const Params& p, const int32_t* lens, int max_len, float* k_out,
+                              float* v_out, cudaStream_t s);
+cudaError_t launch_rotate_keys(const Params& p, const void* k, int in_bf16, int rows, float* out,
+                               cudaStream_t s);
+cudaError_t launch_decode(const Params& p, const void* q, int q_bf16, const int32_t* lens,
+                          int max_len, float sm_scale, float* out, float* lse, void* ws,
+                          const DecodePlan& plan, cudaStream_t s);
+
+}  // namespace kvq

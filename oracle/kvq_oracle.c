@@ -162,8 +162,10 @@ static float op_mode(float a, float b, int op, int rmode)
 }
 float kvqo_sub_ru(float a, float b) { return op_mode(a, b, 0, FE_UPWARD); }
 float kvqo_div_ru(float a, float b) { return op_mode(a, b, 1, FE_UPWARD); }
-float kvqo_sub_rn(float a, float b) { return op_mode(a, b, 0, FE_TONEAREST); }
-float kvqo_div_rn(float a, float b) { return op_mode(a, b, 1, FE_TONEAREST); }
+/* Round-to-nearest is the default mode of the process (the oracle never
+ * leaves another mode set), so these are the plain IEEE operations. */
+float kvqo_sub_rn(float a, float b) { volatile float va = a, vb = b; return va - vb; }
+float kvqo_div_rn(float a, float b) { volatile float va = a, vb = b; return va / vb; }
 
 /* ------------------------------------------------------------------------
  * Group quantizer.  [P1] "Granularitas kuantisasi ...": a group of values

@@ -191,19 +191,34 @@ def seq_kv(w: Workload, b: int, n: int, start: int = 0):
     return kr, vr, kf, vf
 
 
-def prefill(w: Workload, lens: Optional[np.ndarray] = None):
+def prefill(w: Workload, lens: Optional[np.ndarray] = None, with_f32: bool = True):
     """Ragged prefill batch: (k_raw, v_raw, k_f32, v_f32, cu_new, lens).
 
     k_raw is [sum(lens)][Hkv][d] (bf16 bits as uint16, or fp32); cu_new is the
-    exclusive prefix sum [B+1].
+    exclusive prefix sum [B+1].  With with_f32=False the fp32 views are None
+    (saves host memory on the large workloads).
     """
     if lens is None:
         lens = lengths(w)
-    parts = [seq_kv(w, b, int(lens[b])) for b in range(w.batch)]
+    lens = np.asarray(lens, dtype=np.int32)
     cu = np.zeros(w.batch + 1, dtype=np.int32)
     cu[1:] = np.cumsum(lens)
-    cat = [np.concatenate([p[i] for p in parts], axis=0) for i in range(4)]
-    return cat[0], cat[1], cat[2], cat[3], cu, np.asarray(lens, dtype=np.int32)
+    total = int(cu[-1])
+    shape = (total, w.num_kv_heads, w.head_dim)
+    rdt = np.uint16 if w.in_dtype == DT_BF16 else np.float32
+    kr = np.empty(shape, rdt)
+    vr = np.empty(shape, rdt)
+    kf = np.empty(shape, np.float32) if with_f32 else None
+    vf = np.empty(shape, np.float32) if with_f32 else None
+    for b in range(w.batch):
+        if lens[b] == 0:
+            continue
+        a, e = int(cu[b]), int(cu[b + 1])
+        k_raw, v_raw, k_f, v_f = seq_kv(w, b, int(lens[b]))
+        kr[a:e], vr[a:e] = k_raw, v_raw
+        if with_f32:
+            kf[a:e], vf[a:e] = k_f, v_f
+    return kr, vr, kf, vf, cu, lens
 
 
 def new_tokens(w: Workload, step: int):
