@@ -138,6 +138,21 @@ int kvq_window_bytes(const kvq_layout* layout, int batch, size_t* bytes);
  * lengths on the current device (split partials); 0 on invalid input. */
 size_t kvq_decode_workspace_bytes(const kvq_layout* layout, int batch, int max_len);
 
+/* Select the decode kernel family for subsequent kvq_decode_attention and
+ * kvq_decode_workspace_bytes calls (process-wide):
+ *   0  automatic (default): tensor-core kernel where the layout supports it
+ *      (head_dim 128, key groups of 32, value groups of 128, bit pairs
+ *      K/V in {4/2, 4/4, 8/8, 2/4, 2/2, 1/2}), CUDA-core kernel otherwise
+ *   1  CUDA-core kernel for every layout
+ *   2  same as 0 (tensor cores where supported)
+ * Not thread-safe with concurrent calls; query workspace sizes after
+ * changing it.  Returns KVQ_ERR_INVALID_ARG for other values. */
+int kvq_set_decode_path(int path);
+
+/* Decode kernel family the current setting picks for this layout:
+ * 2 = tensor cores, 1 = CUDA cores, or a negative KVQ_ERR_* code. */
+int kvq_get_decode_path(const kvq_layout* layout);
+
 /* Append new tokens and quantize what leaves the bf16 window.
  * ("Granularitas kuantisasi ..." group quantizer; "Pertumbuhan cache ..."
  * recent-token window; "Quantize What Counts" K/V bit split.)

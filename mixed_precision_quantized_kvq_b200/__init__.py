@@ -71,6 +71,10 @@ def lib() -> C.CDLL:
         L.kvq_decode_attention.argtypes = [LP, CP, P, I, P, I, C.c_float, P, P, P, S, P]
         L.kvq_dequantize.argtypes = [LP, CP, P, I, P, P, P]
         L.kvq_rotate_keys.argtypes = [LP, P, I, I, P, P]
+        L.kvq_set_decode_path.argtypes = [I]
+        L.kvq_set_decode_path.restype = I
+        L.kvq_get_decode_path.argtypes = [LP]
+        L.kvq_get_decode_path.restype = I
         for n in ("kvq_page_bytes", "kvq_window_bytes", "kvq_quantize_append",
                   "kvq_decode_attention", "kvq_dequantize", "kvq_rotate_keys"):
             getattr(L, n).restype = I
@@ -214,6 +218,21 @@ def kvq_rotate_keys(layout: Layout, k: torch.Tensor, out: torch.Tensor, stream=N
     rows = k.numel() // layout.head_dim
     _call("kvq_rotate_keys", C.byref(layout.c()), _ptr(k), _dtype_code(k), int(rows), _ptr(out),
           _stream(stream))
+
+
+DECODE_AUTO, DECODE_CUDA_CORES, DECODE_TENSOR_CORES = 0, 1, 2
+
+
+def kvq_set_decode_path(path: int) -> None:
+    """kvq.h kvq_set_decode_path: 0 automatic, 1 CUDA cores, 2 tensor cores."""
+    _call("kvq_set_decode_path", int(path))
+
+
+def kvq_get_decode_path(layout: Layout) -> int:
+    rc = int(lib().kvq_get_decode_path(C.byref(layout.c())))
+    if rc < 0:
+        raise KVQError("kvq_get_decode_path", rc)
+    return rc
 
 
 # ---------------------------------------------------------------- helpers

@@ -141,6 +141,19 @@ size_t kvq_decode_workspace_bytes(const kvq_layout* layout, int batch, int max_l
     return kvq::decode_workspace_bytes(p, batch, pl);
 }
 
+int kvq_set_decode_path(int path) {
+    if (path < 0 || path > 2) return KVQ_ERR_INVALID_ARG;
+    kvq::g_decode_path = path;
+    return KVQ_OK;
+}
+
+int kvq_get_decode_path(const kvq_layout* layout) {
+    int rc = check_layout(layout);
+    if (rc) return rc;
+    Params p = make_params(layout, nullptr);
+    return (kvq::g_decode_path != 1 && kvq::tc_supported(p)) ? 2 : 1;
+}
+
 int kvq_quantize_append(const kvq_layout* layout, const kvq_cache* cache, const void* k_new,
                         const void* v_new, int in_dtype, const int32_t* cu_new, const int32_t* lens,
                         int max_new, kvq_stream_t stream) {

@@ -18,12 +18,35 @@
 
 namespace kvq {
 
+int g_decode_path = 0;
+
 DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count) {
     DecodePlan pl{};
     const int maxq = max_len - p.W > 0 ? max_len - p.W : 0;
     const int npages = (maxq + kPage - 1) / kPage;
     pl.window_split = p.W > 0 ? 1 : 0;
     const int units = batch * p.hkv > 0 ? batch * p.hkv : 1;
+    pl.tc = (g_decode_path != 1 && tc_supported(p)) ? 1 : 0;
+    if (pl.tc) {
+        // one wave of CTAs: as many splits per (sequence, kv-head) as the
+        // resident CTA slots allow, each a whole number of 128-token tiles
+        const int slots = sm_count * tc_ctas_per_sm(p);
+        const int tiles = (npages + 1) / 2;
+        int want = slots / units;
+        if (want < 1) want = 1;
+        if (npages == 0) {
+            pl.splits_q = 0;
+            pl.pages_per_split = 2;
+        } else {
+            if (want > tiles) want = tiles;
+            pl.pages_per_split = 2 * ((tiles + want - 1) / want);
+            pl.splits_q = (npages + pl.pages_per_split - 1) / pl.pages_per_split;
+        }
+        pl.grid_x = pl.splits_q > 0 ? pl.splits_q : 1;
+        pl.window_slot = pl.grid_x;
+        pl.total_splits = pl.grid_x + pl.window_split;
+        return pl;
+    }
     // about four resident CTAs per SM over the quantized pages
     int want = (4 * sm_count + units - 1) / units;
     if (want < 1) want = 1;
@@ -37,6 +60,8 @@ DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count) {
     }
     pl.total_splits = pl.splits_q + pl.window_split;
     if (pl.total_splits == 0) pl.total_splits = 1;   // all-empty: one split writes zeros
+    pl.grid_x = pl.total_splits;
+    pl.window_slot = pl.total_splits - 1;
     return pl;
 }
 
@@ -244,10 +269,22 @@ __global__ void __launch_bounds__(128) decode_split_simt(Params p, const void* _
         // ---------------- values
         if (is_win) {
             for (int r = hsel; r < g; r += hstep) o[r] *= a_s[r];
-            for (int tt = 0; tt < kPage; ++tt) {
-                const int ps = chunk_base + tt;
-                if (ps >= c_end) break;
-                const float v = __bfloat162float(p.v_win[win_off(p, b, h, ps) + jc]);
+            const int n = min(kPage, c_end - chunk_base);
+            int tt = 0;
+            for (; tt + 16 <= n; tt += 16) {               // 16 independent loads in flight
+                float v[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    v[k] = __bfloat162float(p.v_win[win_off(p, b, h, chunk_base + tt + k) + jc]);
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+#pragma unroll
+                    for (int r = 0; r < kMaxGqa; ++r)
+                        if (r < g && (r - hsel) % hstep == 0 && r >= hsel)
+                            o[r] = fmaf(pv_s[r][0][tt + k], v[k], o[r]);
+            }
+            for (; tt < n; ++tt) {
+                const float v = __bfloat162float(p.v_win[win_off(p, b, h, chunk_base + tt) + jc]);
 #pragma unroll
                 for (int r = 0; r < kMaxGqa; ++r)
                     if (r < g && (r - hsel) % hstep == 0 && r >= hsel) o[r] = fmaf(pv_s[r][0][tt], v, o[r]);
@@ -364,7 +401,8 @@ cudaError_t launch_decode(const Params& p, const void* q, int q_bf16, const int3
     size_t ob = (rows * pl.total_splits * p.d * sizeof(float) + 255) & ~size_t(255);
     float* ws_ml = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + ob);
     const float sl2 = sm_scale * 1.4426950408889634f;
-    cudaError_t e = (p.d == 128) ? dispatch_kb<128>(p, q, q_bf16, lens, max_len, sl2, ws_o, ws_ml, pl, s)
+    cudaError_t e = pl.tc ? launch_decode_tc(p, q, q_bf16, lens, max_len, sl2, ws_o, ws_ml, pl, s)
+                  : (p.d == 128) ? dispatch_kb<128>(p, q, q_bf16, lens, max_len, sl2, ws_o, ws_ml, pl, s)
                                  : dispatch_kb<64>(p, q, q_bf16, lens, max_len, sl2, ws_o, ws_ml, pl, s);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((rows + 3) / 4));

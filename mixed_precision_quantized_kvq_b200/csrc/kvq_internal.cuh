@@ -104,12 +104,21 @@ __device__ __forceinline__ void rotate_warp(float (&x)[D / 32], const int8_t* si
 
 // ---- launchers -----------------------------------------------------------
 struct DecodePlan {
+    int tc;             // 1: tensor-core kernel, 0: CUDA-core kernel
     int splits_q;       // splits over quantized pages
     int pages_per_split;
-    int window_split;   // 1 if a separate split handles the bf16 window
-    int total_splits;
+    int window_split;   // 1 if the layout has a bf16 window (one more partial slot)
+    int total_splits;   // partial slots per (sequence, query head)
+    int grid_x;         // CTAs per (sequence, kv-head)
+    int window_slot;    // slot index of the window partial
 };
+// decode path selection: 0 = automatic, 1 = CUDA cores, 2 = tensor cores
+extern int g_decode_path;
 DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count);
+bool tc_supported(const Params& p);
+int tc_ctas_per_sm(const Params& p);
+cudaError_t launch_decode_tc(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len,
+                             float scale_log2, float* ws_o, float* ws_ml, const DecodePlan& pl, cudaStream_t s);
 size_t decode_workspace_bytes(const Params& p, int batch, const DecodePlan& plan);
 
 cudaError_t launch_quantize_append(const Params& p, const void* k_new, const void* v_new,

@@ -121,6 +121,9 @@ class Pair:
 def check_close(got, want, what="value"):
     got = np.asarray(got, np.float64)
     want = np.asarray(want, np.float64)
+    assert got.shape == want.shape
+    if got.size == 0:
+        return 0.0
     err = np.abs(got - want)
     lim = ATOL + RTOL * np.abs(want)
     if not np.all(err <= lim):

@@ -15,6 +15,22 @@ from gpu_harness import Pair, check_close, torch_raw
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(autouse=True, params=[kvq.DECODE_AUTO, kvq.DECODE_CUDA_CORES], ids=["auto", "cuda_cores"])
+def decode_path(request):
+    """Every case runs on the automatic choice (tensor cores where the layout
+    allows) and on the CUDA-core kernel."""
+    kvq.kvq_set_decode_path(request.param)
+    yield request.param
+    kvq.kvq_set_decode_path(kvq.DECODE_AUTO)
+
+
+def test_tensor_core_path_selected_for_k4v2_layout(decode_path):
+    lay = kvq.Layout(128, 32, 8, 4, 2, 32, 128, 64, 128)
+    want = kvq.DECODE_TENSOR_CORES if decode_path == kvq.DECODE_AUTO else kvq.DECODE_CUDA_CORES
+    assert kvq.kvq_get_decode_path(lay) == want
+    assert kvq.kvq_get_decode_path(kvq.Layout(64, 4, 4, 4, 2, 32, 64, 64, 0)) == kvq.DECODE_CUDA_CORES
+
+
 def small(**kw):
     base = dict(name="small", batch=4, num_q_heads=8, num_kv_heads=2, head_dim=128, seq_len=0,
                 k_bits=4, v_bits=2, k_group=32, v_group=128, window=0, ragged=(1, 700),
@@ -70,9 +86,9 @@ def test_fp32_inputs_with_window():
     run_prefill_and_decode(small(in_dtype=wl.DT_F32, window=40, head_dim=64, k_group=32, v_group=64))
 
 
-@pytest.mark.parametrize("d", [64, 128])
-def test_rotation(d):
-    w = small(rotate_keys=True, head_dim=d, v_group=64, outliers=("student_t", 4, 10.0, 3.0))
+@pytest.mark.parametrize("d,vg", [(64, 64), (128, 128)])
+def test_rotation(d, vg):
+    w = small(rotate_keys=True, head_dim=d, v_group=vg, outliers=("student_t", 4, 10.0, 3.0))
     lens = wl.lengths(w)
     kr, vr, kf, vf, cu, _ = wl.prefill(w, lens)
     pair = Pair(w, lens)
