@@ -50,6 +50,12 @@
  *    v_meta  [num_pages][Hkv][P][d/v_group] x {uint16 scale, uint16 zero}
  *    k_win, v_win [batch][Hkv][window][d] bf16 ring, slot = position % window
  *    page_table [batch][max_pages_per_seq] int32 physical page ids
+ *  Code rows longer than 16 bytes (key rows of d*k_bits/8 bytes, value
+ *  channel runs of P*v_bits/8 bytes) are stored as 16-byte chunks,
+ *  chunk-major inside each (page, kv-head) block: chunk i of token slot t
+ *  at byte i*(P*16) + t*16 of the key block, chunk i of channel j at byte
+ *  i*(d*16) + j*16 of the value block.  A row of at most 16 bytes is one
+ *  chunk, so the plain row-major form above is then exact.
  *  Position p of sequence b lives in page page_table[b][p / P], slot p % P,
  *  when p < len - window, and in ring slot p % window otherwise.  All
  *  buffers must be 16-byte aligned.

@@ -76,6 +76,8 @@ Params make_params(const kvq_layout* l, const kvq_cache* c) {
     p.signs = l->rot_signs;
     p.krow_bytes = p.d * p.kb / 8;
     p.vchan_bytes = kvq::kPage * p.vb / 8;
+    p.kch = p.krow_bytes < 16 ? p.krow_bytes : 16;
+    p.vch = p.vchan_bytes < 16 ? p.vchan_bytes : 16;
     if (c) {
         p.k_codes = static_cast<uint8_t*>(c->k_codes);
         p.v_codes = static_cast<uint8_t*>(c->v_codes);

@@ -126,8 +126,7 @@ __global__ void __launch_bounds__(128) quantize_pages_kernel(Params p, const voi
         const int lpw = 32 / lane_bits;                  // lanes per 32-bit word
         bitsv <<= (lane % lpw) * lane_bits;
         for (int o = 1; o < lpw; o <<= 1) bitsv |= __shfl_xor_sync(FULL, bitsv, o);
-        if (lane % lpw == 0)
-            reinterpret_cast<uint32_t*>(k_code_row(p, page, h, slot))[lane / lpw] = bitsv;
+        if (lane % lpw == 0) *k_word(p, page, h, slot, lane / lpw) = bitsv;
         // ---- values: metadata per token, codes staged per channel
         uint32_t vc[CPL];
         uint32_t vm = quantize_warp<D>(vx, p.vg, p.vb, vc);
@@ -142,9 +141,9 @@ __global__ void __launch_bounds__(128) quantize_pages_kernel(Params p, const voi
     const int slot0 = base % kPage;
     for (int t = threadIdx.x; t < D * words; t += blockDim.x) {
         const int j = t / words, wi = t % words;
-        uint32_t* dst = reinterpret_cast<uint32_t*>(v_code_chan(p, page, h, j)) + (slot0 + wi * per) / per;
+        uint32_t* dst = v_word(p, page, h, j, (slot0 + wi * per) / per);
         uint32_t word = 0, keep = 0;
-        const uint32_t fmask = (p.vb == 32) ? FULL : ((1u << p.vb) - 1u);
+        const uint32_t fmask = (1u << p.vb) - 1u;
         for (int i = 0; i < per; ++i) {
             const int s32 = wi * per + i;
             const int pos = base + s32;
@@ -223,7 +222,6 @@ __global__ void __launch_bounds__(128) dequantize_kernel(Params p, const int32_t
     const int page = phys_page(p, b, pos / kPage);
     if (page < 0) return;
     const int slot = pos % kPage;
-    const uint32_t* krow = reinterpret_cast<const uint32_t*>(k_code_row(p, page, h, slot));
     const uint32_t* kmr = k_meta_row(p, page, h, slot);
     const uint32_t* vmr = v_meta_row(p, page, h, slot);
     const int kper = 32 / p.kb, vper = 32 / p.vb;
@@ -231,11 +229,10 @@ __global__ void __launch_bounds__(128) dequantize_kernel(Params p, const int32_t
 #pragma unroll
     for (int i = 0; i < CPL; ++i) {
         const int j = lane * CPL + i;
-        uint32_t kc = (krow[j / kper] >> (p.kb * (j % kper))) & kmask;
+        uint32_t kc = (*k_word(p, page, h, slot, j / kper) >> (p.kb * (j % kper))) & kmask;
         float2 km = meta_f2(kmr[j / p.kg]);
         ko[i] = __fmaf_rn((float)kc, km.x, km.y);
-        const uint32_t* vch = reinterpret_cast<const uint32_t*>(v_code_chan(p, page, h, j));
-        uint32_t vc = (vch[slot / vper] >> (p.vb * (slot % vper))) & vmask;
+        uint32_t vc = (*v_word(p, page, h, j, slot / vper) >> (p.vb * (slot % vper))) & vmask;
         float2 vm = meta_f2(vmr[j / p.vg]);
         vo[i] = __fmaf_rn((float)vc, vm.x, vm.y);
     }

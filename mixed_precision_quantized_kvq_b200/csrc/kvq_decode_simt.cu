@@ -40,11 +40,12 @@ DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count) {
         } else {
             if (want > tiles) want = tiles;
             pl.pages_per_split = 2 * ((tiles + want - 1) / want);
+            if (pl.pages_per_split > 256) pl.pages_per_split = 256;   // page ids staged in shared memory
             pl.splits_q = (npages + pl.pages_per_split - 1) / pl.pages_per_split;
         }
         pl.grid_x = pl.splits_q > 0 ? pl.splits_q : 1;
-        pl.window_slot = pl.grid_x;
-        pl.total_splits = pl.grid_x + pl.window_split;
+        pl.window_slot = pl.grid_x - 1;                 // window tiles join the last split
+        pl.total_splits = pl.grid_x;
         return pl;
     }
     // about four resident CTAs per SM over the quantized pages
@@ -206,9 +207,8 @@ __global__ void __launch_bounds__(128) decode_split_simt(Params p, const void* _
             uint32_t kw[KW];
             float2 km[D / 16];
             if (ok) {
-                const uint32_t* kr = reinterpret_cast<const uint32_t*>(k_code_row(p, page, h, pos % kPage));
 #pragma unroll
-                for (int w = 0; w < KW; ++w) kw[w] = kr[w];
+                for (int w = 0; w < KW; ++w) kw[w] = *k_word(p, page, h, pos % kPage, w);
                 const uint32_t* mr = k_meta_row(p, page, h, pos % kPage);
                 for (int gi = 0; gi < p.nkg; ++gi) km[gi] = meta_f2(mr[gi]);
             }
@@ -292,9 +292,8 @@ __global__ void __launch_bounds__(128) decode_split_simt(Params p, const void* _
         } else {
             uint32_t vw[VW];
             if (page >= 0) {
-                const uint32_t* vr = reinterpret_cast<const uint32_t*>(v_code_chan(p, page, h, jc));
 #pragma unroll
-                for (int w = 0; w < VW; ++w) vw[w] = vr[w];
+                for (int w = 0; w < VW; ++w) vw[w] = *v_word(p, page, h, jc, w);
             }
 #pragma unroll
             for (int r = 0; r < kMaxGqa; ++r) {

@@ -33,17 +33,31 @@ struct Params {
     int batch, max_pages, num_pages;
     int krow_bytes;                // d*kb/8
     int vchan_bytes;               // page*vb/8
+    int kch, vch;                  // chunk bytes: min(16, row bytes)
 };
 
 // ---- cache addressing (layout documented in kvq.h) ----------------------
-__device__ __forceinline__ uint8_t* k_code_row(const Params& p, int page, int h, int slot) {
-    return p.k_codes + ((size_t(page) * p.hkv + h) * kPage + slot) * p.krow_bytes;
+// Code rows longer than 16 bytes are stored as 16-byte chunks, chunk-major
+// inside the (page, kv-head) block, so that one thread per token (keys) or
+// per channel (values) reading chunk i hits consecutive 16-byte units.
+__device__ __forceinline__ uint8_t* k_block(const Params& p, int page, int h) {
+    return p.k_codes + (size_t(page) * p.hkv + h) * size_t(kPage) * p.krow_bytes;
+}
+__device__ __forceinline__ uint32_t* k_word(const Params& p, int page, int h, int slot, int w) {
+    const int byte = 4 * w;
+    return reinterpret_cast<uint32_t*>(k_block(p, page, h) + (byte / p.kch) * (kPage * p.kch) + slot * p.kch +
+                                       (byte % p.kch));
 }
 __device__ __forceinline__ uint32_t* k_meta_row(const Params& p, int page, int h, int slot) {
     return p.k_meta + ((size_t(page) * p.hkv + h) * kPage + slot) * p.nkg;
 }
-__device__ __forceinline__ uint8_t* v_code_chan(const Params& p, int page, int h, int j) {
-    return p.v_codes + ((size_t(page) * p.hkv + h) * p.d + j) * p.vchan_bytes;
+__device__ __forceinline__ uint8_t* v_block(const Params& p, int page, int h) {
+    return p.v_codes + (size_t(page) * p.hkv + h) * size_t(p.d) * p.vchan_bytes;
+}
+__device__ __forceinline__ uint32_t* v_word(const Params& p, int page, int h, int j, int w) {
+    const int byte = 4 * w;
+    return reinterpret_cast<uint32_t*>(v_block(p, page, h) + (byte / p.vch) * (p.d * p.vch) + j * p.vch +
+                                       (byte % p.vch));
 }
 __device__ __forceinline__ uint32_t* v_meta_row(const Params& p, int page, int h, int slot) {
     return p.v_meta + ((size_t(page) * p.hkv + h) * kPage + slot) * p.nvg;

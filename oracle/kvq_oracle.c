@@ -294,8 +294,10 @@ void kvqo_rotate(const float* x, const int8_t* signs, int d, float* y)
  * Cache layout (this library's storage format; the oracle writes it out on
  * its own).  Per layer:
  *   k_codes [pages][Hkv][P][d*kb/8]       token rows, channels packed
+ *           (rows over 16 bytes stored as 16-byte chunks, chunk-major)
  *   k_meta  [pages][Hkv][P][d/kg] {u16 scale, u16 zero}
  *   v_codes [pages][Hkv][d][P*vb/8]       channel rows, tokens packed
+ *           (likewise chunk-major when over 16 bytes)
  *   v_meta  [pages][Hkv][P][d/vg] {u16 scale, u16 zero}
  *   k_win, v_win [B][Hkv][W][d] bf16 ring, slot = position mod W
  *   page_table [B][max_pages] int32
@@ -351,18 +353,48 @@ int kvqo_page_bytes(const kvqo_layout* l, size_t* kc, size_t* km, size_t* vc, si
 static size_t krow_bytes(const kvqo_layout* l) { return (size_t)l->head_dim * l->k_bits / 8; }
 static size_t vrow_bytes(const kvqo_layout* l) { return (size_t)l->page_size * l->v_bits / 8; }
 
-static uint8_t* k_code_row(const kvqo_layout* l, const kvqo_cache* c, int page, int h, int slot)
+/* Code rows longer than 16 bytes are stored in 16-byte chunks, chunk-major
+ * inside the (page, kv-head) block: chunk i of token slot t of a key block
+ * sits at i*(P*16) + t*16 (and chunk i of value channel j at i*(d*16) +
+ * j*16).  Rows of at most 16 bytes are a single chunk. */
+static size_t chunk_of(size_t row_bytes) { return row_bytes < 16 ? row_bytes : 16; }
+
+static uint8_t* k_block(const kvqo_layout* l, const kvqo_cache* c, int page, int h)
 {
-    return c->k_codes + (((size_t)page * l->num_kv_heads + h) * l->page_size + slot) * krow_bytes(l);
+    return c->k_codes + ((size_t)page * l->num_kv_heads + h) * (size_t)l->page_size * krow_bytes(l);
+}
+static uint8_t* v_block(const kvqo_layout* l, const kvqo_cache* c, int page, int h)
+{
+    return c->v_codes + ((size_t)page * l->num_kv_heads + h) * (size_t)l->head_dim * vrow_bytes(l);
+}
+/* gather (put = 0) or scatter (put = 1) the packed key row of one token */
+static void k_row_io(const kvqo_layout* l, const kvqo_cache* c, int page, int h, int slot,
+                     uint8_t* row, int put)
+{
+    size_t rb = krow_bytes(l), ch = chunk_of(rb);
+    uint8_t* base = k_block(l, c, page, h);
+    for (size_t i = 0; i < rb / ch; ++i) {
+        uint8_t* at = base + i * (size_t)l->page_size * ch + (size_t)slot * ch;
+        if (put) memcpy(at, row + i * ch, ch);
+        else memcpy(row + i * ch, at, ch);
+    }
+}
+/* gather or scatter the packed token run of one value channel */
+static void v_chan_io(const kvqo_layout* l, const kvqo_cache* c, int page, int h, int j,
+                      uint8_t* run, int put)
+{
+    size_t rb = vrow_bytes(l), ch = chunk_of(rb);
+    uint8_t* base = v_block(l, c, page, h);
+    for (size_t i = 0; i < rb / ch; ++i) {
+        uint8_t* at = base + i * (size_t)l->head_dim * ch + (size_t)j * ch;
+        if (put) memcpy(at, run + i * ch, ch);
+        else memcpy(run + i * ch, at, ch);
+    }
 }
 static uint8_t* k_meta_row(const kvqo_layout* l, const kvqo_cache* c, int page, int h, int slot)
 {
     return c->k_meta + (((size_t)page * l->num_kv_heads + h) * l->page_size + slot) *
                            (size_t)(l->head_dim / l->k_group) * 4;
-}
-static uint8_t* v_code_chan(const kvqo_layout* l, const kvqo_cache* c, int page, int h, int j)
-{
-    return c->v_codes + (((size_t)page * l->num_kv_heads + h) * l->head_dim + j) * vrow_bytes(l);
 }
 static uint8_t* v_meta_row(const kvqo_layout* l, const kvqo_cache* c, int page, int h, int slot)
 {
@@ -404,7 +436,9 @@ static void quantize_token(const kvqo_layout* l, const kvqo_cache* c, int b, int
                             codes + g * l->k_group);
         put_meta(km + 4 * g, s, z);
     }
-    kvqo_pack(codes, d, l->k_bits, k_code_row(l, c, page, h, slot));
+    uint8_t row[256];
+    kvqo_pack(codes, d, l->k_bits, row);
+    k_row_io(l, c, page, h, slot, row, 1);
     /* values: groups of v_group channels; codes stored per channel */
     uint8_t* vm = v_meta_row(l, c, page, h, slot);
     for (int g = 0; g < d / l->v_group; ++g) {
@@ -413,8 +447,12 @@ static void quantize_token(const kvqo_layout* l, const kvqo_cache* c, int b, int
                             codes + g * l->v_group);
         put_meta(vm + 4 * g, s, z);
     }
-    for (int j = 0; j < d; ++j)
-        set_packed(v_code_chan(l, c, page, h, j), slot, l->v_bits, codes[j]);
+    for (int j = 0; j < d; ++j) {
+        uint8_t run[64];
+        v_chan_io(l, c, page, h, j, run, 0);
+        set_packed(run, slot, l->v_bits, codes[j]);
+        v_chan_io(l, c, page, h, j, run, 1);
+    }
 }
 
 static float load_in(const void* p, int in_dtype, size_t idx)
@@ -505,7 +543,8 @@ static int reconstruct(const kvqo_layout* l, const kvqo_cache* c, int b, int h,
     }
     int page = c->page_table[(size_t)b * c->max_pages_per_seq + pos / l->page_size];
     int slot = pos % l->page_size;
-    const uint8_t* kc = k_code_row(l, c, page, h, slot);
+    uint8_t kc[256], vrun[64];
+    k_row_io(l, c, page, h, slot, kc, 0);
     const uint8_t* km = k_meta_row(l, c, page, h, slot);
     const uint8_t* vm = v_meta_row(l, c, page, h, slot);
     for (int j = 0; j < d; ++j) {
@@ -513,7 +552,8 @@ static int reconstruct(const kvqo_layout* l, const kvqo_cache* c, int b, int h,
         get_meta(km + 4 * (j / l->k_group), &s, &z);
         k[j] = kvqo_dequant_code(kvqo_unpack_one(kc, j, l->k_bits), s, z);
         get_meta(vm + 4 * (j / l->v_group), &s, &z);
-        v[j] = kvqo_dequant_code(kvqo_unpack_one(v_code_chan(l, c, page, h, j), slot, l->v_bits), s, z);
+        v_chan_io(l, c, page, h, j, vrun, 0);
+        v[j] = kvqo_dequant_code(kvqo_unpack_one(vrun, slot, l->v_bits), s, z);
     }
     return 1;
 }

@@ -162,3 +162,33 @@ def test_max_len_larger_than_lengths():
     qr, out, lse = pair.decode(max_len=int(pair.lens.max()) + 1000)
     ref, _ = pair.oracle_decode(qr)
     check_close(out, ref)
+
+
+@pytest.mark.parametrize("window", [48, 200])
+def test_rotation_with_window(window):
+    """Rotated keys in pages, unrotated keys in the bf16 window: each scored
+    against the matching query."""
+    w = small(rotate_keys=True, window=window, ragged=(1, 900),
+              outliers=("student_t", 4, 10.0, 3.0))
+    lens = wl.lengths(w)
+    kr, vr, kf, vf, cu, _ = wl.prefill(w, lens)
+    pair = Pair(w, lens)
+    kt = torch_raw(kr)
+    rot = torch.empty(kt.shape, dtype=torch.float32, device="cuda")
+    kvq.kvq_rotate_keys(pair.glay, kt, rot)
+    rot = rot.cpu().numpy()
+    # oracle rows: rotated keys where the position ends up quantized, raw keys in the window
+    ok_rows = kf.astype(np.float32).copy()
+    for b in range(w.batch):
+        nq = max(0, int(lens[b]) - window)
+        ok_rows[cu[b]:cu[b] + nq] = rot[cu[b]:cu[b] + nq]
+    olay = oracle.Layout.from_workload(w.with_(rotate_keys=False))
+    pair.ocache = oracle.Cache(olay, w.batch, pair.pt, pair.num_pages)
+    pair.lens[:] = 0
+    pair.glens.zero_()
+    pair.append(kr, vr, cu, oracle_k=np.ascontiguousarray(ok_rows), oracle_dtype=oracle.IN_F32)
+    # the oracle's window holds fp32 rows rounded to bf16 (exact: they came from bf16)
+    pair.compare_cache()
+    pair.ocache.layout = pair.olay
+    pair.ocache._signs = np.ascontiguousarray(pair.signs)
+    pair.check_decode()

@@ -185,3 +185,31 @@ def test_fp32_inputs_enter_window_rounded_to_bf16():
     kh, _ = c.dequantize(lens, 20)
     want = wl.bf16_to_f32(oracle.f32_to_bf16(kf[cu[0] + 12:cu[0] + 20, 0].ravel()))
     np.testing.assert_array_equal(kh[0, 0, 12:20].ravel(), want)
+
+
+def test_chunked_code_positions_hand_derived():
+    """Storage format: key rows and value channel runs over 16 bytes are kept
+    as 16-byte chunks, chunk-major inside a (page, kv-head) block.  K4 at
+    head_dim 128: channel 40 of token slot 5 is nibble 0 of row byte 20 =
+    chunk 1, byte 4 -> block offset 1*(64*16) + 5*16 + 4 = 1108.  V4: token
+    slot 37 of channel 9 is the high nibble of run byte 18 = chunk 1, byte 2
+    -> block offset 1*(128*16) + 9*16 + 2 = 2194."""
+    d = 128
+    lay = oracle.Layout(d, 1, 1, 4, 4, 32, 128, 64, 0)
+    pt = np.zeros((1, 1), np.int32)
+    c = oracle.Cache(lay, 1, pt, 1)
+    # on-grid values: zero 0, scale 1 -> code == value
+    k = np.zeros((64, 1, d), np.float32)
+    v = np.zeros((64, 1, d), np.float32)
+    k[:, :, 127] = 15.0                      # fixes every key group's range
+    for g0 in range(0, d, 32):
+        k[:, :, g0 + 31] = 15.0
+    v[:, :, 127] = 15.0
+    k[5, 0, 40] = 9.0
+    v[37, 0, 9] = 6.0
+    c.append(k, v, oracle.IN_F32, np.array([0, 64], np.int32), np.zeros(1, np.int32))
+    kb = c.k_codes.ravel()
+    vb = c.v_codes.ravel()
+    assert kb[1108] & 0x0F == 9
+    assert (vb[2194] >> 4) == 6
+    assert kb[1108 - 16] & 0x0F == 0         # same byte of token slot 4
