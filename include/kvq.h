@@ -194,6 +194,34 @@ int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache,
                          float sm_scale, float* out, float* lse,
                          void* workspace, size_t workspace_bytes, kvq_stream_t stream);
 
+/* Bytes of the library's static decode scratch (per device). */
+#define KVQ_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
+
+/* kvq_decode_attention without a caller-supplied workspace.  The pages
+ * have no counterpart to this call: it is a deployment convenience.  The
+ * split partials live in a file-scope static device array of
+ * KVQ_STATIC_SCRATCH_BYTES (8 MiB, 256-byte aligned) that the library
+ * holds in each device's context.  Its address is looked up once per
+ * device, on that device's first call.  The call allocates and frees
+ * nothing.
+ * Arguments, output and error behaviour are those of kvq_decode_attention,
+ * plus one case: KVQ_ERR_WORKSPACE, with nothing enqueued, when
+ * kvq_decode_workspace_bytes(layout, cache->batch, max_len) exceeds
+ * KVQ_STATIC_SCRATCH_BYTES.  For scale: batch 64 at lengths up to 16384
+ * with 40/8 heads needs 1.3 MB.
+ * Nothing needs to start at zero: each call writes every partial before
+ * its combine step reads it.
+ * One scratch array serves every call on a device.  Calls whose GPU
+ * execution overlaps (different streams without ordering between them, or
+ * several host threads) race on it and give undefined results.  Order them
+ * on one stream, or use kvq_decode_attention with a workspace per stream.
+ * The cached address belongs to the device's current context: do not call
+ * this after cudaDeviceReset. */
+int kvq_decode_attention_static_scratch(const kvq_layout* layout, const kvq_cache* cache,
+                                        const void* q, int q_dtype, const int32_t* lens,
+                                        int max_len, float sm_scale, float* out, float* lse,
+                                        kvq_stream_t stream);
+
 /* Reconstruct the cache to fp32 [batch][Hkv][max_len][d] (check path;
  * "dequantization into temporary storage").  Quantized positions give
  * code*scale+zero (keys in the rotated domain when rotate_keys), window

@@ -24,6 +24,7 @@ KVQ_ERR_WORKSPACE = -3
 KVQ_ERR_CUDA = -4
 KVQ_F32 = 0
 KVQ_BF16 = 1
+KVQ_STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
 PAGE_SIZE = 64
 
 
@@ -69,6 +70,7 @@ def lib() -> C.CDLL:
         L.kvq_decode_workspace_bytes.argtypes = [LP, I, I]
         L.kvq_quantize_append.argtypes = [LP, CP, P, P, I, P, P, I, P]
         L.kvq_decode_attention.argtypes = [LP, CP, P, I, P, I, C.c_float, P, P, P, S, P]
+        L.kvq_decode_attention_static_scratch.argtypes = [LP, CP, P, I, P, I, C.c_float, P, P, P]
         L.kvq_dequantize.argtypes = [LP, CP, P, I, P, P, P]
         L.kvq_rotate_keys.argtypes = [LP, P, I, I, P, P]
         L.kvq_set_decode_path.argtypes = [I]
@@ -76,7 +78,8 @@ def lib() -> C.CDLL:
         L.kvq_get_decode_path.argtypes = [LP]
         L.kvq_get_decode_path.restype = I
         for n in ("kvq_page_bytes", "kvq_window_bytes", "kvq_quantize_append",
-                  "kvq_decode_attention", "kvq_dequantize", "kvq_rotate_keys"):
+                  "kvq_decode_attention", "kvq_decode_attention_static_scratch", "kvq_dequantize",
+                  "kvq_rotate_keys"):
             getattr(L, n).restype = I
         _lib_handle = L
     return _lib_handle
@@ -204,6 +207,18 @@ def kvq_decode_attention(layout: Layout, cache: PagedCache, q: torch.Tensor, len
     _call("kvq_decode_attention", C.byref(layout.c()), C.byref(cache.c()), _ptr(q), _dtype_code(q),
           _ptr(lens), int(max_len), C.c_float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace),
           C.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
+
+
+def kvq_decode_attention_static_scratch(layout: Layout, cache: PagedCache, q: torch.Tensor,
+                                        lens: torch.Tensor, max_len: int, sm_scale: float,
+                                        out: torch.Tensor, lse: Optional[torch.Tensor],
+                                        stream=None) -> None:
+    """kvq.h kvq_decode_attention_static_scratch: kvq_decode_attention with the
+    library's static per-device scratch (KVQ_STATIC_SCRATCH_BYTES) instead of a
+    workspace; calls overlapping on the GPU race on that scratch."""
+    _call("kvq_decode_attention_static_scratch", C.byref(layout.c()), C.byref(cache.c()), _ptr(q),
+          _dtype_code(q), _ptr(lens), int(max_len), C.c_float(sm_scale), _ptr(out), _ptr(lse),
+          _stream(stream))
 
 
 def kvq_dequantize(layout: Layout, cache: PagedCache, lens: torch.Tensor, max_len: int,

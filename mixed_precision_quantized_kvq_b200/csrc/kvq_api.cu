@@ -4,6 +4,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "kvq_internal.cuh"
 
 namespace {
@@ -215,3 +217,50 @@ int kvq_rotate_keys(const kvq_layout* layout, const void* k, int in_dtype, int r
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode with library-held scratch: the split partials go to a static device
+// array instead of a caller workspace.  Its address is looked up once per
+// device; no allocating call is made.
+namespace {
+
+static __device__ __align__(256) unsigned char g_decode_scratch[KVQ_STATIC_SCRATCH_BYTES];
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices];   // nullptr = not looked up yet on that device
+
+int static_scratch(void** addr) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cuda_status(cudaErrorInvalidDevice);
+    if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* a = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&a, g_decode_scratch);
+        if (e != cudaSuccess || !a) return cuda_status(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+        g_scratch_addr[dev] = a;
+    }
+    *addr = g_scratch_addr[dev];
+    return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" int kvq_decode_attention_static_scratch(const kvq_layout* layout, const kvq_cache* cache,
+                                                   const void* q, int q_dtype, const int32_t* lens,
+                                                   int max_len, float sm_scale, float* out, float* lse,
+                                                   kvq_stream_t stream) {
+    int rc = check_layout(layout);
+    if (rc) return rc;
+    if ((rc = check_cache(layout, cache))) return rc;
+    if (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+    if (!q || !lens || !out || max_len < 0 || !isfinite(sm_scale)) return KVQ_ERR_INVALID_ARG;
+    if (cache->batch == 0) return KVQ_OK;
+    Params p = make_params(layout, cache);
+    kvq::DecodePlan pl = kvq::plan_decode(p, cache->batch, max_len, device_sm_count());
+    if (kvq::decode_workspace_bytes(p, cache->batch, pl) > KVQ_STATIC_SCRATCH_BYTES) return KVQ_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if ((rc = static_scratch(&scratch))) return rc;
+    return cuda_status(kvq::launch_decode(p, q, q_dtype == KVQ_BF16, lens, max_len, sm_scale, out, lse, scratch,
+                                          pl, reinterpret_cast<cudaStream_t>(stream)));
+}
