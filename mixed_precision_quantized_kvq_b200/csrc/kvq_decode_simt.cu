@@ -28,23 +28,30 @@ DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count) {
     const int units = batch * p.hkv > 0 ? batch * p.hkv : 1;
     pl.tc = (g_decode_path != 1 && tc_supported(p)) ? 1 : 0;
     if (pl.tc) {
-        // one wave of CTAs: as many splits per (sequence, kv-head) as the
-        // resident CTA slots allow, each a whole number of 128-token tiles
+        // window CTAs first (slots 0 .. nws-1, 256 window positions each),
+        // then the quantized splits, each a whole number of 128-token tiles:
+        // one wave of CTAs where the units allow it, else tiles of at most
+        // 16 per split so that ragged lengths balance across the waves
+        const int win = p.W < max_len ? p.W : max_len;
+        pl.window_split = win > 0 ? (win + 255) / 256 : 0;
         const int slots = sm_count * tc_ctas_per_sm(p);
         const int tiles = (npages + 1) / 2;
-        int want = slots / units;
-        if (want < 1) want = 1;
         if (npages == 0) {
             pl.splits_q = 0;
             pl.pages_per_split = 2;
         } else {
+            int want = slots / units;
+            if (want < 1) want = 1;
             if (want > tiles) want = tiles;
-            pl.pages_per_split = 2 * ((tiles + want - 1) / want);
+            int tps = (tiles + want - 1) / want;
+            if (units * ((tiles + tps - 1) / tps) > slots && tps > 16) tps = 16;
+            pl.pages_per_split = 2 * tps;
             if (pl.pages_per_split > 256) pl.pages_per_split = 256;   // page ids staged in shared memory
             pl.splits_q = (npages + pl.pages_per_split - 1) / pl.pages_per_split;
         }
-        pl.grid_x = pl.splits_q > 0 ? pl.splits_q : 1;
-        pl.window_slot = pl.grid_x - 1;                 // window tiles join the last split
+        pl.grid_x = pl.window_split + pl.splits_q;
+        if (pl.grid_x == 0) pl.grid_x = 1;              // all-empty: one CTA writes zeros
+        pl.window_slot = 0;
         pl.total_splits = pl.grid_x;
         return pl;
     }

@@ -1,0 +1,973 @@
+// Decode attention over the quantized cache on the 5th-generation tensor
+// cores (tcgen05, sm_100a): head_dim 128, key groups of 32 channels, value
+// groups of 128 channels, any key/value bit widths in {1, 2, 4, 8}.
+//
+// Attention ("Kuantisasi KV cache mengganggu attention ...", section "Error
+// pada key masuk sebelum softmax"): s = q K^T * sm_scale, a = softmax(s),
+// o = a V, with dequantization fused into the kernel (section "Pertumbuhan
+// cache mengubah trade pada serving").  With x^ = c*scale + zero per group:
+//   q . k^ = sum_groups ( scale * (q . c)_group + zero * (sum q)_group )
+//   o      = sum_t (p_t scale_t) c_t + sum_t p_t zero_t
+// Both contractions run on the tensor cores over the raw integer codes:
+//  - scores: kind::i8.  Key codes are exact int8 (8-bit codes offset by
+//    -128, folded into the zero point); the fp32 query of each head is split
+//    into three int8 limbs a + b/2^7 + c/2^14 times a power of two (exact to
+//    2^-20 of the head's largest element), one column per (head, key group,
+//    limb) so that the group scales apply after the product;
+//  - values: kind::f16.  Value codes are exact bf16; P' = p * value_scale is
+//    a bf16 pair (high part + remainder), accumulated in fp32 in tensor
+//    memory across the whole split.
+//
+// One CTA per (sequence, kv-head, split), 320 threads, two CTAs per SM
+// (256 tensor-memory columns each) when the GQA ratio is at most 4:
+//   warps 0-3  softmax: thread t owns token t of each 128-token tile (two
+//              pages); it prefetches the token's metadata with cp.async,
+//              turns the s32 score products into scores, keeps the running
+//              max (reused while scores stay within 2^8 of it; a larger one
+//              triggers an exact max and a rescale of the ·V accumulator)
+//              and writes P' as the B operand of the ·V MMA;
+//   warps 4-7  loaders: thread i prefetches token i's key codes and channel
+//              i's value codes with cp.async into a ring of shared-memory
+//              stages and unpacks them into tensor memory (score A operand:
+//              M = 128 tokens, K = 128 channels, int8, double buffered; ·V A
+//              operand: M = 128 channels, K = 128 tokens, bf16);
+//   warp 8     issues the score MMAs of each tile;
+//   warp 9     issues the ·V MMAs of each tile.
+// Hand-overs go through mbarriers; every wait is bounded.  The bf16 window
+// positions are handled by separate CTAs of the same grid on CUDA cores
+// (fp32), each writing its own partial.
+#pragma once
+
+#include <math.h>
+
+#include "kvq_internal.cuh"
+#include "kvq_tc_ptx.cuh"
+
+namespace kvq {
+namespace tc {
+
+using namespace ptx;
+
+constexpr int D = 128;
+constexpr int TILE = 128;                     // tokens per tile (two pages)
+constexpr int NKG = 4;                        // key groups of 32 channels
+constexpr int kThreads = 320;
+constexpr int kMaxPagesPerSplit = 256;
+constexpr int kWinPerSplit = 256;             // window positions per window CTA
+constexpr float kLazyMax = 8.0f;              // reuse the running max while scores exceed it by <= 2^8
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr unsigned FULL = 0xffffffffu;
+
+// number of bounded waits that expired (diagnostic; 0 in normal operation)
+static __device__ unsigned int g_tc_wait_timeouts;
+
+template <int KB, int VB, int NHC>
+struct Cfg {
+    static constexpr int NS = ((12 * NHC + 15) / 16) * 16;   // score columns (head, key group, limb)
+    static constexpr int NO = 16;                            // ·V columns (head, high / remainder)
+    static constexpr int COL_AK = 0;                         // 2 x 32 key operand columns (int8)
+    static constexpr int COL_AV = 64;                        // 64 value operand columns (bf16)
+    static constexpr int COL_S = 128;                        // 2 x NS score accumulators
+    static constexpr int COL_O = COL_S + 2 * NS;             // ·V accumulator
+    static constexpr int TMEM_COLS = COL_O + NO <= 256 ? 256 : 512;
+    static constexpr int KROW = D * KB / 8;                  // key row bytes of one token
+    static constexpr int VCH = kPage * VB / 8;               // value bytes of one channel in one page
+    // one ring stage: keys [chunk][token][16 B], values [chunk][channel][16 B],
+    // key meta [token][16 B], value meta [token][4 B]
+    static constexpr int ST_K = 0;
+    static constexpr int ST_V = ST_K + TILE * KROW;
+    static constexpr int ST_KM = ST_V + D * 2 * VCH;
+    static constexpr int ST_VM = ST_KM + TILE * 16;
+    static constexpr int STAGE = ST_VM + TILE * 4;
+    static constexpr int CS_Q = NS * 16 + 16;                // chunk stride of the query operand
+    static constexpr int CS_P = 16 * 16 + 16;                // chunk stride of the P' operand
+    static_assert(2 * NHC <= NO, "two ·V columns per head");
+};
+
+struct Shared {
+    uint64_t kfull[2];       // loaders -> score MMA: key operand written
+    uint64_t sfull[2];       // score MMA -> softmax: accumulator ready (and key operand free)
+    uint64_t sfree[2];       // softmax -> score MMA: accumulator read
+    uint64_t vfull;          // loaders -> ·V MMA: value operand written
+    uint64_t pfull[2];       // softmax -> ·V MMA: P' operand written
+    uint64_t pvdone[2];      // ·V MMA -> softmax, loaders: product of the tile done
+    uint64_t mma_done[2];
+    uint32_t tmem_base;
+    int abort;
+    int vote[2][4];
+    int smax[2][4][kMaxGqa];             // per warp: max score (ordered int) per head
+    float red[4][kMaxGqa], red2[4][kMaxGqa];
+    alignas(16) float qsum[kMaxGqa][NKG];   // sums of the rotated query per key group
+    float qs0[kMaxGqa];                  // query limb unit: 2^-14 of the head's s0
+    alignas(16) float qf[kMaxGqa][D];    // query, fp32, as given
+    alignas(16) float qr[kMaxGqa][D];    // query rotated like the stored keys
+    alignas(16) float wsc[kMaxGqa][TILE];   // window CTAs: scores / weights of a chunk
+    float wred[8][kMaxGqa];
+    int pages[kMaxPagesPerSplit];
+};
+
+// Shared-memory plan: Shared, the query operand, two P' buffers, then a
+// ring of R stages.  Two CTAs share an SM when the tensor memory allows it
+// and three stages still fit in half the shared memory; otherwise one.
+constexpr int kSmemPerSm = 228 * 1024;         // shared memory of an SM (reservations excluded below)
+constexpr int ring_offset(int ns) {
+    return (((((int(sizeof(Shared)) + 127) & ~127) + 8 * (ns * 16 + 16) + 2 * 16 * (16 * 16 + 16)) + 127) & ~127);
+}
+constexpr int stage_bytes(int kb, int vb) { return TILE * (D * kb / 8) + D * 2 * (kPage * vb / 8) + TILE * 16 + TILE * 4; }
+constexpr int ns_cols(int nhc) { return ((12 * nhc + 15) / 16) * 16; }
+constexpr int ctas_per_sm(int kb, int vb, int nhc) {
+    return (128 + 2 * ns_cols(nhc) + 16 <= 256 && (112 * 1024 - ring_offset(ns_cols(nhc))) / stage_bytes(kb, vb) >= 3) ? 2
+                                                                                                                      : 1;
+}
+
+template <int KB, int VB, int NHC>
+struct Layout {
+    using C = Cfg<KB, VB, NHC>;
+    static constexpr int CTAS = ctas_per_sm(KB, VB, NHC);
+    static constexpr int OFF_QB = (int(sizeof(Shared)) + 127) & ~127;
+    static constexpr int OFF_PB = OFF_QB + 8 * C::CS_Q;
+    static constexpr int OFF_RING = (OFF_PB + 2 * 16 * C::CS_P + 127) & ~127;
+    static constexpr int BUDGET = CTAS == 2 ? 112 * 1024 : 224 * 1024;
+    static constexpr int R0 = (BUDGET - OFF_RING) / C::STAGE;
+    static constexpr int R = R0 > 8 ? 8 : R0;                 // ring stages
+    static constexpr int USED = OFF_RING + R * C::STAGE;
+    // never more CTAs per SM than planned (the tensor memory holds no more)
+    static constexpr int MIN_TOTAL = CTAS == 2 ? 80 * 1024 : 120 * 1024;
+    static constexpr int TOTAL = USED > MIN_TOTAL ? USED : MIN_TOTAL;
+    static_assert(R >= 3, "ring needs three stages");
+    static_assert(OFF_RING == ring_offset(C::NS) && C::STAGE == stage_bytes(KB, VB), "plan formulas agree");
+    static_assert(OFF_RING + 4 * D * kMaxGqa * 4 <= TOTAL, "window reduction buffer fits the ring");
+};
+
+// ---------------------------------------------------------------- helpers
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ float ex2(float x) {   // 2^x, hardware approximation (flushes subnormals)
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+    return v;
+}
+__device__ __forceinline__ uint32_t redux_max_u32(uint32_t v) {
+    uint32_t r;
+    asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
+    return r;
+}
+__device__ __forceinline__ int redux_max_s32(int v) {
+    int r;
+    asm volatile("redux.sync.max.s32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
+    return r;
+}
+// order-preserving map of floats onto signed integers, and back
+__device__ __forceinline__ int ord_key(float x) {
+    const int b = __float_as_int(x);
+    return b ^ ((b >> 31) & 0x7FFFFFFF);
+}
+__device__ __forceinline__ float ord_val(int k) { return __int_as_float(k ^ ((k >> 31) & 0x7FFFFFFF)); }
+__device__ __forceinline__ int rni(float x) {
+    int r;
+    asm("cvt.rni.s32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// cp.async: 16 / 8 / 4 bytes global -> shared; src_bytes 0 fills zeros
+__device__ __forceinline__ void cp16(void* dst, const void* src, bool have) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(have ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp8(void* dst, const void* src, bool have) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(have ? 8 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp4(void* dst, const void* src, bool have) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(have ? 4 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// kind::i8 MMA, A from tensor memory, issued by one elected lane of a warp
+__device__ __forceinline__ void mma_i8_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+        : "memory");
+}
+// instruction descriptor: signed int8 A and B (K-major), s32 accumulator
+__host__ __device__ constexpr uint32_t idesc_s8(int M, int N) {
+    return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- unpacking
+// A 32-bit word of b-bit codes -> 8/b words of int8 codes: word s holds, in
+// byte k, the code of element k*(8/b) + s.  So K position 4*s + k of the
+// word's run carries element k*(8/b) + s; 8-bit codes are offset by -128.
+template <int B>
+__device__ __forceinline__ void unpack_i8(uint32_t w, uint32_t* o) {
+    if constexpr (B == 8) {
+        o[0] = w ^ 0x80808080u;
+    } else {
+        constexpr uint32_t M = B == 4 ? 0x0F0F0F0Fu : B == 2 ? 0x03030303u : 0x01010101u;
+#pragma unroll
+        for (int s = 0; s < 8 / B; ++s) o[s] = (w >> (B * s)) & M;
+    }
+}
+// K position (within a run of 32/b-element words) of element e
+__host__ __device__ __forceinline__ int kpos_of(int e, int bits) {
+    const int per = 32 / bits, f = 8 / bits;
+    const int w = e / per, r = e % per;
+    return w * per + 4 * (r % f) + r / f;
+}
+// byte offset of (row n, K position kp) in a K-major int8 B operand stored as
+// [16-byte K chunk][row][16 bytes] with chunk stride cs
+__device__ __forceinline__ int b_off(int n, int kp, int cs) { return (kp >> 4) * cs + n * 16 + (kp & 15); }
+
+// the bf16 bits of a pair, as floats
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// ------------------------------------------------- value codes -> bf16
+// A 32-bit word of b-bit codes becomes 16/b bf16x2 registers; register k
+// holds codes (k, k + 16/b): low half the first.  Codes are exact small
+// integers: bits are placed into the mantissa of bf16 128.0 (0x4300), the
+// offset (and a power-of-two position scale) removed with one exact fma.
+// bf16 bit patterns (both halves) of 2^-S and -128 * 2^-S
+template <int S>
+struct FixConst;
+template <> struct FixConst<0> { static constexpr uint32_t mul = 0x3F803F80u, add = 0xC300C300u; };
+template <> struct FixConst<1> { static constexpr uint32_t mul = 0x3F003F00u, add = 0xC280C280u; };
+template <> struct FixConst<2> { static constexpr uint32_t mul = 0x3E803E80u, add = 0xC200C200u; };
+template <> struct FixConst<3> { static constexpr uint32_t mul = 0x3E003E00u, add = 0xC180C180u; };
+template <> struct FixConst<4> { static constexpr uint32_t mul = 0x3D803D80u, add = 0xC100C100u; };
+template <> struct FixConst<5> { static constexpr uint32_t mul = 0x3D003D00u, add = 0xC080C080u; };
+template <> struct FixConst<6> { static constexpr uint32_t mul = 0x3C803C80u, add = 0xC000C000u; };
+
+template <int S>
+__device__ __forceinline__ uint32_t fix_bf16(uint32_t x) {
+    uint32_t r;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(x), "r"(FixConst<S>::mul), "r"(FixConst<S>::add));
+    return r;
+}
+
+constexpr uint32_t kMagic = 0x43004300u;
+
+template <int B>
+struct Unpack;
+
+template <>
+struct Unpack<4> {
+    __device__ static __forceinline__ void word(uint32_t w, uint32_t* o) {
+        o[0] = fix_bf16<0>((w & 0x000F000Fu) | kMagic);
+        o[1] = fix_bf16<3>(((w >> 1) & 0x00780078u) | kMagic);
+        o[2] = fix_bf16<3>(((w >> 5) & 0x00780078u) | kMagic);
+        o[3] = fix_bf16<3>(((w >> 9) & 0x00780078u) | kMagic);
+    }
+};
+template <>
+struct Unpack<2> {
+    __device__ static __forceinline__ void word(uint32_t w, uint32_t* o) {
+        o[0] = fix_bf16<0>((w & 0x00030003u) | kMagic);
+        o[1] = fix_bf16<2>((w & 0x000C000Cu) | kMagic);
+        o[2] = fix_bf16<4>((w & 0x00300030u) | kMagic);
+        const uint32_t w6 = w >> 6;
+        o[3] = fix_bf16<0>((w6 & 0x00030003u) | kMagic);
+        o[4] = fix_bf16<2>((w6 & 0x000C000Cu) | kMagic);
+        o[5] = fix_bf16<4>((w6 & 0x00300030u) | kMagic);
+        const uint32_t w12 = w >> 12;
+        o[6] = fix_bf16<0>((w12 & 0x00030003u) | kMagic);
+        o[7] = fix_bf16<2>((w12 & 0x000C000Cu) | kMagic);
+    }
+};
+template <>
+struct Unpack<1> {
+    __device__ static __forceinline__ void word(uint32_t w, uint32_t* o) {
+        o[0] = fix_bf16<0>((w & 0x00010001u) | kMagic);
+        o[1] = fix_bf16<1>((w & 0x00020002u) | kMagic);
+        o[2] = fix_bf16<2>((w & 0x00040004u) | kMagic);
+        o[3] = fix_bf16<3>((w & 0x00080008u) | kMagic);
+        o[4] = fix_bf16<4>((w & 0x00100010u) | kMagic);
+        o[5] = fix_bf16<5>((w & 0x00200020u) | kMagic);
+        o[6] = fix_bf16<6>((w & 0x00400040u) | kMagic);
+        const uint32_t w7 = w >> 7;
+        o[7] = fix_bf16<0>((w7 & 0x00010001u) | kMagic);
+        o[8] = fix_bf16<1>((w7 & 0x00020002u) | kMagic);
+        o[9] = fix_bf16<2>((w7 & 0x00040004u) | kMagic);
+        o[10] = fix_bf16<3>((w7 & 0x00080008u) | kMagic);
+        o[11] = fix_bf16<4>((w7 & 0x00100010u) | kMagic);
+        o[12] = fix_bf16<5>((w7 & 0x00200020u) | kMagic);
+        o[13] = fix_bf16<6>((w7 & 0x00400040u) | kMagic);
+        const uint32_t w14 = w >> 14;
+        o[14] = fix_bf16<0>((w14 & 0x00010001u) | kMagic);
+        o[15] = fix_bf16<1>((w14 & 0x00020002u) | kMagic);
+    }
+};
+template <>
+struct Unpack<8> {
+    __device__ static __forceinline__ float byte_f(uint32_t w, uint32_t sel) {
+        // float with mantissa = the selected byte, exponent of 2^23; minus 2^23
+        return __uint_as_float(__byte_perm(w, 0x4B000000u, sel)) - 8388608.0f;
+    }
+    __device__ static __forceinline__ void word(uint32_t w, uint32_t* o) {
+        __nv_bfloat162 a = __floats2bfloat162_rn(byte_f(w, 0x7440u), byte_f(w, 0x7442u));
+        __nv_bfloat162 b = __floats2bfloat162_rn(byte_f(w, 0x7441u), byte_f(w, 0x7443u));
+        o[0] = *reinterpret_cast<uint32_t*>(&a);
+        o[1] = *reinterpret_cast<uint32_t*>(&b);
+    }
+};
+
+// position (along the MMA K dimension) of element i of a packed run, and
+// the element at a K position: inverse permutations of the unpack order
+__host__ __device__ __forceinline__ int kpos_bf16(int i, int bits) {
+    const int per = 32 / bits, half = per / 2;
+    const int w = i / per, r = i % per;
+    return w * per + 2 * (r % half) + r / half;
+}
+__host__ __device__ __forceinline__ int elem_at_bf16(int pos, int bits) {
+    const int per = 32 / bits, half = per / 2;
+    const int w = pos / per, r = pos % per;
+    return w * per + (r >> 1) + (r & 1) * half;
+}
+// byte offset of element (row n, K position pos) in a K-major B operand
+// stored as [k step][half][row][8 x bf16] with chunk stride cs
+__device__ __forceinline__ int b_off_bf16(int n, int pos, int cs) {
+    return ((pos >> 4) * 2 + ((pos >> 3) & 1)) * cs + n * 16 + (pos & 7) * 2;
+}
+
+
+__device__ __forceinline__ uint16_t bf16_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+
+template <int N>
+__device__ __forceinline__ void cp_wait_n() {
+    if constexpr (N <= 0) cp_wait<0>();
+    else cp_wait<N>();
+}
+
+static __device__ void write_empty_partial(int g, float* ws_o, float* ws_ml, size_t row0, int slots, int slot) {
+    for (int i = threadIdx.x; i < g * D; i += blockDim.x) {
+        const int r = i / D;
+        ws_o[(row0 + size_t(r) * slots + slot) * D + (i % D)] = 0.0f;
+        if (i % D == 0) {
+            ws_ml[(row0 + size_t(r) * slots + slot) * 2 + 0] = -INFINITY;
+            ws_ml[(row0 + size_t(r) * slots + slot) * 2 + 1] = 0.0f;
+        }
+    }
+}
+
+// --------------------------------------------------------- window partial
+// CUDA-core attention over window positions [w0, w1) (bf16 keys and values,
+// unrotated query), chunks of 128 positions with an online softmax.  256
+// threads (warps 0-7); every phase issues all of its loads before using them.
+//   scores:  thread pair (2t, 2t+1) splits position t's 128 channels;
+//   ·V:      thread (jp, tq) owns channels 2jp, 2jp+1 and positions tq mod 4;
+//            the four position classes are summed through shared memory.
+static __device__ void window_partial(const Params& p, Shared& sh, float* scratch, int b, int h, int w0, int w1,
+                                      float scale_log2, float* ws_o, float* ws_ml, size_t row0, int slots,
+                                      int slot) {
+    const int g = p.g, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (warp >= 8) return;
+    const int t = tid >> 1, hf = tid & 1;          // scores: position t of the chunk, channel half hf
+    const int jp = tid & 63, tq = tid >> 6;        // ·V: channel pair, position class
+    float m[kMaxGqa], l[kMaxGqa], o0[kMaxGqa], o1[kMaxGqa];
+#pragma unroll
+    for (int r = 0; r < kMaxGqa; ++r) {
+        m[r] = -INFINITY;
+        l[r] = 0.0f;
+        o0[r] = 0.0f;
+        o1[r] = 0.0f;
+    }
+    const size_t hb = (size_t(b) * p.hkv + h) * size_t(p.W);
+    for (int c0 = w0; c0 < w1; c0 += TILE) {
+        const int n = min(TILE, w1 - c0);
+        float s[kMaxGqa];
+        {
+            uint4 kv4[8];
+            const bool in = t < n;
+            int sl = c0 - w0 + t;                       // ring slot of position c0 + t
+            sl = (w0 + sl) % p.W;
+            const uint4* kr = reinterpret_cast<const uint4*>(p.k_win + (hb + size_t(sl)) * D + 64 * hf);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) kv4[c] = in ? __ldg(kr + c) : make_uint4(0, 0, 0, 0);
+            float acc[kMaxGqa];
+#pragma unroll
+            for (int r = 0; r < kMaxGqa; ++r) acc[r] = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float kv[8] = {bf_lo(kv4[c].x), bf_hi(kv4[c].x), bf_lo(kv4[c].y), bf_hi(kv4[c].y),
+                                     bf_lo(kv4[c].z), bf_hi(kv4[c].z), bf_lo(kv4[c].w), bf_hi(kv4[c].w)};
+#pragma unroll
+                for (int r = 0; r < kMaxGqa; ++r) {
+                    if (r < g) {
+                        const float4 qa = *reinterpret_cast<const float4*>(&sh.qf[r][64 * hf + 8 * c]);
+                        const float4 qb = *reinterpret_cast<const float4*>(&sh.qf[r][64 * hf + 8 * c + 4]);
+                        acc[r] = fmaf(qa.x, kv[0], acc[r]);
+                        acc[r] = fmaf(qa.y, kv[1], acc[r]);
+                        acc[r] = fmaf(qa.z, kv[2], acc[r]);
+                        acc[r] = fmaf(qa.w, kv[3], acc[r]);
+                        acc[r] = fmaf(qb.x, kv[4], acc[r]);
+                        acc[r] = fmaf(qb.y, kv[5], acc[r]);
+                        acc[r] = fmaf(qb.z, kv[6], acc[r]);
+                        acc[r] = fmaf(qb.w, kv[7], acc[r]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < kMaxGqa; ++r) {
+                const float tot = acc[r] + __shfl_xor_sync(FULL, acc[r], 1);
+                s[r] = (in && r < g) ? tot * scale_log2 : -INFINITY;
+                const float wm = warp_max(s[r]);
+                if (lane == 0 && r < g) sh.wred[warp][r] = wm;
+            }
+        }
+        named_sync(2, 256);
+        float mnew[kMaxGqa], alpha[kMaxGqa];
+#pragma unroll
+        for (int r = 0; r < kMaxGqa; ++r) {
+            mnew[r] = m[r];
+            alpha[r] = 1.0f;
+            if (r < g) {
+                float cm = sh.wred[0][r];
+#pragma unroll
+                for (int w = 1; w < 8; ++w) cm = fmaxf(cm, sh.wred[w][r]);
+                mnew[r] = fmaxf(m[r], cm);
+                alpha[r] = (mnew[r] == -INFINITY) ? 1.0f : ex2(m[r] - mnew[r]);
+                m[r] = mnew[r];
+                const float pr = (s[r] == -INFINITY) ? 0.0f : ex2(s[r] - mnew[r]);
+                l[r] = fmaf(l[r], alpha[r], hf == 0 ? pr : 0.0f);
+                if (hf == 0) sh.wsc[r][t] = pr;
+                o0[r] *= alpha[r];
+                o1[r] *= alpha[r];
+            }
+        }
+        named_sync(2, 256);
+        {
+            uint32_t vv[TILE / 4];
+            const __nv_bfloat16* vc = p.v_win + hb * D + 2 * jp;
+#pragma unroll
+            for (int k = 0; k < TILE / 4; ++k) {
+                const int tt = tq + 4 * k;
+                const int sl = (c0 + tt) % p.W;
+                vv[k] = tt < n ? __ldg(reinterpret_cast<const uint32_t*>(vc + size_t(sl) * D)) : 0u;
+            }
+#pragma unroll
+            for (int k = 0; k < TILE / 4; ++k) {
+                const int tt = tq + 4 * k;
+                const float va = bf_lo(vv[k]), vb = bf_hi(vv[k]);
+#pragma unroll
+                for (int r = 0; r < kMaxGqa; ++r) {
+                    if (r < g) {
+                        const float pr = tt < n ? sh.wsc[r][tt] : 0.0f;
+                        o0[r] = fmaf(pr, va, o0[r]);
+                        o1[r] = fmaf(pr, vb, o1[r]);
+                    }
+                }
+            }
+        }
+        named_sync(2, 256);                         // wsc and wred are rewritten by the next chunk
+    }
+    // position classes -> channel sums; l over the score threads
+#pragma unroll
+    for (int r = 0; r < kMaxGqa; ++r) {
+        if (r < g) {
+            scratch[(tq * kMaxGqa + r) * D + 2 * jp] = o0[r];
+            scratch[(tq * kMaxGqa + r) * D + 2 * jp + 1] = o1[r];
+        }
+        const float ls = warp_sum(l[r]);
+        if (lane == 0 && r < g) sh.wred[warp][r] = ls;
+    }
+    named_sync(2, 256);
+    if (tid < D) {
+        const int j = tid;
+#pragma unroll
+        for (int r = 0; r < kMaxGqa; ++r) {
+            if (r >= g) continue;
+            const float v = (scratch[(0 * kMaxGqa + r) * D + j] + scratch[(1 * kMaxGqa + r) * D + j]) +
+                            (scratch[(2 * kMaxGqa + r) * D + j] + scratch[(3 * kMaxGqa + r) * D + j]);
+            const size_t row = row0 + size_t(r) * slots + slot;
+            ws_o[row * D + j] = v;
+            if (j == 0) {
+                float ls = 0.0f;
+#pragma unroll
+                for (int w = 0; w < 8; ++w) ls += sh.wred[w][r];
+                ws_ml[row * 2 + 0] = m[r];
+                ws_ml[row * 2 + 1] = ls;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ kernel
+// grid (nws + splits_q, Hkv, B).  blockIdx.x < nws: window CTA covering
+// window positions [Lq + x*256, Lq + (x+1)*256); otherwise quantized split
+// x - nws covering pages [s*pps, (s+1)*pps).  Every CTA writes one partial
+// (m, l, o) per query head into slot blockIdx.x.
+template <int KB, int VB, int NHC>
+__global__ void __launch_bounds__(kThreads, ctas_per_sm(KB, VB, NHC))
+decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, const int32_t* __restrict__ lens,
+                 const int max_len, const float scale_log2, float* __restrict__ ws_o, float* __restrict__ ws_ml,
+                 const int pps, const int nws, const int slots) {
+    using C = Cfg<KB, VB, NHC>;
+    using LY = Layout<KB, VB, NHC>;
+    constexpr int R = LY::R;
+    constexpr int NS = C::NS;
+    constexpr uint32_t IDESC_S = idesc_s8(128, NS);
+    constexpr uint32_t IDESC_O = idesc_bf16_f32(128, C::NO);
+    constexpr int VWP = kPage * VB / 32;     // value words per channel per page
+    constexpr int VREG = 16 / VB;            // bf16x2 registers per value word
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    Shared& sh = *reinterpret_cast<Shared*>(smem);
+    uint8_t* qb = smem + LY::OFF_QB;
+    uint8_t* pb = smem + LY::OFF_PB;
+    uint8_t* ring = smem + LY::OFF_RING;
+
+    const int b = blockIdx.z, h = blockIdx.y, x = blockIdx.x;
+    const int g = p.g, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int L = max(0, min(lens[b], max_len));
+    const int Lq = max(0, L - p.W);
+    const size_t row0 = (size_t(b) * p.hq + size_t(h) * g) * slots;
+
+    // ---- which work this CTA has
+    const bool is_win = x < nws;
+    int w0 = 0, w1 = 0, pg0 = 0, pg1 = 0, ntiles = 0;
+    if (is_win) {
+        w0 = Lq + x * kWinPerSplit;
+        w1 = min(L, w0 + kWinPerSplit);
+    } else {
+        const int npg = (Lq + kPage - 1) / kPage;
+        pg0 = (x - nws) * pps;
+        pg1 = min(npg, pg0 + pps);
+        ntiles = pg1 > pg0 ? (pg1 - pg0 + 1) / 2 : 0;
+    }
+    if ((is_win && w0 >= w1) || (!is_win && ntiles == 0)) {
+        write_empty_partial(g, ws_o, ws_ml, row0, slots, x);
+        return;
+    }
+
+    // ---- query (fp32; rotated copy for the quantized keys)
+    for (int i = tid; i < g * D; i += kThreads) {
+        const size_t off = (size_t(b) * p.hq + size_t(h) * g + i / D) * D + (i % D);
+        sh.qf[i / D][i % D] = q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(q)[off])
+                                     : reinterpret_cast<const float*>(q)[off];
+    }
+    __syncthreads();
+    if (is_win) {
+        window_partial(p, sh, reinterpret_cast<float*>(ring), b, h, w0, w1, scale_log2, ws_o, ws_ml, row0, slots,
+                       x);
+        __syncthreads();
+        return;
+    }
+
+    if (tid == 0) {
+        for (int u = 0; u < 2; ++u) {
+            mbar_init(&sh.kfull[u], 4);
+            mbar_init(&sh.sfull[u], 1);
+            mbar_init(&sh.sfree[u], 4);
+            mbar_init(&sh.pfull[u], 4);
+            mbar_init(&sh.pvdone[u], 1);
+            mbar_init(&sh.mma_done[u], 1);
+        }
+        mbar_init(&sh.vfull, 4);
+        mbar_fence_init();
+        sh.abort = 0;
+    }
+    if (warp == 8) {
+        tmem_alloc(&sh.tmem_base, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    for (int i = tid; i < pg1 - pg0; i += kThreads) sh.pages[i] = phys_page(p, b, pg0 + i);
+    for (int i = tid; i < 8 * C::CS_Q / 4; i += kThreads) reinterpret_cast<uint32_t*>(qb)[i] = 0u;
+    for (int i = tid; i < 2 * 16 * C::CS_P / 4; i += kThreads) reinterpret_cast<uint32_t*>(pb)[i] = 0u;
+    __syncthreads();
+    // query operand: row n = 12r + 3grp + l (head r, key group grp, limb l),
+    // K position of channel j in the int8 key operand; zeros outside the group.
+    // One warp per head; lane owns channels 4*lane .. 4*lane+3.
+    for (int r = warp; r < g; r += kThreads / 32) {
+        float xr[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) xr[c] = sh.qf[r][lane * 4 + c];
+        if (p.rotate) rotate_warp<D>(xr, p.signs, lane);
+        float amax = fmaxf(fmaxf(fabsf(xr[0]), fabsf(xr[1])), fmaxf(fabsf(xr[2]), fabsf(xr[3])));
+        amax = warp_max(amax);
+        float gs = (xr[0] + xr[1]) + (xr[2] + xr[3]);
+        gs += __shfl_xor_sync(FULL, gs, 1);
+        gs += __shfl_xor_sync(FULL, gs, 2);
+        gs += __shfl_xor_sync(FULL, gs, 4);                   // lanes 8grp .. 8grp+7 = key group grp
+        if ((lane & 7) == 0) sh.qsum[r][lane >> 3] = gs;
+        const uint32_t eb = __float_as_uint(amax) >> 23;      // biased exponent: amax < 2^(eb-126)
+        const bool use = eb >= 40;
+        const float inv_s0 = use ? __uint_as_float((259u - eb) << 23) : 0.0f;   // 2^(132-eb) = 1/s0
+        if (lane == 0) sh.qs0[r] = use ? __uint_as_float((eb - 19u) << 23) : 0.0f;   // s0 * 2^-14
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int j = lane * 4 + c, grp = j >> 5, kp = kpos_of(j, KB);
+            const float xs = xr[c] * inv_s0;                   // |xs| < 64, exact
+            const int a = rni(xs);
+            const float r1 = (xs - (float)a) * 128.0f;
+            const int bl = rni(r1);
+            const float r2 = (r1 - (float)bl) * 128.0f;
+            const int cl = rni(r2);
+            const int n0 = 12 * r + 3 * grp;
+            qb[b_off(n0 + 0, kp, C::CS_Q)] = (uint8_t)(int8_t)a;
+            qb[b_off(n0 + 1, kp, C::CS_Q)] = (uint8_t)(int8_t)bl;
+            qb[b_off(n0 + 2, kp, C::CS_Q)] = (uint8_t)(int8_t)cl;
+        }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = sh.tmem_base;
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;     // this warp's tensor-memory lanes
+    bool ok = true;
+    auto wait = [&](uint64_t* bar, uint32_t parity) {
+        if (!ok || sh.abort) {
+            ok = false;
+            return;
+        }
+        if (!mbar_wait(bar, parity, kWaitNs)) {
+            ok = false;
+            sh.abort = 1;
+        }
+    };
+
+    if (warp == 8) {
+        // ======================================================== score MMA
+        const uint64_t qd = smem_desc(smem_u32(qb), C::CS_Q, 128);
+        for (int i = 0; i < ntiles; ++i) {
+            const int u = i & 1;
+            wait(&sh.kfull[u], (i >> 1) & 1);
+            if (i >= 2) wait(&sh.sfree[u], ((i - 2) >> 1) & 1);
+            if (__any_sync(FULL, !ok)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                mma_i8_warp(tbase + C::COL_S + NS * u, tbase + C::COL_AK + 32 * u + 8 * k,
+                            qd + uint64_t((k * 2 * C::CS_Q) >> 4), IDESC_S, k > 0 ? 1u : 0u);
+            tc_commit_warp(&sh.sfull[u]);
+        }
+        tc_commit_warp(&sh.mma_done[0]);          // every MMA above has completed before the teardown
+        mbar_wait(&sh.mma_done[0], 0, kWaitNs);
+    } else if (warp == 9) {
+        // =========================================================== ·V MMA
+        const uint32_t pb_s = smem_u32(pb);
+        for (int j = 0; j < ntiles; ++j) {
+            const int u = j & 1;
+            wait(&sh.vfull, j & 1);
+            wait(&sh.pfull[u], (j >> 1) & 1);
+            if (__any_sync(FULL, !ok)) break;
+            tc_fence_after();
+            const uint64_t pd = smem_desc(pb_s + u * 16 * C::CS_P, C::CS_P, 128);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                tc_mma_ts_warp(tbase + C::COL_O, tbase + C::COL_AV + 8 * k, pd + uint64_t((k * 2 * C::CS_P) >> 4),
+                               IDESC_O, (j > 0 || k > 0) ? 1u : 0u);
+            tc_commit_warp(&sh.pvdone[u]);
+        }
+        tc_commit_warp(&sh.mma_done[1]);
+        mbar_wait(&sh.mma_done[1], 0, kWaitNs);
+    } else if (warp >= 4) {
+        // =========================================================== loaders
+        const int ti = tid - 128;                 // token ti (keys) and channel ti (values)
+        const int pp_k = ti >> 6, slot_k = ti & 63;
+        auto issue = [&](int i) {
+            uint8_t* st = ring + (i % R) * C::STAGE;
+            {   // key codes of token ti
+                const int lp = pg0 + 2 * i + pp_k;
+                const int pg = lp < pg1 ? sh.pages[2 * i + pp_k] : -1;
+                const bool have = pg >= 0;
+                const uint8_t* kb = p.k_codes + (size_t(have ? pg : 0) * p.hkv + h) * (kPage * C::KROW) + slot_k * 16;
+#pragma unroll
+                for (int c = 0; c < C::KROW / 16; ++c)
+                    cp16(st + C::ST_K + c * (TILE * 16) + ti * 16, kb + c * (kPage * 16), have);
+            }
+#pragma unroll
+            for (int pp = 0; pp < 2; ++pp) {      // value codes of channel ti, both pages
+                const int lp = pg0 + 2 * i + pp;
+                const int pg = lp < pg1 ? sh.pages[2 * i + pp] : -1;
+                const bool have = pg >= 0;
+                const uint8_t* vb = p.v_codes + (size_t(have ? pg : 0) * p.hkv + h) * (D * C::VCH);
+                if constexpr (C::VCH >= 16) {
+#pragma unroll
+                    for (int c = 0; c < C::VCH / 16; ++c)
+                        cp16(st + C::ST_V + (pp * (C::VCH / 16) + c) * (D * 16) + ti * 16, vb + c * (D * 16) + ti * 16,
+                             have);
+                } else {
+                    cp8(st + C::ST_V + ti * 16 + pp * 8, vb + ti * 8, have);
+                }
+            }
+        };
+        auto keys = [&](int i) {                  // key codes of tile i -> int8 operand buffer i&1
+            const uint8_t* st = ring + (i % R) * C::STAGE;
+            uint32_t a[32];
+#pragma unroll
+            for (int c = 0; c < C::KROW / 16; ++c) {
+                const uint4 w4 = *reinterpret_cast<const uint4*>(st + C::ST_K + c * (TILE * 16) + ti * 16);
+                unpack_i8<KB>(w4.x, &a[(4 * c + 0) * (8 / KB)]);
+                unpack_i8<KB>(w4.y, &a[(4 * c + 1) * (8 / KB)]);
+                unpack_i8<KB>(w4.z, &a[(4 * c + 2) * (8 / KB)]);
+                unpack_i8<KB>(w4.w, &a[(4 * c + 3) * (8 / KB)]);
+            }
+            if (i >= 2) wait(&sh.sfull[i & 1], ((i - 2) >> 1) & 1);   // score MMA of tile i-2 read the buffer
+            tc_fence_after();
+            tmem_st32(tbase + lane_off + C::COL_AK + 32 * (i & 1), a);
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.kfull[i & 1]);
+        };
+        auto values = [&](int i) {                // value codes of tile i -> bf16 operand
+            const uint8_t* st = ring + (i % R) * C::STAGE + C::ST_V;
+            uint32_t a[64];
+#pragma unroll
+            for (int pp = 0; pp < 2; ++pp) {
+                if constexpr (VB == 1) {
+                    const uint2 w2 = *reinterpret_cast<const uint2*>(st + ti * 16 + pp * 8);
+                    Unpack<1>::word(w2.x, &a[pp * 32]);
+                    Unpack<1>::word(w2.y, &a[pp * 32 + VREG]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < VWP / 4; ++c) {
+                        const uint4 w4 = *reinterpret_cast<const uint4*>(st + (pp * (VWP / 4) + c) * (D * 16) + ti * 16);
+                        Unpack<VB>::word(w4.x, &a[pp * 32 + c * 4 * VREG + 0 * VREG]);
+                        Unpack<VB>::word(w4.y, &a[pp * 32 + c * 4 * VREG + 1 * VREG]);
+                        Unpack<VB>::word(w4.z, &a[pp * 32 + c * 4 * VREG + 2 * VREG]);
+                        Unpack<VB>::word(w4.w, &a[pp * 32 + c * 4 * VREG + 3 * VREG]);
+                    }
+                }
+            }
+            if (i >= 1) wait(&sh.pvdone[(i - 1) & 1], ((i - 1) >> 1) & 1);   // ·V MMA of tile i-1 read the operand
+            tc_fence_after();
+            tmem_st32(tbase + lane_off + C::COL_AV, a);
+            tmem_st32(tbase + lane_off + C::COL_AV + 32, a + 32);
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.vfull);
+        };
+        // keys run one tile ahead of values: iteration i unpacks keys of
+        // tile i+1 and values of tile i (ring slots of tiles i .. i+R-1 live)
+        for (int i = 0; i < R - 1; ++i) {
+            if (i < ntiles) issue(i);
+            cp_commit();
+        }
+        cp_wait_n<R - 2>();
+        keys(0);
+        for (int i = 0; i < ntiles; ++i) {
+            if (__any_sync(FULL, !ok)) break;
+            if (i + R - 1 < ntiles) issue(i + R - 1);
+            cp_commit();
+            cp_wait_n<R - 2>();                   // tiles i and i+1 landed
+            if (i + 1 < ntiles) keys(i + 1);
+            values(i);
+        }
+        cp_wait_all();
+    } else {
+        // =========================================================== softmax
+        const int t = tid, pp_t = t >> 6, slot_t = t & 63;
+        const int kpos_t = pp_t * kPage + kpos_bf16(slot_t, VB);   // position along the ·V K dimension
+        auto issue = [&](int i) {
+            uint8_t* st = ring + (i % R) * C::STAGE;
+            const int lp = pg0 + 2 * i + pp_t;
+            const int pg = lp < pg1 ? sh.pages[2 * i + pp_t] : -1;
+            const bool have = pg >= 0;
+            const size_t ph = size_t(have ? pg : 0) * p.hkv + h;
+            cp16(st + C::ST_KM + t * 16, p.k_meta + (ph * kPage + slot_t) * NKG, have);
+            cp4(st + C::ST_VM + t * 4, p.v_meta + (ph * kPage + slot_t), have);
+        };
+        for (int i = 0; i < R - 1; ++i) {
+            if (i < ntiles) issue(i);
+            cp_commit();
+        }
+        float qsum[NHC][NKG], qs0[NHC];
+#pragma unroll
+        for (int r = 0; r < NHC; ++r) {
+            qs0[r] = sh.qs0[r < g ? r : 0];
+#pragma unroll
+            for (int grp = 0; grp < NKG; ++grp) qsum[r][grp] = sh.qsum[r < g ? r : 0][grp];
+        }
+        float m[NHC], l[NHC], pz[NHC];
+#pragma unroll
+        for (int r = 0; r < NHC; ++r) {
+            m[r] = -INFINITY;
+            l[r] = 0.0f;
+            pz[r] = 0.0f;
+        }
+        for (int j = 0; j < ntiles; ++j) {
+            const int u = j & 1;
+            if (j + R - 1 < ntiles) issue(j + R - 1);
+            cp_commit();
+            cp_wait<R - 1>();
+            const uint8_t* st = ring + (j % R) * C::STAGE;
+            const uint4 km4 = *reinterpret_cast<const uint4*>(st + C::ST_KM + t * 16);
+            const uint32_t vmw = *reinterpret_cast<const uint32_t*>(st + C::ST_VM + t * 4);
+            const int lp = pg0 + 2 * j + pp_t;
+            const bool valid = lp < pg1 && sh.pages[2 * j + pp_t] >= 0 && lp * kPage + slot_t < Lq;
+            // ---- s32 score products of token t
+            wait(&sh.sfull[u], (j >> 1) & 1);
+            tc_fence_after();
+            uint32_t ds[NS];
+#pragma unroll
+            for (int c = 0; c < NS / 16; ++c)
+                tmem_ld16(tbase + lane_off + C::COL_S + NS * u + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(&ds[16 * c]));
+            tc_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.sfree[u]);
+            const uint32_t kmw[NKG] = {km4.x, km4.y, km4.z, km4.w};
+            float ksc[NKG], kzp[NKG];
+#pragma unroll
+            for (int grp = 0; grp < NKG; ++grp) {
+                const float2 f = meta_f2(kmw[grp]);
+                ksc[grp] = f.x;
+                kzp[grp] = KB == 8 ? fmaf(128.0f, f.x, f.y) : f.y;   // folds the -128 code offset
+            }
+            const float2 vf = meta_f2(vmw);
+            const float vsc = valid ? vf.x : 0.0f;
+            const float vzp = valid ? vf.y : 0.0f;                       // value codes are exact bf16
+            float sc[NHC];
+            bool exceed = false;
+#pragma unroll
+            for (int r = 0; r < NHC; ++r) {
+                float a1 = 0.0f, a2 = 0.0f;
+#pragma unroll
+                for (int grp = 0; grp < NKG; ++grp) {
+                    const int n0 = 12 * r + 3 * grp;
+                    float dot;
+                    if constexpr (KB <= 4) {
+                        dot = (float)(int(ds[n0]) * 16384 + int(ds[n0 + 1]) * 128 + int(ds[n0 + 2]));
+                    } else {
+                        dot = fmaf((float)int(ds[n0]), 16384.0f, fmaf((float)int(ds[n0 + 1]), 128.0f, (float)int(ds[n0 + 2])));
+                    }
+                    a1 = fmaf(ksc[grp], dot, a1);
+                    a2 = fmaf(kzp[grp], qsum[r][grp], a2);
+                }
+                sc[r] = (valid && r < g) ? fmaf(a1, qs0[r], a2) * scale_log2 : -INFINITY;
+                exceed |= sc[r] > m[r] + kLazyMax;
+            }
+            // ---- running max shared by the 4 softmax warps; the vote also
+            // carries a failed wait, so the 4 warps leave together
+            const int wv = (__any_sync(FULL, exceed) ? 1 : 0) | (__any_sync(FULL, !ok) ? 2 : 0);
+            if (lane == 0) sh.vote[u][warp] = wv;
+            named_sync(1, 128);
+            const int votes = sh.vote[u][0] | sh.vote[u][1] | sh.vote[u][2] | sh.vote[u][3];
+            if (votes & 2) {
+                ok = false;
+                break;
+            }
+            if (votes & 1) {
+                // exact max of the tile; rescale l, pz and the ·V accumulator
+#pragma unroll
+                for (int r = 0; r < NHC; ++r) {
+                    const int k = redux_max_s32(ord_key(sc[r]));
+                    if (lane == 0) sh.smax[u][warp][r] = k;
+                }
+                named_sync(1, 128);
+                float alpha[NHC];
+#pragma unroll
+                for (int r = 0; r < NHC; ++r) {
+                    const int k = max(max(sh.smax[u][0][r], sh.smax[u][1][r]), max(sh.smax[u][2][r], sh.smax[u][3][r]));
+                    const float mnew = fmaxf(m[r], ord_val(k));
+                    alpha[r] = (mnew == -INFINITY) ? 1.0f : ex2(m[r] - mnew);
+                    l[r] *= alpha[r];
+                    pz[r] *= alpha[r];
+                    m[r] = mnew;
+                }
+                if (j >= 1) {
+                    wait(&sh.pvdone[(j - 1) & 1], ((j - 1) >> 1) & 1);   // ·V MMA of tile j-1 done
+                    tc_fence_after();
+                    uint32_t o[16];
+                    tmem_ld16(tbase + lane_off + C::COL_O, o);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int n = 0; n < 16; ++n)
+                        o[n] = __float_as_uint(__uint_as_float(o[n]) * alpha[(n >> 1) < NHC ? (n >> 1) : 0]);
+                    tmem_st16(tbase + lane_off + C::COL_O, o);
+                    tc_wait_st();
+                }
+            }
+            // ---- P' of token t into buffer u (free once the ·V MMA of tile j-2 is done)
+            if (j >= 2) wait(&sh.pvdone[u], ((j - 2) >> 1) & 1);
+            uint8_t* pbu = pb + u * 16 * C::CS_P;
+#pragma unroll
+            for (int r = 0; r < NHC; ++r) {
+                if (r >= g) continue;
+                const float mu = (m[r] == -INFINITY) ? 0.0f : m[r];
+                const float pr = ex2(sc[r] - mu);
+                l[r] += pr;
+                pz[r] = fmaf(pr, vzp, pz[r]);
+                const float pv = pr * vsc;
+                const float hi = __bfloat162float(__float2bfloat16_rn(pv));
+                *reinterpret_cast<uint16_t*>(pbu + b_off_bf16(2 * r, kpos_t, C::CS_P)) = bf16_bits(pv);
+                *reinterpret_cast<uint16_t*>(pbu + b_off_bf16(2 * r + 1, kpos_t, C::CS_P)) = bf16_bits(pv - hi);
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.pfull[u]);
+        }
+        cp_wait_all();
+        // ---- partial of this split: o for channel t, m, l
+        const int last = ntiles - 1;
+        wait(&sh.pvdone[last & 1], (last >> 1) & 1);
+        tc_fence_after();
+        uint32_t o[16];
+        tmem_ld16(tbase + lane_off + C::COL_O, o);
+        tc_wait_ld();
+#pragma unroll
+        for (int r = 0; r < NHC; ++r) {
+            const float ls = warp_sum(l[r]);
+            const float zs = warp_sum(pz[r]);
+            if (lane == 0 && r < g) {
+                sh.red[warp][r] = ls;
+                sh.red2[warp][r] = zs;
+            }
+        }
+        named_sync(1, 128);
+        const bool bad = !ok || sh.abort;
+#pragma unroll
+        for (int r = 0; r < NHC; ++r) {
+            if (r >= g) continue;
+            const float z = (sh.red2[0][r] + sh.red2[1][r]) + (sh.red2[2][r] + sh.red2[3][r]);
+            const size_t row = row0 + size_t(r) * slots + x;
+            ws_o[row * D + t] = bad ? NAN : __uint_as_float(o[2 * r]) + __uint_as_float(o[2 * r + 1]) + z;
+            if (t == 0) {
+                const float ls = (sh.red[0][r] + sh.red[1][r]) + (sh.red[2][r] + sh.red[3][r]);
+                ws_ml[row * 2 + 0] = bad ? 0.0f : m[r];
+                ws_ml[row * 2 + 1] = bad ? NAN : ls;
+            }
+        }
+        if (bad && t == 0) atomicAdd(&g_tc_wait_timeouts, 1u);
+    }
+    // ------------------------------------------------------------------ teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tbase, C::TMEM_COLS);
+    }
+}
+
+}  // namespace tc
+}  // namespace kvq

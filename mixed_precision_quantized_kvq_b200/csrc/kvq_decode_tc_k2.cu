@@ -1,0 +1,11 @@
+// Tensor-core decode kernel instantiations for 2-bit keys.
+#include "kvq_decode_tc_launch.cuh"
+
+namespace kvq {
+
+cudaError_t launch_decode_tc_k2(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len,
+                                float sl2, float* ws_o, float* ws_ml, const DecodePlan& pl, cudaStream_t s) {
+    return tc::launch_kb<2>(p, q, q_bf16, lens, max_len, sl2, ws_o, ws_ml, pl, s);
+}
+
+}  // namespace kvq

@@ -121,7 +121,8 @@ struct DecodePlan {
     int tc;             // 1: tensor-core kernel, 0: CUDA-core kernel
     int splits_q;       // splits over quantized pages
     int pages_per_split;
-    int window_split;   // 1 if the layout has a bf16 window (one more partial slot)
+    int window_split;   // partial slots of the bf16 window (CUDA-core kernel: 0 or 1; tensor-core
+                        // kernel: window CTAs per (sequence, kv-head), in slots 0 .. window_split-1)
     int total_splits;   // partial slots per (sequence, query head)
     int grid_x;         // CTAs per (sequence, kv-head)
     int window_slot;    // slot index of the window partial
