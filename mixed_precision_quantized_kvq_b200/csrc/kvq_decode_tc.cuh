@@ -51,9 +51,11 @@ using namespace ptx;
 constexpr int D = 128;
 constexpr int TILE = 128;                     // tokens per tile (two pages)
 constexpr int NKG = 4;                        // key groups of 32 channels
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;
 constexpr int kMaxPagesPerSplit = 256;
 constexpr int kWinPerSplit = 256;             // window positions per window CTA
+constexpr int WCH = 64;                       // window positions per chunk
+constexpr int kWinSmem = 2 * WCH * D * 2;     // key and value rows of a chunk
 constexpr float kLazyMax = 8.0f;              // reuse the running max while scores exceed it by <= 2^8
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr unsigned FULL = 0xffffffffu;
@@ -136,7 +138,8 @@ struct Layout {
     static constexpr int TOTAL = USED > MIN_TOTAL ? USED : MIN_TOTAL;
     static_assert(R >= 3, "ring needs three stages");
     static_assert(OFF_RING == ring_offset(C::NS) && C::STAGE == stage_bytes(KB, VB), "plan formulas agree");
-    static_assert(OFF_RING + 4 * D * kMaxGqa * 4 <= TOTAL, "window reduction buffer fits the ring");
+    static_assert(OFF_RING + kWinSmem <= TOTAL && 4 * D * kMaxGqa * 4 <= WCH * D * 2 * 2,
+                  "window rows and the reduction buffer fit the ring");
 };
 
 // ---------------------------------------------------------------- helpers
@@ -377,50 +380,66 @@ static __device__ void write_empty_partial(int g, float* ws_o, float* ws_ml, siz
 
 // --------------------------------------------------------- window partial
 // CUDA-core attention over window positions [w0, w1) (bf16 keys and values,
-// unrotated query), chunks of 128 positions with an online softmax.  256
-// threads (warps 0-7); every phase issues all of its loads before using them.
-//   scores:  thread pair (2t, 2t+1) splits position t's 128 channels;
+// unrotated query) in chunks of 64 positions with an online softmax.  Every
+// thread of the CTA copies a share of the chunk's key and value rows into
+// shared memory (cp.async); warps 0-7 then compute from shared memory:
+//   scores:  four threads per position, 32 channels each;
 //   ·V:      thread (jp, tq) owns channels 2jp, 2jp+1 and positions tq mod 4;
 //            the four position classes are summed through shared memory.
-static __device__ void window_partial(const Params& p, Shared& sh, float* scratch, int b, int h, int w0, int w1,
-                                      float scale_log2, float* ws_o, float* ws_ml, size_t row0, int slots,
-                                      int slot) {
+
+template <int NHC>
+__device__ __forceinline__ void window_partial(const Params& p, Shared& sh, uint8_t* buf, int b, int h, int w0,
+                                               int w1, float scale_log2, float* ws_o, float* ws_ml, size_t row0,
+                                               int slots, int slot) {
     const int g = p.g, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (warp >= 8) return;
-    const int t = tid >> 1, hf = tid & 1;          // scores: position t of the chunk, channel half hf
-    const int jp = tid & 63, tq = tid >> 6;        // ·V: channel pair, position class
-    float m[kMaxGqa], l[kMaxGqa], o0[kMaxGqa], o1[kMaxGqa];
+    const bool cw = warp < 8;                  // compute warps
+    const int t = (tid >> 2) & (WCH - 1), qq = tid & 3;   // scores: position t, channel quarter qq
+    const int jp = tid & 63, tq = (tid >> 6) & 3;          // ·V: channel pair, position class
+    const __nv_bfloat16* krow = reinterpret_cast<const __nv_bfloat16*>(buf);
+    const __nv_bfloat16* vrow = reinterpret_cast<const __nv_bfloat16*>(buf + WCH * D * 2);
+    float* scratch = reinterpret_cast<float*>(buf);         // reuses the key rows at the end
+    float m[NHC], l[NHC], o0[NHC], o1[NHC];
 #pragma unroll
-    for (int r = 0; r < kMaxGqa; ++r) {
+    for (int r = 0; r < NHC; ++r) {
         m[r] = -INFINITY;
         l[r] = 0.0f;
         o0[r] = 0.0f;
         o1[r] = 0.0f;
     }
     const size_t hb = (size_t(b) * p.hkv + h) * size_t(p.W);
-    for (int c0 = w0; c0 < w1; c0 += TILE) {
-        const int n = min(TILE, w1 - c0);
-        float s[kMaxGqa];
-        {
-            uint4 kv4[8];
+    for (int c0 = w0; c0 < w1; c0 += WCH) {
+        const int n = min(WCH, w1 - c0);
+        // ---- rows of the chunk -> shared memory (16-byte pieces, keys then values)
+        for (int idx = tid; idx < 2 * n * 16; idx += kThreads) {
+            const int kv = idx >= n * 16, rem = kv ? idx - n * 16 : idx;
+            const int row = rem >> 4, piece = rem & 15;
+            const size_t src = (hb + size_t((c0 + row) % p.W)) * D + piece * 8;
+            cp16(buf + kv * (WCH * D * 2) + row * (D * 2) + piece * 16, (kv ? p.v_win : p.k_win) + src, true);
+        }
+        cp_commit();
+        cp_wait<0>();
+        __syncthreads();
+        float s[NHC];
+#pragma unroll
+        for (int r = 0; r < NHC; ++r) s[r] = -INFINITY;
+        if (cw) {
+            // ---- scores: thread (t, qq) takes channels 32qq .. 32qq+31 of position t
+            float acc[NHC];
+#pragma unroll
+            for (int r = 0; r < NHC; ++r) acc[r] = 0.0f;
             const bool in = t < n;
-            int sl = c0 - w0 + t;                       // ring slot of position c0 + t
-            sl = (w0 + sl) % p.W;
-            const uint4* kr = reinterpret_cast<const uint4*>(p.k_win + (hb + size_t(sl)) * D + 64 * hf);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) kv4[c] = in ? __ldg(kr + c) : make_uint4(0, 0, 0, 0);
-            float acc[kMaxGqa];
+            for (int c = 0; c < 4; ++c) {
+                const int cc = (c + (t >> 1)) & 3;             // rotate the 16-byte pieces across lanes
+                const uint4 w4 = in ? *reinterpret_cast<const uint4*>(krow + t * D + 32 * qq + 8 * cc)
+                                    : make_uint4(0, 0, 0, 0);
+                const float kv[8] = {bf_lo(w4.x), bf_hi(w4.x), bf_lo(w4.y), bf_hi(w4.y),
+                                     bf_lo(w4.z), bf_hi(w4.z), bf_lo(w4.w), bf_hi(w4.w)};
 #pragma unroll
-            for (int r = 0; r < kMaxGqa; ++r) acc[r] = 0.0f;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float kv[8] = {bf_lo(kv4[c].x), bf_hi(kv4[c].x), bf_lo(kv4[c].y), bf_hi(kv4[c].y),
-                                     bf_lo(kv4[c].z), bf_hi(kv4[c].z), bf_lo(kv4[c].w), bf_hi(kv4[c].w)};
-#pragma unroll
-                for (int r = 0; r < kMaxGqa; ++r) {
+                for (int r = 0; r < NHC; ++r) {
                     if (r < g) {
-                        const float4 qa = *reinterpret_cast<const float4*>(&sh.qf[r][64 * hf + 8 * c]);
-                        const float4 qb = *reinterpret_cast<const float4*>(&sh.qf[r][64 * hf + 8 * c + 4]);
+                        const float4 qa = *reinterpret_cast<const float4*>(&sh.qf[r][32 * qq + 8 * cc]);
+                        const float4 qb = *reinterpret_cast<const float4*>(&sh.qf[r][32 * qq + 8 * cc + 4]);
                         acc[r] = fmaf(qa.x, kv[0], acc[r]);
                         acc[r] = fmaf(qa.y, kv[1], acc[r]);
                         acc[r] = fmaf(qa.z, kv[2], acc[r]);
@@ -433,74 +452,72 @@ static __device__ void window_partial(const Params& p, Shared& sh, float* scratc
                 }
             }
 #pragma unroll
-            for (int r = 0; r < kMaxGqa; ++r) {
-                const float tot = acc[r] + __shfl_xor_sync(FULL, acc[r], 1);
+            for (int r = 0; r < NHC; ++r) {
+                float tot = acc[r] + __shfl_xor_sync(FULL, acc[r], 1);
+                tot += __shfl_xor_sync(FULL, tot, 2);
                 s[r] = (in && r < g) ? tot * scale_log2 : -INFINITY;
                 const float wm = warp_max(s[r]);
                 if (lane == 0 && r < g) sh.wred[warp][r] = wm;
             }
         }
-        named_sync(2, 256);
-        float mnew[kMaxGqa], alpha[kMaxGqa];
+        __syncthreads();
+        if (cw) {
 #pragma unroll
-        for (int r = 0; r < kMaxGqa; ++r) {
-            mnew[r] = m[r];
-            alpha[r] = 1.0f;
-            if (r < g) {
-                float cm = sh.wred[0][r];
+            for (int r = 0; r < NHC; ++r) {
+                if (r < g) {
+                    float cm = sh.wred[0][r];
 #pragma unroll
-                for (int w = 1; w < 8; ++w) cm = fmaxf(cm, sh.wred[w][r]);
-                mnew[r] = fmaxf(m[r], cm);
-                alpha[r] = (mnew[r] == -INFINITY) ? 1.0f : ex2(m[r] - mnew[r]);
-                m[r] = mnew[r];
-                const float pr = (s[r] == -INFINITY) ? 0.0f : ex2(s[r] - mnew[r]);
-                l[r] = fmaf(l[r], alpha[r], hf == 0 ? pr : 0.0f);
-                if (hf == 0) sh.wsc[r][t] = pr;
-                o0[r] *= alpha[r];
-                o1[r] *= alpha[r];
+                    for (int w = 1; w < 8; ++w) cm = fmaxf(cm, sh.wred[w][r]);
+                    const float mnew = fmaxf(m[r], cm);
+                    const float alpha = (mnew == -INFINITY) ? 1.0f : ex2(m[r] - mnew);
+                    m[r] = mnew;
+                    const float pr = (s[r] == -INFINITY) ? 0.0f : ex2(s[r] - mnew);
+                    l[r] = fmaf(l[r], alpha, qq == 0 ? pr : 0.0f);
+                    if (qq == 0) sh.wsc[r][t] = pr;
+                    o0[r] *= alpha;
+                    o1[r] *= alpha;
+                }
             }
         }
-        named_sync(2, 256);
-        {
-            uint32_t vv[TILE / 4];
-            const __nv_bfloat16* vc = p.v_win + hb * D + 2 * jp;
-#pragma unroll
-            for (int k = 0; k < TILE / 4; ++k) {
+        __syncthreads();
+        if (cw) {
+            // ---- ·V: positions tq, tq+4, ... of the chunk, channels 2jp, 2jp+1
+#pragma unroll 4
+            for (int k = 0; k < WCH / 4; ++k) {
                 const int tt = tq + 4 * k;
-                const int sl = (c0 + tt) % p.W;
-                vv[k] = tt < n ? __ldg(reinterpret_cast<const uint32_t*>(vc + size_t(sl) * D)) : 0u;
-            }
+                if (tt < n) {
+                    const uint32_t vv = *reinterpret_cast<const uint32_t*>(vrow + tt * D + 2 * jp);
+                    const float va = bf_lo(vv), vb = bf_hi(vv);
 #pragma unroll
-            for (int k = 0; k < TILE / 4; ++k) {
-                const int tt = tq + 4 * k;
-                const float va = bf_lo(vv[k]), vb = bf_hi(vv[k]);
-#pragma unroll
-                for (int r = 0; r < kMaxGqa; ++r) {
-                    if (r < g) {
-                        const float pr = tt < n ? sh.wsc[r][tt] : 0.0f;
-                        o0[r] = fmaf(pr, va, o0[r]);
-                        o1[r] = fmaf(pr, vb, o1[r]);
+                    for (int r = 0; r < NHC; ++r) {
+                        if (r < g) {
+                            const float pr = sh.wsc[r][tt];
+                            o0[r] = fmaf(pr, va, o0[r]);
+                            o1[r] = fmaf(pr, vb, o1[r]);
+                        }
                     }
                 }
             }
         }
-        named_sync(2, 256);                         // wsc and wred are rewritten by the next chunk
+        __syncthreads();                            // rows, wsc and wred are rewritten next
     }
     // position classes -> channel sums; l over the score threads
+    if (cw) {
 #pragma unroll
-    for (int r = 0; r < kMaxGqa; ++r) {
-        if (r < g) {
-            scratch[(tq * kMaxGqa + r) * D + 2 * jp] = o0[r];
-            scratch[(tq * kMaxGqa + r) * D + 2 * jp + 1] = o1[r];
+        for (int r = 0; r < NHC; ++r) {
+            if (r < g) {
+                scratch[(tq * kMaxGqa + r) * D + 2 * jp] = o0[r];
+                scratch[(tq * kMaxGqa + r) * D + 2 * jp + 1] = o1[r];
+            }
+            const float ls = warp_sum(l[r]);
+            if (lane == 0 && r < g) sh.wred[warp][r] = ls;
         }
-        const float ls = warp_sum(l[r]);
-        if (lane == 0 && r < g) sh.wred[warp][r] = ls;
     }
-    named_sync(2, 256);
+    __syncthreads();
     if (tid < D) {
         const int j = tid;
 #pragma unroll
-        for (int r = 0; r < kMaxGqa; ++r) {
+        for (int r = 0; r < NHC; ++r) {
             if (r >= g) continue;
             const float v = (scratch[(0 * kMaxGqa + r) * D + j] + scratch[(1 * kMaxGqa + r) * D + j]) +
                             (scratch[(2 * kMaxGqa + r) * D + j] + scratch[(3 * kMaxGqa + r) * D + j]);
@@ -573,9 +590,7 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
     }
     __syncthreads();
     if (is_win) {
-        window_partial(p, sh, reinterpret_cast<float*>(ring), b, h, w0, w1, scale_log2, ws_o, ws_ml, row0, slots,
-                       x);
-        __syncthreads();
+        window_partial<NHC>(p, sh, ring, b, h, w0, w1, scale_log2, ws_o, ws_ml, row0, slots, x);
         return;
     }
 
@@ -592,7 +607,7 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
         mbar_fence_init();
         sh.abort = 0;
     }
-    if (warp == 8) {
+    if (warp == 12) {
         tmem_alloc(&sh.tmem_base, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -652,7 +667,7 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
         }
     };
 
-    if (warp == 8) {
+    if (warp == 12) {
         // ======================================================== score MMA
         const uint64_t qd = smem_desc(smem_u32(qb), C::CS_Q, 128);
         for (int i = 0; i < ntiles; ++i) {
@@ -669,7 +684,7 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
         }
         tc_commit_warp(&sh.mma_done[0]);          // every MMA above has completed before the teardown
         mbar_wait(&sh.mma_done[0], 0, kWaitNs);
-    } else if (warp == 9) {
+    } else if (warp == 13) {
         // =========================================================== ·V MMA
         const uint32_t pb_s = smem_u32(pb);
         for (int j = 0; j < ntiles; ++j) {
@@ -687,23 +702,55 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
         }
         tc_commit_warp(&sh.mma_done[1]);
         mbar_wait(&sh.mma_done[1], 0, kWaitNs);
-    } else if (warp >= 4) {
-        // =========================================================== loaders
-        const int ti = tid - 128;                 // token ti (keys) and channel ti (values)
+    } else if (warp >= 4 && warp < 8) {
+        // ======================================================= key loaders
+        const int ti = tid - 128;                 // token ti of each tile
         const int pp_k = ti >> 6, slot_k = ti & 63;
         auto issue = [&](int i) {
             uint8_t* st = ring + (i % R) * C::STAGE;
-            {   // key codes of token ti
-                const int lp = pg0 + 2 * i + pp_k;
-                const int pg = lp < pg1 ? sh.pages[2 * i + pp_k] : -1;
-                const bool have = pg >= 0;
-                const uint8_t* kb = p.k_codes + (size_t(have ? pg : 0) * p.hkv + h) * (kPage * C::KROW) + slot_k * 16;
+            const int lp = pg0 + 2 * i + pp_k;
+            const int pg = lp < pg1 ? sh.pages[2 * i + pp_k] : -1;
+            const bool have = pg >= 0;
+            const uint8_t* kb = p.k_codes + (size_t(have ? pg : 0) * p.hkv + h) * (kPage * C::KROW) + slot_k * 16;
 #pragma unroll
-                for (int c = 0; c < C::KROW / 16; ++c)
-                    cp16(st + C::ST_K + c * (TILE * 16) + ti * 16, kb + c * (kPage * 16), have);
+            for (int c = 0; c < C::KROW / 16; ++c)
+                cp16(st + C::ST_K + c * (TILE * 16) + ti * 16, kb + c * (kPage * 16), have);
+        };
+        for (int i = 0; i < R - 1; ++i) {
+            if (i < ntiles) issue(i);
+            cp_commit();
+        }
+        for (int i = 0; i < ntiles; ++i) {
+            if (i + R - 1 < ntiles) issue(i + R - 1);
+            cp_commit();
+            cp_wait<R - 1>();
+            const uint8_t* st = ring + (i % R) * C::STAGE;
+            uint32_t a[32];
+#pragma unroll
+            for (int c = 0; c < C::KROW / 16; ++c) {
+                const uint4 w4 = *reinterpret_cast<const uint4*>(st + C::ST_K + c * (TILE * 16) + ti * 16);
+                unpack_i8<KB>(w4.x, &a[(4 * c + 0) * (8 / KB)]);
+                unpack_i8<KB>(w4.y, &a[(4 * c + 1) * (8 / KB)]);
+                unpack_i8<KB>(w4.z, &a[(4 * c + 2) * (8 / KB)]);
+                unpack_i8<KB>(w4.w, &a[(4 * c + 3) * (8 / KB)]);
             }
+            if (i >= 2) wait(&sh.sfull[i & 1], ((i - 2) >> 1) & 1);   // score MMA of tile i-2 read the buffer
+            if (__any_sync(FULL, !ok)) break;
+            tc_fence_after();
+            tmem_st32(tbase + lane_off + C::COL_AK + 32 * (i & 1), a);
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.kfull[i & 1]);
+        }
+        cp_wait_all();
+    } else if (warp >= 8 && warp < 12) {
+        // ===================================================== value loaders
+        const int ti = tid - 256;                 // value channel ti
+        auto issue = [&](int i) {
+            uint8_t* st = ring + (i % R) * C::STAGE;
 #pragma unroll
-            for (int pp = 0; pp < 2; ++pp) {      // value codes of channel ti, both pages
+            for (int pp = 0; pp < 2; ++pp) {
                 const int lp = pg0 + 2 * i + pp;
                 const int pg = lp < pg1 ? sh.pages[2 * i + pp] : -1;
                 const bool have = pg >= 0;
@@ -718,69 +765,41 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
                 }
             }
         };
-        auto keys = [&](int i) {                  // key codes of tile i -> int8 operand buffer i&1
-            const uint8_t* st = ring + (i % R) * C::STAGE;
-            uint32_t a[32];
-#pragma unroll
-            for (int c = 0; c < C::KROW / 16; ++c) {
-                const uint4 w4 = *reinterpret_cast<const uint4*>(st + C::ST_K + c * (TILE * 16) + ti * 16);
-                unpack_i8<KB>(w4.x, &a[(4 * c + 0) * (8 / KB)]);
-                unpack_i8<KB>(w4.y, &a[(4 * c + 1) * (8 / KB)]);
-                unpack_i8<KB>(w4.z, &a[(4 * c + 2) * (8 / KB)]);
-                unpack_i8<KB>(w4.w, &a[(4 * c + 3) * (8 / KB)]);
-            }
-            if (i >= 2) wait(&sh.sfull[i & 1], ((i - 2) >> 1) & 1);   // score MMA of tile i-2 read the buffer
-            tc_fence_after();
-            tmem_st32(tbase + lane_off + C::COL_AK + 32 * (i & 1), a);
-            tc_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.kfull[i & 1]);
-        };
-        auto values = [&](int i) {                // value codes of tile i -> bf16 operand
-            const uint8_t* st = ring + (i % R) * C::STAGE + C::ST_V;
-            uint32_t a[64];
-#pragma unroll
-            for (int pp = 0; pp < 2; ++pp) {
-                if constexpr (VB == 1) {
-                    const uint2 w2 = *reinterpret_cast<const uint2*>(st + ti * 16 + pp * 8);
-                    Unpack<1>::word(w2.x, &a[pp * 32]);
-                    Unpack<1>::word(w2.y, &a[pp * 32 + VREG]);
-                } else {
-#pragma unroll
-                    for (int c = 0; c < VWP / 4; ++c) {
-                        const uint4 w4 = *reinterpret_cast<const uint4*>(st + (pp * (VWP / 4) + c) * (D * 16) + ti * 16);
-                        Unpack<VB>::word(w4.x, &a[pp * 32 + c * 4 * VREG + 0 * VREG]);
-                        Unpack<VB>::word(w4.y, &a[pp * 32 + c * 4 * VREG + 1 * VREG]);
-                        Unpack<VB>::word(w4.z, &a[pp * 32 + c * 4 * VREG + 2 * VREG]);
-                        Unpack<VB>::word(w4.w, &a[pp * 32 + c * 4 * VREG + 3 * VREG]);
-                    }
-                }
-            }
-            if (i >= 1) wait(&sh.pvdone[(i - 1) & 1], ((i - 1) >> 1) & 1);   // ·V MMA of tile i-1 read the operand
-            tc_fence_after();
-            tmem_st32(tbase + lane_off + C::COL_AV, a);
-            tmem_st32(tbase + lane_off + C::COL_AV + 32, a + 32);
-            tc_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.vfull);
-        };
-        // keys run one tile ahead of values: iteration i unpacks keys of
-        // tile i+1 and values of tile i (ring slots of tiles i .. i+R-1 live)
         for (int i = 0; i < R - 1; ++i) {
             if (i < ntiles) issue(i);
             cp_commit();
         }
-        cp_wait_n<R - 2>();
-        keys(0);
         for (int i = 0; i < ntiles; ++i) {
-            if (__any_sync(FULL, !ok)) break;
             if (i + R - 1 < ntiles) issue(i + R - 1);
             cp_commit();
-            cp_wait_n<R - 2>();                   // tiles i and i+1 landed
-            if (i + 1 < ntiles) keys(i + 1);
-            values(i);
+            cp_wait<R - 1>();
+            const uint8_t* st = ring + (i % R) * C::STAGE + C::ST_V;
+            if (i >= 1) wait(&sh.pvdone[(i - 1) & 1], ((i - 1) >> 1) & 1);   // ·V MMA of tile i-1 read the operand
+            if (__any_sync(FULL, !ok)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int pp = 0; pp < 2; ++pp) {      // one page (32 columns) at a time
+                uint32_t a[32];
+                if constexpr (VB == 1) {
+                    const uint2 w2 = *reinterpret_cast<const uint2*>(st + ti * 16 + pp * 8);
+                    Unpack<1>::word(w2.x, &a[0]);
+                    Unpack<1>::word(w2.y, &a[VREG]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < VWP / 4; ++c) {
+                        const uint4 w4 = *reinterpret_cast<const uint4*>(st + (pp * (VWP / 4) + c) * (D * 16) + ti * 16);
+                        Unpack<VB>::word(w4.x, &a[c * 4 * VREG + 0 * VREG]);
+                        Unpack<VB>::word(w4.y, &a[c * 4 * VREG + 1 * VREG]);
+                        Unpack<VB>::word(w4.z, &a[c * 4 * VREG + 2 * VREG]);
+                        Unpack<VB>::word(w4.w, &a[c * 4 * VREG + 3 * VREG]);
+                    }
+                }
+                tmem_st32(tbase + lane_off + C::COL_AV + 32 * pp, a);
+            }
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.vfull);
         }
         cp_wait_all();
     } else {
@@ -824,17 +843,7 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
             const uint32_t vmw = *reinterpret_cast<const uint32_t*>(st + C::ST_VM + t * 4);
             const int lp = pg0 + 2 * j + pp_t;
             const bool valid = lp < pg1 && sh.pages[2 * j + pp_t] >= 0 && lp * kPage + slot_t < Lq;
-            // ---- s32 score products of token t
-            wait(&sh.sfull[u], (j >> 1) & 1);
-            tc_fence_after();
-            uint32_t ds[NS];
-#pragma unroll
-            for (int c = 0; c < NS / 16; ++c)
-                tmem_ld16(tbase + lane_off + C::COL_S + NS * u + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(&ds[16 * c]));
-            tc_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.sfree[u]);
+            // ---- scores of token t from the s32 products, two heads at a time
             const uint32_t kmw[NKG] = {km4.x, km4.y, km4.z, km4.w};
             float ksc[NKG], kzp[NKG];
 #pragma unroll
@@ -846,26 +855,40 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
             const float2 vf = meta_f2(vmw);
             const float vsc = valid ? vf.x : 0.0f;
             const float vzp = valid ? vf.y : 0.0f;                       // value codes are exact bf16
+            wait(&sh.sfull[u], (j >> 1) & 1);
+            tc_fence_after();
             float sc[NHC];
             bool exceed = false;
 #pragma unroll
-            for (int r = 0; r < NHC; ++r) {
-                float a1 = 0.0f, a2 = 0.0f;
+            for (int hp = 0; hp < NHC / 2; ++hp) {
+                uint32_t ds[24];
 #pragma unroll
-                for (int grp = 0; grp < NKG; ++grp) {
-                    const int n0 = 12 * r + 3 * grp;
-                    float dot;
-                    if constexpr (KB <= 4) {
-                        dot = (float)(int(ds[n0]) * 16384 + int(ds[n0 + 1]) * 128 + int(ds[n0 + 2]));
-                    } else {
-                        dot = fmaf((float)int(ds[n0]), 16384.0f, fmaf((float)int(ds[n0 + 1]), 128.0f, (float)int(ds[n0 + 2])));
+                for (int c = 0; c < 3; ++c) tmem_ld8(tbase + lane_off + C::COL_S + NS * u + 24 * hp + 8 * c, &ds[8 * c]);
+                tc_wait_ld();
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int r = 2 * hp + rr;
+                    float a1 = 0.0f, a2 = 0.0f;
+#pragma unroll
+                    for (int grp = 0; grp < NKG; ++grp) {
+                        const int n0 = 12 * rr + 3 * grp;
+                        float dot;
+                        if constexpr (KB <= 4) {
+                            dot = (float)(int(ds[n0]) * 16384 + int(ds[n0 + 1]) * 128 + int(ds[n0 + 2]));
+                        } else {
+                            dot = fmaf((float)int(ds[n0]), 16384.0f,
+                                       fmaf((float)int(ds[n0 + 1]), 128.0f, (float)int(ds[n0 + 2])));
+                        }
+                        a1 = fmaf(ksc[grp], dot, a1);
+                        a2 = fmaf(kzp[grp], qsum[r][grp], a2);
                     }
-                    a1 = fmaf(ksc[grp], dot, a1);
-                    a2 = fmaf(kzp[grp], qsum[r][grp], a2);
+                    sc[r] = (valid && r < g) ? fmaf(a1, qs0[r], a2) * scale_log2 : -INFINITY;
+                    exceed |= sc[r] > m[r] + kLazyMax;
                 }
-                sc[r] = (valid && r < g) ? fmaf(a1, qs0[r], a2) * scale_log2 : -INFINITY;
-                exceed |= sc[r] > m[r] + kLazyMax;
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.sfree[u]);
             // ---- running max shared by the 4 softmax warps; the vote also
             // carries a failed wait, so the 4 warps leave together
             const int wv = (__any_sync(FULL, exceed) ? 1 : 0) | (__any_sync(FULL, !ok) ? 2 : 0);
@@ -963,7 +986,7 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
     // ------------------------------------------------------------------ teardown
     tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == 12) {
         tc_fence_after();
         tmem_dealloc(tbase, C::TMEM_COLS);
     }
