@@ -30,8 +30,7 @@ DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count) {
     if (pl.tc) {
         // window CTAs first (slots 0 .. nws-1, 256 window positions each),
         // then the quantized splits, each a whole number of 128-token tiles:
-        // one wave of CTAs where the units allow it, else tiles of at most
-        // 16 per split so that ragged lengths balance across the waves
+        // one wave of CTAs where the units allow it, at most 16 tiles per split
         const int win = p.W < max_len ? p.W : max_len;
         pl.window_split = win > 0 ? (win + 255) / 256 : 0;
         const int slots = sm_count * tc_ctas_per_sm(p);
@@ -44,7 +43,7 @@ DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count) {
             if (want < 1) want = 1;
             if (want > tiles) want = tiles;
             int tps = (tiles + want - 1) / want;
-            if (units * ((tiles + tps - 1) / tps) > slots && tps > 16) tps = 16;
+            if (tps > 16) tps = 16;                     // the kernel keeps a split's scores on chip
             pl.pages_per_split = 2 * tps;
             if (pl.pages_per_split > 256) pl.pages_per_split = 256;   // page ids staged in shared memory
             pl.splits_q = (npages + pl.pages_per_split - 1) / pl.pages_per_split;

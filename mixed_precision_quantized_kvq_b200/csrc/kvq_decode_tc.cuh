@@ -18,21 +18,20 @@
 //    a bf16 pair (high part + remainder), accumulated in fp32 in tensor
 //    memory across the whole split.
 //
-// One CTA per (sequence, kv-head, split), 320 threads, two CTAs per SM
-// (256 tensor-memory columns each) when the GQA ratio is at most 4:
-//   warps 0-3  softmax: thread t owns token t of each 128-token tile (two
-//              pages); it prefetches the token's metadata with cp.async,
-//              turns the s32 score products into scores, keeps the running
-//              max (reused while scores stay within 2^8 of it; a larger one
-//              triggers an exact max and a rescale of the ·V accumulator)
-//              and writes P' as the B operand of the ·V MMA;
-//   warps 4-7  loaders: thread i prefetches token i's key codes and channel
-//              i's value codes with cp.async into a ring of shared-memory
-//              stages and unpacks them into tensor memory (score A operand:
-//              M = 128 tokens, K = 128 channels, int8, double buffered; ·V A
-//              operand: M = 128 channels, K = 128 tokens, bf16);
-//   warp 8     issues the score MMAs of each tile;
-//   warp 9     issues the ·V MMAs of each tile.
+// One CTA per (sequence, kv-head, split of at most 16 tiles of 128 tokens),
+// 288 threads, two CTAs per SM when they fit.  Two phases:
+//   1. scores: loader warps unpack key codes to int8 in tensor memory
+//      (double buffered), the MMA warp multiplies them with the query limbs,
+//      the softmax warps turn the s32 products into fp32 scores, keep them in
+//      shared memory and track their maximum;
+//   2. values: with the exact maximum known, the softmax warps write
+//      P' = 2^(s - max) * value_scale as a bf16 pair, the loader warps unpack
+//      value codes to bf16 in tensor memory (double buffered in the columns
+//      phase 1 used), and the MMA warp accumulates ·V in tensor memory.
+// Warps 0-3 softmax (thread t owns token t of each tile: metadata, scores,
+// P'), warps 4-7 loaders (thread i owns token i's key codes and channel i's
+// value codes; per-thread cp.async into a ring of shared-memory stages that
+// runs through both phases), warp 8 issues every MMA (one elected lane).
 // Hand-overs go through mbarriers; every wait is bounded.  The bf16 window
 // positions are handled by separate CTAs of the same grid on CUDA cores
 // (fp32), each writing its own partial.
@@ -51,53 +50,63 @@ using namespace ptx;
 constexpr int D = 128;
 constexpr int TILE = 128;                     // tokens per tile (two pages)
 constexpr int NKG = 4;                        // key groups of 32 channels
-constexpr int kThreads = 448;
+constexpr int kThreads = 288;
 constexpr int kMaxPagesPerSplit = 256;
+constexpr int kMaxTiles = 16;                 // tiles per quantized split (scores are kept in shared memory)
 constexpr int kWinPerSplit = 256;             // window positions per window CTA
 constexpr int WCH = 64;                       // window positions per chunk
 constexpr int kWinSmem = 2 * WCH * D * 2;     // key and value rows of a chunk
-constexpr float kLazyMax = 8.0f;              // reuse the running max while scores exceed it by <= 2^8
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr unsigned FULL = 0xffffffffu;
 
 // number of bounded waits that expired (diagnostic; 0 in normal operation)
 static __device__ unsigned int g_tc_wait_timeouts;
 
+constexpr int ns_cols(int nhc) { return ((12 * nhc + 15) / 16) * 16; }
+// score accumulator buffers: two when they fit in 256 columns with the rest
+constexpr int s_bufs(int nhc) { return 64 + 2 * ns_cols(nhc) + 16 <= 256 ? 2 : 1; }
+
 template <int KB, int VB, int NHC>
 struct Cfg {
-    static constexpr int NS = ((12 * NHC + 15) / 16) * 16;   // score columns (head, key group, limb)
+    static constexpr int NS = ns_cols(NHC);                  // score columns (head, key group, limb)
+    static constexpr int SB = s_bufs(NHC);                   // score accumulator buffers
     static constexpr int NO = 16;                            // ·V columns (head, high / remainder)
-    static constexpr int COL_AK = 0;                         // 2 x 32 key operand columns (int8)
-    static constexpr int COL_AV = 64;                        // 64 value operand columns (bf16)
-    static constexpr int COL_S = 128;                        // 2 x NS score accumulators
-    static constexpr int COL_O = COL_S + 2 * NS;             // ·V accumulator
-    static constexpr int TMEM_COLS = COL_O + NO <= 256 ? 256 : 512;
+    // tensor-memory columns.  Phase 1: key operands (int8) at 0 and 32, score
+    // accumulators from 64.  Phase 2: value operands (bf16) at 0 and 64,
+    // over the phase-1 columns.  The ·V accumulator after both.
+    static constexpr int COL_AK = 0;
+    static constexpr int COL_S = 64;
+    static constexpr int COL_AV = 0;
+    static constexpr int COL_O = COL_S + SB * NS;
+    static constexpr int TMEM_COLS = 256;
+    static_assert(COL_S + SB * NS >= 128, "second value operand lies inside the phase-1 columns");
+    static_assert(COL_O + NO <= TMEM_COLS, "tensor-memory plan fits 256 columns");
     static constexpr int KROW = D * KB / 8;                  // key row bytes of one token
     static constexpr int VCH = kPage * VB / 8;               // value bytes of one channel in one page
-    // one ring stage: keys [chunk][token][16 B], values [chunk][channel][16 B],
-    // key meta [token][16 B], value meta [token][4 B]
-    static constexpr int ST_K = 0;
-    static constexpr int ST_V = ST_K + TILE * KROW;
-    static constexpr int ST_KM = ST_V + D * 2 * VCH;
-    static constexpr int ST_VM = ST_KM + TILE * 16;
-    static constexpr int STAGE = ST_VM + TILE * 4;
+    // one ring stage holds either a key step (codes [chunk][token][16 B],
+    // key meta [token][16 B]) or a value step (codes [chunk][channel][16 B],
+    // value meta in the first 4 bytes of [token][16 B]).  Every thread reads
+    // back only bytes it copied itself, in both phases: warps run at their
+    // own pace, so no two threads may share bytes of a stage.
+    static constexpr int CODES = TILE * KROW > D * 2 * VCH ? TILE * KROW : D * 2 * VCH;
+    static constexpr int ST_M = CODES;
+    static constexpr int STAGE = CODES + TILE * 16;
     static constexpr int CS_Q = NS * 16 + 16;                // chunk stride of the query operand
     static constexpr int CS_P = 16 * 16 + 16;                // chunk stride of the P' operand
     static_assert(2 * NHC <= NO, "two ·V columns per head");
 };
 
 struct Shared {
-    uint64_t kfull[2];       // loaders -> score MMA: key operand written
-    uint64_t sfull[2];       // score MMA -> softmax: accumulator ready (and key operand free)
-    uint64_t sfree[2];       // softmax -> score MMA: accumulator read
-    uint64_t vfull;          // loaders -> ·V MMA: value operand written
-    uint64_t pfull[2];       // softmax -> ·V MMA: P' operand written
-    uint64_t pvdone[2];      // ·V MMA -> softmax, loaders: product of the tile done
-    uint64_t mma_done[2];
+    uint64_t kfull[2];       // loaders -> MMA: key operand written
+    uint64_t sfull[2];       // MMA -> softmax, loaders: score products ready (key operand read)
+    uint64_t sfree[2];       // softmax -> MMA, loaders: score accumulator read
+    uint64_t vfull[2];       // loaders -> MMA: value operand written
+    uint64_t pfull[2];       // softmax -> MMA: P' operand written
+    uint64_t pvdone[2];      // MMA -> softmax, loaders: ·V product of the tile done
+    uint64_t mma_done;
     uint32_t tmem_base;
     int abort;
-    int vote[2][4];
-    int smax[2][4][kMaxGqa];             // per warp: max score (ordered int) per head
+    float smax[4][kMaxGqa];              // softmax warps: score maxima
     float red[4][kMaxGqa], red2[4][kMaxGqa];
     alignas(16) float qsum[kMaxGqa][NKG];   // sums of the rotated query per key group
     float qs0[kMaxGqa];                  // query limb unit: 2^-14 of the head's s0
@@ -108,18 +117,19 @@ struct Shared {
     int pages[kMaxPagesPerSplit];
 };
 
-// Shared-memory plan: Shared, the query operand, two P' buffers, then a
-// ring of R stages.  Two CTAs share an SM when the tensor memory allows it
-// and three stages still fit in half the shared memory; otherwise one.
-constexpr int kSmemPerSm = 228 * 1024;         // shared memory of an SM (reservations excluded below)
-constexpr int ring_offset(int ns) {
-    return (((((int(sizeof(Shared)) + 127) & ~127) + 8 * (ns * 16 + 16) + 2 * 16 * (16 * 16 + 16)) + 127) & ~127);
+// Shared-memory plan: Shared, the query operand, two P' buffers, the scores
+// of the split, then a ring of R stages.  Two CTAs share an SM when three
+// stages still fit in half the shared memory; otherwise one.
+constexpr int stage_bytes(int kb, int vb) {
+    return (TILE * (D * kb / 8) > D * 2 * (kPage * vb / 8) ? TILE * (D * kb / 8) : D * 2 * (kPage * vb / 8)) +
+           TILE * 16;
 }
-constexpr int stage_bytes(int kb, int vb) { return TILE * (D * kb / 8) + D * 2 * (kPage * vb / 8) + TILE * 16 + TILE * 4; }
-constexpr int ns_cols(int nhc) { return ((12 * nhc + 15) / 16) * 16; }
+constexpr int ring_offset(int nhc) {
+    return ((((int(sizeof(Shared)) + 127) & ~127) + 8 * (ns_cols(nhc) * 16 + 16) + 2 * 16 * (16 * 16 + 16) +
+             kMaxTiles * nhc * TILE * 4) + 127) & ~127;
+}
 constexpr int ctas_per_sm(int kb, int vb, int nhc) {
-    return (128 + 2 * ns_cols(nhc) + 16 <= 256 && (112 * 1024 - ring_offset(ns_cols(nhc))) / stage_bytes(kb, vb) >= 3) ? 2
-                                                                                                                      : 1;
+    return (112 * 1024 - ring_offset(nhc)) / stage_bytes(kb, vb) >= 3 ? 2 : 1;
 }
 
 template <int KB, int VB, int NHC>
@@ -128,7 +138,8 @@ struct Layout {
     static constexpr int CTAS = ctas_per_sm(KB, VB, NHC);
     static constexpr int OFF_QB = (int(sizeof(Shared)) + 127) & ~127;
     static constexpr int OFF_PB = OFF_QB + 8 * C::CS_Q;
-    static constexpr int OFF_RING = (OFF_PB + 2 * 16 * C::CS_P + 127) & ~127;
+    static constexpr int OFF_SC = OFF_PB + 2 * 16 * C::CS_P;          // scores [tile][head][token] fp32
+    static constexpr int OFF_RING = (OFF_SC + kMaxTiles * NHC * TILE * 4 + 127) & ~127;
     static constexpr int BUDGET = CTAS == 2 ? 112 * 1024 : 224 * 1024;
     static constexpr int R0 = (BUDGET - OFF_RING) / C::STAGE;
     static constexpr int R = R0 > 8 ? 8 : R0;                 // ring stages
@@ -137,9 +148,9 @@ struct Layout {
     static constexpr int MIN_TOTAL = CTAS == 2 ? 80 * 1024 : 120 * 1024;
     static constexpr int TOTAL = USED > MIN_TOTAL ? USED : MIN_TOTAL;
     static_assert(R >= 3, "ring needs three stages");
-    static_assert(OFF_RING == ring_offset(C::NS) && C::STAGE == stage_bytes(KB, VB), "plan formulas agree");
-    static_assert(OFF_RING + kWinSmem <= TOTAL && 4 * D * kMaxGqa * 4 <= WCH * D * 2 * 2,
-                  "window rows and the reduction buffer fit the ring");
+    static_assert(OFF_RING == ring_offset(NHC) && C::STAGE == stage_bytes(KB, VB), "plan formulas agree");
+    static_assert(OFF_SC + kWinSmem <= TOTAL && 4 * D * kMaxGqa * 4 <= WCH * D * 2 * 2,
+                  "window rows and the reduction buffer fit from the score area on");
 };
 
 // ---------------------------------------------------------------- helpers
@@ -547,7 +558,7 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
     using C = Cfg<KB, VB, NHC>;
     using LY = Layout<KB, VB, NHC>;
     constexpr int R = LY::R;
-    constexpr int NS = C::NS;
+    constexpr int NS = C::NS, SB = C::SB;
     constexpr uint32_t IDESC_S = idesc_s8(128, NS);
     constexpr uint32_t IDESC_O = idesc_bf16_f32(128, C::NO);
     constexpr int VWP = kPage * VB / 32;     // value words per channel per page
@@ -558,6 +569,7 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
     uint8_t* qb = smem + LY::OFF_QB;
     uint8_t* pb = smem + LY::OFF_PB;
     uint8_t* ring = smem + LY::OFF_RING;
+    float* scs = reinterpret_cast<float*>(smem + LY::OFF_SC);   // [tile][head][token]
 
     const int b = blockIdx.z, h = blockIdx.y, x = blockIdx.x;
     const int g = p.g, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -590,7 +602,7 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
     }
     __syncthreads();
     if (is_win) {
-        window_partial<NHC>(p, sh, ring, b, h, w0, w1, scale_log2, ws_o, ws_ml, row0, slots, x);
+        window_partial<NHC>(p, sh, smem + LY::OFF_SC, b, h, w0, w1, scale_log2, ws_o, ws_ml, row0, slots, x);
         return;
     }
 
@@ -599,15 +611,15 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
             mbar_init(&sh.kfull[u], 4);
             mbar_init(&sh.sfull[u], 1);
             mbar_init(&sh.sfree[u], 4);
+            mbar_init(&sh.vfull[u], 4);
             mbar_init(&sh.pfull[u], 4);
             mbar_init(&sh.pvdone[u], 1);
-            mbar_init(&sh.mma_done[u], 1);
         }
-        mbar_init(&sh.vfull, 4);
+        mbar_init(&sh.mma_done, 1);
         mbar_fence_init();
         sh.abort = 0;
     }
-    if (warp == 12) {
+    if (warp == 8) {
         tmem_alloc(&sh.tmem_base, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -655,6 +667,7 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
     tc_fence_after();
     const uint32_t tbase = sh.tmem_base;
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;     // this warp's tensor-memory lanes
+    const int nt = ntiles;
     bool ok = true;
     auto wait = [&](uint64_t* bar, uint32_t parity) {
         if (!ok || sh.abort) {
@@ -666,184 +679,172 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
             sh.abort = 1;
         }
     };
+    // ring steps: step k < nt is key tile k, step k >= nt is value tile k - nt
 
-    if (warp == 12) {
-        // ======================================================== score MMA
+    if (warp == 8) {
+        // =============================================================== MMA
         const uint64_t qd = smem_desc(smem_u32(qb), C::CS_Q, 128);
-        for (int i = 0; i < ntiles; ++i) {
-            const int u = i & 1;
-            wait(&sh.kfull[u], (i >> 1) & 1);
-            if (i >= 2) wait(&sh.sfree[u], ((i - 2) >> 1) & 1);
+        for (int i = 0; i < nt; ++i) {                         // phase 1: scores
+            const int sb = i % SB;
+            wait(&sh.kfull[i & 1], (i >> 1) & 1);
+            if (i >= SB) wait(&sh.sfree[sb], ((i - SB) / SB) & 1);   // softmax read the accumulator
             if (__any_sync(FULL, !ok)) break;
             tc_fence_after();
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-                mma_i8_warp(tbase + C::COL_S + NS * u, tbase + C::COL_AK + 32 * u + 8 * k,
+                mma_i8_warp(tbase + C::COL_S + NS * sb, tbase + C::COL_AK + 32 * (i & 1) + 8 * k,
                             qd + uint64_t((k * 2 * C::CS_Q) >> 4), IDESC_S, k > 0 ? 1u : 0u);
-            tc_commit_warp(&sh.sfull[u]);
+            tc_commit_warp(&sh.sfull[sb]);
         }
-        tc_commit_warp(&sh.mma_done[0]);          // every MMA above has completed before the teardown
-        mbar_wait(&sh.mma_done[0], 0, kWaitNs);
-    } else if (warp == 13) {
-        // =========================================================== ·V MMA
+        ok = __all_sync(FULL, ok);
         const uint32_t pb_s = smem_u32(pb);
-        for (int j = 0; j < ntiles; ++j) {
+        for (int j = 0; j < nt && ok; ++j) {                   // phase 2: ·V
             const int u = j & 1;
-            wait(&sh.vfull, j & 1);
+            wait(&sh.vfull[u], (j >> 1) & 1);
             wait(&sh.pfull[u], (j >> 1) & 1);
             if (__any_sync(FULL, !ok)) break;
             tc_fence_after();
             const uint64_t pd = smem_desc(pb_s + u * 16 * C::CS_P, C::CS_P, 128);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-                tc_mma_ts_warp(tbase + C::COL_O, tbase + C::COL_AV + 8 * k, pd + uint64_t((k * 2 * C::CS_P) >> 4),
-                               IDESC_O, (j > 0 || k > 0) ? 1u : 0u);
+                tc_mma_ts_warp(tbase + C::COL_O, tbase + C::COL_AV + 64 * u + 8 * k,
+                               pd + uint64_t((k * 2 * C::CS_P) >> 4), IDESC_O, (j > 0 || k > 0) ? 1u : 0u);
             tc_commit_warp(&sh.pvdone[u]);
         }
-        tc_commit_warp(&sh.mma_done[1]);
-        mbar_wait(&sh.mma_done[1], 0, kWaitNs);
-    } else if (warp >= 4 && warp < 8) {
-        // ======================================================= key loaders
-        const int ti = tid - 128;                 // token ti of each tile
+        tc_commit_warp(&sh.mma_done);          // every MMA above has completed before the teardown
+        mbar_wait(&sh.mma_done, 0, kWaitNs);
+    } else if (warp >= 4) {
+        // =========================================================== loaders
+        const int ti = tid - 128;                 // token ti (keys) and channel ti (values)
         const int pp_k = ti >> 6, slot_k = ti & 63;
-        auto issue = [&](int i) {
-            uint8_t* st = ring + (i % R) * C::STAGE;
-            const int lp = pg0 + 2 * i + pp_k;
-            const int pg = lp < pg1 ? sh.pages[2 * i + pp_k] : -1;
-            const bool have = pg >= 0;
-            const uint8_t* kb = p.k_codes + (size_t(have ? pg : 0) * p.hkv + h) * (kPage * C::KROW) + slot_k * 16;
-#pragma unroll
-            for (int c = 0; c < C::KROW / 16; ++c)
-                cp16(st + C::ST_K + c * (TILE * 16) + ti * 16, kb + c * (kPage * 16), have);
-        };
-        for (int i = 0; i < R - 1; ++i) {
-            if (i < ntiles) issue(i);
-            cp_commit();
-        }
-        for (int i = 0; i < ntiles; ++i) {
-            if (i + R - 1 < ntiles) issue(i + R - 1);
-            cp_commit();
-            cp_wait<R - 1>();
-            const uint8_t* st = ring + (i % R) * C::STAGE;
-            uint32_t a[32];
-#pragma unroll
-            for (int c = 0; c < C::KROW / 16; ++c) {
-                const uint4 w4 = *reinterpret_cast<const uint4*>(st + C::ST_K + c * (TILE * 16) + ti * 16);
-                unpack_i8<KB>(w4.x, &a[(4 * c + 0) * (8 / KB)]);
-                unpack_i8<KB>(w4.y, &a[(4 * c + 1) * (8 / KB)]);
-                unpack_i8<KB>(w4.z, &a[(4 * c + 2) * (8 / KB)]);
-                unpack_i8<KB>(w4.w, &a[(4 * c + 3) * (8 / KB)]);
-            }
-            if (i >= 2) wait(&sh.sfull[i & 1], ((i - 2) >> 1) & 1);   // score MMA of tile i-2 read the buffer
-            if (__any_sync(FULL, !ok)) break;
-            tc_fence_after();
-            tmem_st32(tbase + lane_off + C::COL_AK + 32 * (i & 1), a);
-            tc_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.kfull[i & 1]);
-        }
-        cp_wait_all();
-    } else if (warp >= 8 && warp < 12) {
-        // ===================================================== value loaders
-        const int ti = tid - 256;                 // value channel ti
-        auto issue = [&](int i) {
-            uint8_t* st = ring + (i % R) * C::STAGE;
-#pragma unroll
-            for (int pp = 0; pp < 2; ++pp) {
-                const int lp = pg0 + 2 * i + pp;
-                const int pg = lp < pg1 ? sh.pages[2 * i + pp] : -1;
+        auto issue = [&](int k) {
+            uint8_t* st = ring + (k % R) * C::STAGE;
+            if (k < nt) {                         // key codes of token ti
+                const int lp = pg0 + 2 * k + pp_k;
+                const int pg = lp < pg1 ? sh.pages[2 * k + pp_k] : -1;
                 const bool have = pg >= 0;
-                const uint8_t* vb = p.v_codes + (size_t(have ? pg : 0) * p.hkv + h) * (D * C::VCH);
-                if constexpr (C::VCH >= 16) {
+                const uint8_t* kb = p.k_codes + (size_t(have ? pg : 0) * p.hkv + h) * (kPage * C::KROW) + slot_k * 16;
 #pragma unroll
-                    for (int c = 0; c < C::VCH / 16; ++c)
-                        cp16(st + C::ST_V + (pp * (C::VCH / 16) + c) * (D * 16) + ti * 16, vb + c * (D * 16) + ti * 16,
-                             have);
-                } else {
-                    cp8(st + C::ST_V + ti * 16 + pp * 8, vb + ti * 8, have);
-                }
-            }
-        };
-        for (int i = 0; i < R - 1; ++i) {
-            if (i < ntiles) issue(i);
-            cp_commit();
-        }
-        for (int i = 0; i < ntiles; ++i) {
-            if (i + R - 1 < ntiles) issue(i + R - 1);
-            cp_commit();
-            cp_wait<R - 1>();
-            const uint8_t* st = ring + (i % R) * C::STAGE + C::ST_V;
-            if (i >= 1) wait(&sh.pvdone[(i - 1) & 1], ((i - 1) >> 1) & 1);   // ·V MMA of tile i-1 read the operand
-            if (__any_sync(FULL, !ok)) break;
-            tc_fence_after();
+                for (int c = 0; c < C::KROW / 16; ++c)
+                    cp16(st + c * (TILE * 16) + ti * 16, kb + c * (kPage * 16), have);
+            } else {                              // value codes of channel ti, both pages
+                const int i = k - nt;
 #pragma unroll
-            for (int pp = 0; pp < 2; ++pp) {      // one page (32 columns) at a time
-                uint32_t a[32];
-                if constexpr (VB == 1) {
-                    const uint2 w2 = *reinterpret_cast<const uint2*>(st + ti * 16 + pp * 8);
-                    Unpack<1>::word(w2.x, &a[0]);
-                    Unpack<1>::word(w2.y, &a[VREG]);
-                } else {
+                for (int pp = 0; pp < 2; ++pp) {
+                    const int lp = pg0 + 2 * i + pp;
+                    const int pg = lp < pg1 ? sh.pages[2 * i + pp] : -1;
+                    const bool have = pg >= 0;
+                    const uint8_t* vb = p.v_codes + (size_t(have ? pg : 0) * p.hkv + h) * (D * C::VCH);
+                    if constexpr (C::VCH >= 16) {
 #pragma unroll
-                    for (int c = 0; c < VWP / 4; ++c) {
-                        const uint4 w4 = *reinterpret_cast<const uint4*>(st + (pp * (VWP / 4) + c) * (D * 16) + ti * 16);
-                        Unpack<VB>::word(w4.x, &a[c * 4 * VREG + 0 * VREG]);
-                        Unpack<VB>::word(w4.y, &a[c * 4 * VREG + 1 * VREG]);
-                        Unpack<VB>::word(w4.z, &a[c * 4 * VREG + 2 * VREG]);
-                        Unpack<VB>::word(w4.w, &a[c * 4 * VREG + 3 * VREG]);
+                        for (int c = 0; c < C::VCH / 16; ++c)
+                            cp16(st + (pp * (C::VCH / 16) + c) * (D * 16) + ti * 16, vb + c * (D * 16) + ti * 16, have);
+                    } else {
+                        cp8(st + ti * 16 + pp * 8, vb + ti * 8, have);
                     }
                 }
-                tmem_st32(tbase + lane_off + C::COL_AV + 32 * pp, a);
             }
-            tc_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.vfull);
+        };
+        for (int k = 0; k < R - 1; ++k) {
+            if (k < 2 * nt) issue(k);
+            cp_commit();
+        }
+        for (int k = 0; k < 2 * nt; ++k) {
+            if (k + R - 1 < 2 * nt) issue(k + R - 1);
+            cp_commit();
+            cp_wait<R - 1>();
+            const uint8_t* st = ring + (k % R) * C::STAGE;
+            if (k < nt) {
+                // ---- key codes of tile i -> int8 operand buffer i&1
+                const int i = k;
+                uint32_t a[32];
+#pragma unroll
+                for (int c = 0; c < C::KROW / 16; ++c) {
+                    const uint4 w4 = *reinterpret_cast<const uint4*>(st + c * (TILE * 16) + ti * 16);
+                    unpack_i8<KB>(w4.x, &a[(4 * c + 0) * (8 / KB)]);
+                    unpack_i8<KB>(w4.y, &a[(4 * c + 1) * (8 / KB)]);
+                    unpack_i8<KB>(w4.z, &a[(4 * c + 2) * (8 / KB)]);
+                    unpack_i8<KB>(w4.w, &a[(4 * c + 3) * (8 / KB)]);
+                }
+                // score MMA of tile i-2 done (waiting on tile i-SB: a later phase of the
+                // same barrier cannot complete before this operand is written)
+                if (i >= SB) wait(&sh.sfull[(i - SB) % SB], ((i - SB) / SB) & 1);
+                if (__any_sync(FULL, !ok)) break;
+                tc_fence_after();
+                tmem_st32(tbase + lane_off + C::COL_AK + 32 * (i & 1), a);
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh.kfull[i & 1]);
+            } else {
+                // ---- value codes of tile j -> bf16 operand buffer j&1
+                const int j = k - nt, u = j & 1;
+                const int last = nt - 1;
+                if (j == 0) wait(&sh.sfull[last % SB], (last / SB) & 1);   // every score MMA done
+                if (j == 1) wait(&sh.sfree[last % SB], (last / SB) & 1);   // every score accumulator read
+                if (j >= 2) wait(&sh.pvdone[u], ((j - 2) >> 1) & 1);        // ·V MMA of tile j-2 done
+                if (__any_sync(FULL, !ok)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int pp = 0; pp < 2; ++pp) {      // one page (32 columns) at a time
+                    uint32_t a[32];
+                    if constexpr (VB == 1) {
+                        const uint2 w2 = *reinterpret_cast<const uint2*>(st + ti * 16 + pp * 8);
+                        Unpack<1>::word(w2.x, &a[0]);
+                        Unpack<1>::word(w2.y, &a[VREG]);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < VWP / 4; ++c) {
+                            const uint4 w4 = *reinterpret_cast<const uint4*>(st + (pp * (VWP / 4) + c) * (D * 16) + ti * 16);
+                            Unpack<VB>::word(w4.x, &a[c * 4 * VREG + 0 * VREG]);
+                            Unpack<VB>::word(w4.y, &a[c * 4 * VREG + 1 * VREG]);
+                            Unpack<VB>::word(w4.z, &a[c * 4 * VREG + 2 * VREG]);
+                            Unpack<VB>::word(w4.w, &a[c * 4 * VREG + 3 * VREG]);
+                        }
+                    }
+                    tmem_st32(tbase + lane_off + C::COL_AV + 64 * u + 32 * pp, a);
+                }
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sh.vfull[u]);
+            }
         }
         cp_wait_all();
     } else {
         // =========================================================== softmax
         const int t = tid, pp_t = t >> 6, slot_t = t & 63;
         const int kpos_t = pp_t * kPage + kpos_bf16(slot_t, VB);   // position along the ·V K dimension
-        auto issue = [&](int i) {
-            uint8_t* st = ring + (i % R) * C::STAGE;
+        auto issue = [&](int k) {                 // metadata of token t: keys in phase 1, values in phase 2
+            uint8_t* st = ring + (k % R) * C::STAGE + C::ST_M;
+            const int i = k < nt ? k : k - nt;
             const int lp = pg0 + 2 * i + pp_t;
             const int pg = lp < pg1 ? sh.pages[2 * i + pp_t] : -1;
             const bool have = pg >= 0;
             const size_t ph = size_t(have ? pg : 0) * p.hkv + h;
-            cp16(st + C::ST_KM + t * 16, p.k_meta + (ph * kPage + slot_t) * NKG, have);
-            cp4(st + C::ST_VM + t * 4, p.v_meta + (ph * kPage + slot_t), have);
+            if (k < nt) cp16(st + t * 16, p.k_meta + (ph * kPage + slot_t) * NKG, have);
+            else cp4(st + t * 16, p.v_meta + (ph * kPage + slot_t), have);   // same bytes as the key step
         };
-        for (int i = 0; i < R - 1; ++i) {
-            if (i < ntiles) issue(i);
+        for (int k = 0; k < R - 1; ++k) {
+            if (k < 2 * nt) issue(k);
             cp_commit();
         }
-        float qsum[NHC][NKG], qs0[NHC];
+        float qsum[NHC][NKG], qs0[NHC], mloc[NHC];
 #pragma unroll
         for (int r = 0; r < NHC; ++r) {
             qs0[r] = sh.qs0[r < g ? r : 0];
+            mloc[r] = -INFINITY;
 #pragma unroll
             for (int grp = 0; grp < NKG; ++grp) qsum[r][grp] = sh.qsum[r < g ? r : 0][grp];
         }
-        float m[NHC], l[NHC], pz[NHC];
-#pragma unroll
-        for (int r = 0; r < NHC; ++r) {
-            m[r] = -INFINITY;
-            l[r] = 0.0f;
-            pz[r] = 0.0f;
-        }
-        for (int j = 0; j < ntiles; ++j) {
-            const int u = j & 1;
-            if (j + R - 1 < ntiles) issue(j + R - 1);
+        // ---- phase 1: scores of every tile, into shared memory
+        for (int i = 0; i < nt; ++i) {
+            if (i + R - 1 < 2 * nt) issue(i + R - 1);
             cp_commit();
             cp_wait<R - 1>();
-            const uint8_t* st = ring + (j % R) * C::STAGE;
-            const uint4 km4 = *reinterpret_cast<const uint4*>(st + C::ST_KM + t * 16);
-            const uint32_t vmw = *reinterpret_cast<const uint32_t*>(st + C::ST_VM + t * 4);
-            const int lp = pg0 + 2 * j + pp_t;
-            const bool valid = lp < pg1 && sh.pages[2 * j + pp_t] >= 0 && lp * kPage + slot_t < Lq;
-            // ---- scores of token t from the s32 products, two heads at a time
+            const uint4 km4 = *reinterpret_cast<const uint4*>(ring + (i % R) * C::STAGE + C::ST_M + t * 16);
+            const int lp = pg0 + 2 * i + pp_t;
+            const bool valid = lp < pg1 && sh.pages[2 * i + pp_t] >= 0 && lp * kPage + slot_t < Lq;
             const uint32_t kmw[NKG] = {km4.x, km4.y, km4.z, km4.w};
             float ksc[NKG], kzp[NKG];
 #pragma unroll
@@ -852,18 +853,15 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
                 ksc[grp] = f.x;
                 kzp[grp] = KB == 8 ? fmaf(128.0f, f.x, f.y) : f.y;   // folds the -128 code offset
             }
-            const float2 vf = meta_f2(vmw);
-            const float vsc = valid ? vf.x : 0.0f;
-            const float vzp = valid ? vf.y : 0.0f;                       // value codes are exact bf16
-            wait(&sh.sfull[u], (j >> 1) & 1);
+            const int sb = i % SB;
+            wait(&sh.sfull[sb], (i / SB) & 1);
+            if (__any_sync(FULL, !ok)) break;
             tc_fence_after();
-            float sc[NHC];
-            bool exceed = false;
 #pragma unroll
             for (int hp = 0; hp < NHC / 2; ++hp) {
                 uint32_t ds[24];
 #pragma unroll
-                for (int c = 0; c < 3; ++c) tmem_ld8(tbase + lane_off + C::COL_S + NS * u + 24 * hp + 8 * c, &ds[8 * c]);
+                for (int c = 0; c < 3; ++c) tmem_ld8(tbase + lane_off + C::COL_S + NS * sb + 24 * hp + 8 * c, &ds[8 * c]);
                 tc_wait_ld();
 #pragma unroll
                 for (int rr = 0; rr < 2; ++rr) {
@@ -882,62 +880,52 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
                         a1 = fmaf(ksc[grp], dot, a1);
                         a2 = fmaf(kzp[grp], qsum[r][grp], a2);
                     }
-                    sc[r] = (valid && r < g) ? fmaf(a1, qs0[r], a2) * scale_log2 : -INFINITY;
-                    exceed |= sc[r] > m[r] + kLazyMax;
+                    const float sc = (valid && r < g) ? fmaf(a1, qs0[r], a2) * scale_log2 : -INFINITY;
+                    scs[(i * NHC + r) * TILE + t] = sc;
+                    mloc[r] = fmaxf(mloc[r], sc);
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.sfree[u]);
-            // ---- running max shared by the 4 softmax warps; the vote also
-            // carries a failed wait, so the 4 warps leave together
-            const int wv = (__any_sync(FULL, exceed) ? 1 : 0) | (__any_sync(FULL, !ok) ? 2 : 0);
-            if (lane == 0) sh.vote[u][warp] = wv;
-            named_sync(1, 128);
-            const int votes = sh.vote[u][0] | sh.vote[u][1] | sh.vote[u][2] | sh.vote[u][3];
-            if (votes & 2) {
-                ok = false;
-                break;
-            }
-            if (votes & 1) {
-                // exact max of the tile; rescale l, pz and the ·V accumulator
+            if (lane == 0) mbar_arrive(&sh.sfree[sb]);
+        }
+        // ---- the split's score maximum per head
+        const int bad1 = __any_sync(FULL, !ok);
 #pragma unroll
-                for (int r = 0; r < NHC; ++r) {
-                    const int k = redux_max_s32(ord_key(sc[r]));
-                    if (lane == 0) sh.smax[u][warp][r] = k;
-                }
-                named_sync(1, 128);
-                float alpha[NHC];
+        for (int r = 0; r < NHC; ++r) {
+            const float wm = warp_max(mloc[r]);
+            if (lane == 0) sh.smax[warp][r] = wm;
+        }
+        if (lane == 0 && bad1) sh.abort = 1;
+        named_sync(1, 128);
+        if (sh.abort) ok = false;
+        float m[NHC], mu[NHC], l[NHC], pz[NHC];
 #pragma unroll
-                for (int r = 0; r < NHC; ++r) {
-                    const int k = max(max(sh.smax[u][0][r], sh.smax[u][1][r]), max(sh.smax[u][2][r], sh.smax[u][3][r]));
-                    const float mnew = fmaxf(m[r], ord_val(k));
-                    alpha[r] = (mnew == -INFINITY) ? 1.0f : ex2(m[r] - mnew);
-                    l[r] *= alpha[r];
-                    pz[r] *= alpha[r];
-                    m[r] = mnew;
-                }
-                if (j >= 1) {
-                    wait(&sh.pvdone[(j - 1) & 1], ((j - 1) >> 1) & 1);   // ·V MMA of tile j-1 done
-                    tc_fence_after();
-                    uint32_t o[16];
-                    tmem_ld16(tbase + lane_off + C::COL_O, o);
-                    tc_wait_ld();
-#pragma unroll
-                    for (int n = 0; n < 16; ++n)
-                        o[n] = __float_as_uint(__uint_as_float(o[n]) * alpha[(n >> 1) < NHC ? (n >> 1) : 0]);
-                    tmem_st16(tbase + lane_off + C::COL_O, o);
-                    tc_wait_st();
-                }
-            }
-            // ---- P' of token t into buffer u (free once the ·V MMA of tile j-2 is done)
-            if (j >= 2) wait(&sh.pvdone[u], ((j - 2) >> 1) & 1);
+        for (int r = 0; r < NHC; ++r) {
+            m[r] = fmaxf(fmaxf(sh.smax[0][r], sh.smax[1][r]), fmaxf(sh.smax[2][r], sh.smax[3][r]));
+            mu[r] = (m[r] == -INFINITY) ? 0.0f : m[r];
+            l[r] = 0.0f;
+            pz[r] = 0.0f;
+        }
+        // ---- phase 2: P' of every tile
+        for (int j = 0; j < nt && ok; ++j) {
+            const int k = nt + j, u = j & 1;
+            if (k + R - 1 < 2 * nt) issue(k + R - 1);
+            cp_commit();
+            cp_wait<R - 1>();
+            const uint32_t vmw = *reinterpret_cast<const uint32_t*>(ring + (k % R) * C::STAGE + C::ST_M + t * 16);
+            const int lp = pg0 + 2 * j + pp_t;
+            const bool valid = lp < pg1 && sh.pages[2 * j + pp_t] >= 0 && lp * kPage + slot_t < Lq;
+            const float2 vf = meta_f2(vmw);
+            const float vsc = valid ? vf.x : 0.0f;
+            const float vzp = valid ? vf.y : 0.0f;                   // value codes are exact bf16
+            if (j >= 2) wait(&sh.pvdone[u], ((j - 2) >> 1) & 1);     // ·V MMA of tile j-2 read buffer u
+            if (__any_sync(FULL, !ok)) break;
             uint8_t* pbu = pb + u * 16 * C::CS_P;
 #pragma unroll
             for (int r = 0; r < NHC; ++r) {
                 if (r >= g) continue;
-                const float mu = (m[r] == -INFINITY) ? 0.0f : m[r];
-                const float pr = ex2(sc[r] - mu);
+                const float pr = ex2(scs[(j * NHC + r) * TILE + t] - mu[r]);
                 l[r] += pr;
                 pz[r] = fmaf(pr, vzp, pz[r]);
                 const float pv = pr * vsc;
@@ -946,13 +934,12 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
                 *reinterpret_cast<uint16_t*>(pbu + b_off_bf16(2 * r + 1, kpos_t, C::CS_P)) = bf16_bits(pv - hi);
             }
             fence_proxy_async();
-            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sh.pfull[u]);
         }
         cp_wait_all();
         // ---- partial of this split: o for channel t, m, l
-        const int last = ntiles - 1;
+        const int last = nt - 1;
         wait(&sh.pvdone[last & 1], (last >> 1) & 1);
         tc_fence_after();
         uint32_t o[16];
@@ -986,7 +973,7 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
     // ------------------------------------------------------------------ teardown
     tc_fence_before();
     __syncthreads();
-    if (warp == 12) {
+    if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tbase, C::TMEM_COLS);
     }
