@@ -182,6 +182,108 @@ __global__ void __launch_bounds__(128) window_write_kernel(Params p, const void*
     }
 }
 
+// Appends of at most kSmallAppend tokens per sequence, no more than the
+// window (the decode step), in one launch: one CTA per (kv-head, sequence),
+// one warp per job.  With n <= W every position leaving the ring is older
+// than L, and the slot it frees receives position pos + W of this call, so a
+// quantize job reads the old row, writes the new token into the same slot,
+// then quantizes the old row.  Ring positions below W (slots that held
+// nothing) are write-only jobs.  Value codes of one channel share 32-bit
+// words across positions: they are merged with atomic and/or, which needs no
+// read round trip and leaves the other positions' bits alone.
+constexpr int kSmallAppend = 8;
+
+template <int D>
+__global__ void __launch_bounds__(128) append_small_kernel(Params p, const void* __restrict__ k_new,
+                                                           const void* __restrict__ v_new, int in_bf16,
+                                                           const int32_t* __restrict__ cu_new,
+                                                           const int32_t* __restrict__ lens) {
+    constexpr int CPL = D / 32;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int L = lens[b];
+    const int c0 = cu_new[b], n = cu_new[b + 1] - c0;
+    if (n <= 0 || L < 0) return;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int q0, q1, nd;
+    if (p.W > 0) {
+        q0 = max(0, L - p.W);
+        q1 = max(0, L + n - p.W);
+        nd = max(0, min(L + n, p.W) - L);        // ring positions whose slot held nothing
+    } else {
+        q0 = L;
+        q1 = L + n;
+        nd = 0;
+    }
+    const int nq = q1 - q0;
+    for (int job = warp; job < nq + nd; job += 4) {
+        if (job >= nq) {                             // write-only ring job
+            const int pos = L + (job - nq);
+            float kx[CPL], vx[CPL];
+            const size_t off = (size_t(c0 + pos - L) * p.hkv + h) * D;
+            load_row<D>(k_new, in_bf16, off, lane, kx);
+            load_row<D>(v_new, in_bf16, off, lane, vx);
+            const size_t wo = win_off(p, b, h, pos) + lane * CPL;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                p.k_win[wo + i] = __float2bfloat16_rn(kx[i]);
+                p.v_win[wo + i] = __float2bfloat16_rn(vx[i]);
+            }
+            continue;
+        }
+        const int pos = q0 + job;
+        float kx[CPL], vx[CPL];
+        if (p.W > 0) {                               // pos < L: the row is in the ring
+            const size_t off = win_off(p, b, h, pos);
+            load_row<D>(p.k_win, 1, off, lane, kx);
+            load_row<D>(p.v_win, 1, off, lane, vx);
+            // the new token pos + W takes over the slot
+            float nk[CPL], nv[CPL];
+            const size_t noff = (size_t(c0 + pos + p.W - L) * p.hkv + h) * D;
+            load_row<D>(k_new, in_bf16, noff, lane, nk);
+            load_row<D>(v_new, in_bf16, noff, lane, nv);
+            const size_t wo = off + lane * CPL;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                p.k_win[wo + i] = __float2bfloat16_rn(nk[i]);
+                p.v_win[wo + i] = __float2bfloat16_rn(nv[i]);
+            }
+        } else {
+            const size_t off = (size_t(c0 + pos - L) * p.hkv + h) * D;
+            load_row<D>(k_new, in_bf16, off, lane, kx);
+            load_row<D>(v_new, in_bf16, off, lane, vx);
+        }
+        const int page = phys_page(p, b, pos / kPage);
+        if (page < 0) continue;
+        if (p.rotate) rotate_warp<D>(kx, p.signs, lane);
+        const int slot = pos % kPage;
+        // ---- keys: token row and metadata
+        uint32_t kc[CPL];
+        const uint32_t km = quantize_warp<D>(kx, p.kg, p.kb, kc);
+        if ((lane * CPL) % p.kg == 0) k_meta_row(p, page, h, slot)[(lane * CPL) / p.kg] = km;
+        uint32_t bitsv = 0;
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) bitsv |= kc[i] << (p.kb * i);
+        const int lane_bits = CPL * p.kb;            // <= 32
+        const int lpw = 32 / lane_bits;              // lanes per 32-bit word
+        bitsv <<= (lane % lpw) * lane_bits;
+        for (int o = 1; o < lpw; o <<= 1) bitsv |= __shfl_xor_sync(FULL, bitsv, o);
+        if (lane % lpw == 0) *k_word(p, page, h, slot, lane / lpw) = bitsv;
+        // ---- values: metadata per token, codes merged into the channel words
+        uint32_t vc[CPL];
+        const uint32_t vm = quantize_warp<D>(vx, p.vg, p.vb, vc);
+        if ((lane * CPL) % p.vg == 0) v_meta_row(p, page, h, slot)[(lane * CPL) / p.vg] = vm;
+        const int per = 32 / p.vb;
+        const uint32_t fmask = (1u << p.vb) - 1u;
+        const int shift = p.vb * (slot % per);
+#pragma unroll
+        for (int i = 0; i < CPL; ++i) {
+            uint32_t* word = v_word(p, page, h, lane * CPL + i, slot / per);
+            atomicAnd(word, ~(fmask << shift));
+            atomicOr(word, (vc[i] & fmask) << shift);
+        }
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(128) rotate_rows_kernel(Params p, const void* __restrict__ k, int in_bf16,
                                                           int rows, float* __restrict__ out) {
@@ -244,6 +346,12 @@ cudaError_t launch_quantize_append(const Params& p, const void* k_new, const voi
                                    const int32_t* cu_new, const int32_t* lens, int max_new,
                                    cudaStream_t s) {
     if (max_new <= 0 || p.batch <= 0) return cudaSuccess;
+    if (max_new <= kSmallAppend && (p.W == 0 || max_new <= p.W)) {
+        const dim3 sgrid(p.hkv, p.batch);
+        if (p.d == 128) append_small_kernel<128><<<sgrid, 128, 0, s>>>(p, k_new, v_new, in_bf16, cu_new, lens);
+        else append_small_kernel<64><<<sgrid, 128, 0, s>>>(p, k_new, v_new, in_bf16, cu_new, lens);
+        return cudaGetLastError();
+    }
     dim3 grid(max_new / 32 + 2, p.hkv, p.batch);
     if (p.d == 128) quantize_pages_kernel<128><<<grid, 128, 0, s>>>(p, k_new, v_new, in_bf16, cu_new, lens);
     else quantize_pages_kernel<64><<<grid, 128, 0, s>>>(p, k_new, v_new, in_bf16, cu_new, lens);

@@ -28,8 +28,8 @@ DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count) {
     const int units = batch * p.hkv > 0 ? batch * p.hkv : 1;
     pl.tc = (g_decode_path != 1 && tc_supported(p)) ? 1 : 0;
     if (pl.tc) {
-        // window CTAs first (slots 0 .. nws-1, 256 window positions each),
-        // then the quantized splits, each a whole number of 128-token tiles:
+        // quantized splits (slots 0 .. splits_q-1), each a whole number of
+        // 128-token tiles, then the window CTAs (256 window positions each):
         // one wave of CTAs where the units allow it, at most 16 tiles per split
         const int win = p.W < max_len ? p.W : max_len;
         pl.window_split = win > 0 ? (win + 255) / 256 : 0;
@@ -50,7 +50,7 @@ DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count) {
         }
         pl.grid_x = pl.window_split + pl.splits_q;
         if (pl.grid_x == 0) pl.grid_x = 1;              // all-empty: one CTA writes zeros
-        pl.window_slot = 0;
+        pl.window_slot = pl.splits_q;                   // first window slot
         pl.total_splits = pl.grid_x;
         return pl;
     }

@@ -546,10 +546,11 @@ __device__ __forceinline__ void window_partial(const Params& p, Shared& sh, uint
 }
 
 // ------------------------------------------------------------------ kernel
-// grid (nws + splits_q, Hkv, B).  blockIdx.x < nws: window CTA covering
-// window positions [Lq + x*256, Lq + (x+1)*256); otherwise quantized split
-// x - nws covering pages [s*pps, (s+1)*pps).  Every CTA writes one partial
-// (m, l, o) per query head into slot blockIdx.x.
+// grid (Hkv, B, splits_q + nws); the block scheduler dispatches in linear
+// order, so the split index is the slowest dimension.  z < splits_q:
+// quantized split z covering pages [z*pps, (z+1)*pps); the nws window CTAs
+// come last and cover window positions [Lq + w*256, Lq + (w+1)*256).  Every
+// CTA writes one partial (m, l, o) per query head into slot z.
 template <int KB, int VB, int NHC>
 __global__ void __launch_bounds__(kThreads, ctas_per_sm(KB, VB, NHC))
 decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, const int32_t* __restrict__ lens,
@@ -571,21 +572,24 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
     uint8_t* ring = smem + LY::OFF_RING;
     float* scs = reinterpret_cast<float*>(smem + LY::OFF_SC);   // [tile][head][token]
 
-    const int b = blockIdx.z, h = blockIdx.y, x = blockIdx.x;
+    const int h = blockIdx.x, b = blockIdx.y, x = blockIdx.z;   // split index outermost: dispatched last
     const int g = p.g, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int L = max(0, min(lens[b], max_len));
     const int Lq = max(0, L - p.W);
     const size_t row0 = (size_t(b) * p.hq + size_t(h) * g) * slots;
 
     // ---- which work this CTA has
-    const bool is_win = x < nws;
+    // quantized splits first, so that they all start in the first wave of
+    // CTAs; the short window CTAs fill the remaining slots and the tail
+    const int nsq = (int)gridDim.z - nws;
+    const bool is_win = x >= nsq;
     int w0 = 0, w1 = 0, pg0 = 0, pg1 = 0, ntiles = 0;
     if (is_win) {
-        w0 = Lq + x * kWinPerSplit;
+        w0 = Lq + (x - nsq) * kWinPerSplit;
         w1 = min(L, w0 + kWinPerSplit);
     } else {
         const int npg = (Lq + kPage - 1) / kPage;
-        pg0 = (x - nws) * pps;
+        pg0 = x * pps;
         pg1 = min(npg, pg0 + pps);
         ntiles = pg1 > pg0 ? (pg1 - pg0 + 1) / 2 : 0;
     }

@@ -21,7 +21,7 @@ cudaError_t launch_one(const Params& p, const void* q, int q_bf16, const int32_t
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
-    const dim3 grid(pl.grid_x, p.hkv, p.batch);
+    const dim3 grid(p.hkv, p.batch, pl.grid_x);   // split index outermost
     kern<<<grid, kThreads, LY::TOTAL, s>>>(p, q, q_bf16, lens, max_len, sl2, ws_o, ws_ml, pl.pages_per_split,
                                            pl.window_split, pl.total_splits);
     return cudaGetLastError();

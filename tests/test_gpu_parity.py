@@ -192,3 +192,26 @@ def test_rotation_with_window(window):
     pair.ocache.layout = pair.olay
     pair.ocache._signs = np.ascontiguousarray(pair.signs)
     pair.check_decode()
+
+
+@pytest.mark.parametrize("window,n,in_dtype", [(0, 3, wl.DT_BF16), (8, 8, wl.DT_BF16), (64, 2, wl.DT_BF16),
+                                               (5, 5, wl.DT_F32), (100, 1, wl.DT_BF16), (3, 1, wl.DT_F32)])
+def test_small_appends_after_prefill(window, n, in_dtype):
+    """Appends of n <= 8 tokens per sequence, at most the window, take the
+    single-launch append path: ring slots are read, refilled with the new
+    tokens and the old rows quantized in one pass; value words are merged
+    bit-field by bit-field.  Cache bytes stay bit-identical to the oracle."""
+    w = small(window=window, ragged=(1, 300), in_dtype=in_dtype)
+    lens = wl.lengths(w)
+    lens[0] = 0                                        # an empty sequence that starts filling
+    lens[1] = min(window, 3)                           # a ring that is not yet full
+    steps = 4
+    pair = Pair(w, lens, steps=steps * n + 8)
+    pair.prefill()
+    for s in range(steps):
+        toks = [wl.new_tokens(w, 100 + s * n + i) for i in range(n)]
+        k = np.stack([t[0] for t in toks], axis=1).reshape(w.batch * n, w.num_kv_heads, w.head_dim)
+        v = np.stack([t[1] for t in toks], axis=1).reshape(w.batch * n, w.num_kv_heads, w.head_dim)
+        pair.append(k, v, np.arange(w.batch + 1, dtype=np.int32) * n)
+        pair.compare_cache()
+        pair.check_decode(step=s)
