@@ -195,12 +195,12 @@ int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache,
                          void* workspace, size_t workspace_bytes, kvq_stream_t stream);
 
 /* Bytes of the library's static decode scratch (per device). */
-#define KVQ_STATIC_SCRATCH_BYTES (8u * 1024u * 1024u)
+#define KVQ_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
 
 /* kvq_decode_attention without a caller-supplied workspace.  The pages
  * have no counterpart to this call: it is a deployment convenience.  The
  * split partials live in a file-scope static device array of
- * KVQ_STATIC_SCRATCH_BYTES (8 MiB, 256-byte aligned) that the library
+ * KVQ_STATIC_SCRATCH_BYTES (16 MiB, 256-byte aligned) that the library
  * holds in each device's context.  Its address is looked up once per
  * device, on that device's first call.  The call allocates and frees
  * nothing.
@@ -208,7 +208,7 @@ int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache,
  * plus one case: KVQ_ERR_WORKSPACE, with nothing enqueued, when
  * kvq_decode_workspace_bytes(layout, cache->batch, max_len) exceeds
  * KVQ_STATIC_SCRATCH_BYTES.  For scale: batch 64 at lengths up to 16384
- * with 40/8 heads needs 1.3 MB.
+ * with 40/8 heads needs 12 MB.
  * Nothing needs to start at zero: each call writes every partial before
  * its combine step reads it.
  * One scratch array serves every call on a device.  Calls whose GPU

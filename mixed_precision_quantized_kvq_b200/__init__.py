@@ -24,7 +24,7 @@ KVQ_ERR_WORKSPACE = -3
 KVQ_ERR_CUDA = -4
 KVQ_F32 = 0
 KVQ_BF16 = 1
-KVQ_STATIC_SCRATCH_BYTES = 8 * 1024 * 1024
+KVQ_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 PAGE_SIZE = 64
 
 

@@ -29,10 +29,11 @@ DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count) {
     pl.tc = (g_decode_path != 1 && tc_supported(p)) ? 1 : 0;
     if (pl.tc) {
         // quantized splits (slots 0 .. splits_q-1), each a whole number of
-        // 128-token tiles, then the window CTAs (256 window positions each):
+        // 128-token tiles, then the window CTAs (64 window positions each, short
+        // enough to run in the slots the quantized splits leave free):
         // one wave of CTAs where the units allow it, at most 16 tiles per split
         const int win = p.W < max_len ? p.W : max_len;
-        pl.window_split = win > 0 ? (win + 255) / 256 : 0;
+        pl.window_split = win > 0 ? (win + kTcWindowPerCta - 1) / kTcWindowPerCta : 0;
         const int slots = sm_count * tc_ctas_per_sm(p);
         const int tiles = (npages + 1) / 2;
         if (npages == 0) {

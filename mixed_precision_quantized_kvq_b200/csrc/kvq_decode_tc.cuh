@@ -53,7 +53,7 @@ constexpr int NKG = 4;                        // key groups of 32 channels
 constexpr int kThreads = 288;
 constexpr int kMaxPagesPerSplit = 256;
 constexpr int kMaxTiles = 16;                 // tiles per quantized split (scores are kept in shared memory)
-constexpr int kWinPerSplit = 256;             // window positions per window CTA
+constexpr int kWinPerSplit = kTcWindowPerCta;   // window positions per window CTA (one chunk)
 constexpr int WCH = 64;                       // window positions per chunk
 constexpr int kWinSmem = 2 * WCH * D * 2;     // key and value rows of a chunk
 constexpr uint64_t kWaitNs = 2000000000ull;
@@ -549,7 +549,7 @@ __device__ __forceinline__ void window_partial(const Params& p, Shared& sh, uint
 // grid (Hkv, B, splits_q + nws); the block scheduler dispatches in linear
 // order, so the split index is the slowest dimension.  z < splits_q:
 // quantized split z covering pages [z*pps, (z+1)*pps); the nws window CTAs
-// come last and cover window positions [Lq + w*256, Lq + (w+1)*256).  Every
+// come last and cover window positions [Lq + w*64, Lq + (w+1)*64).  Every
 // CTA writes one partial (m, l, o) per query head into slot z.
 template <int KB, int VB, int NHC>
 __global__ void __launch_bounds__(kThreads, ctas_per_sm(KB, VB, NHC))

@@ -14,6 +14,7 @@ namespace kvq {
 
 constexpr int kPage = 64;          // tokens per page
 constexpr int kMaxGqa = 8;         // query heads per kv-head
+constexpr int kTcWindowPerCta = 64; // window positions per window CTA of the tensor-core decode
 
 // Flat copy of kvq_layout + kvq_cache with the derived strides kernels use.
 struct Params {

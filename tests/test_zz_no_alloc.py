@@ -67,10 +67,10 @@ def test_two_calls_in_a_row_match_workspace_entry_point(path):
 
 
 def test_rejects_problem_larger_than_scratch():
-    """batch 512 x 32 query heads needs more than 8 MiB of partials: refused on
+    """batch 1024 x 32 query heads needs more than 16 MiB of partials: refused on
     the host with KVQ_ERR_WORKSPACE, nothing launched, outputs untouched."""
     lay = kvq.Layout(128, 32, 8, 4, 2, 32, 128, 64, 0)
-    batch, max_len = 512, 4096
+    batch, max_len = 1024, 4096
     assert kvq.kvq_decode_workspace_bytes(lay, batch, max_len) > kvq.KVQ_STATIC_SCRATCH_BYTES
     pt = torch.full((batch, 1), -1, dtype=torch.int32, device="cuda")
     cache = kvq.PagedCache.allocate(lay, pt, 1)
