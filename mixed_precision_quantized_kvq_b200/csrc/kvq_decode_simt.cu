@@ -349,14 +349,26 @@ __global__ void __launch_bounds__(128) combine_kernel(int rows, int S, const flo
     for (int i = 0; i < CPL; ++i) acc[i] = 0.0f;
     float lsum = 0.0f;
     if (M != -INFINITY) {
-        for (int s = 0; s < S; ++s) {
-            const float m = ml[2 * s];
-            if (m == -INFINITY) continue;
-            const float w = exp2f(m - M);
-            lsum = fmaf(ml[2 * s + 1], w, lsum);
-            const float* os = ws_o + (size_t(row) * S + s) * D + lane * CPL;
+        // four splits per round, every load of the round issued before use;
+        // a split with m = -inf (no positions) has o = 0 and weight 0
+        for (int s0 = 0; s0 < S; s0 += 4) {
+            float mv[4], lv[4], ov[4][CPL];
 #pragma unroll
-            for (int i = 0; i < CPL; ++i) acc[i] = fmaf(os[i], w, acc[i]);
+            for (int u = 0; u < 4; ++u) {
+                const bool in = s0 + u < S;
+                mv[u] = in ? ml[2 * (s0 + u)] : -INFINITY;
+                lv[u] = in ? ml[2 * (s0 + u) + 1] : 0.0f;
+                const float* os = ws_o + (size_t(row) * S + (in ? s0 + u : 0)) * D + lane * CPL;
+#pragma unroll
+                for (int i = 0; i < CPL; ++i) ov[u][i] = in ? os[i] : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float w = (mv[u] == -INFINITY) ? 0.0f : exp2f(mv[u] - M);
+                lsum = fmaf(lv[u], w, lsum);
+#pragma unroll
+                for (int i = 0; i < CPL; ++i) acc[i] = fmaf(ov[u][i], w, acc[i]);
+            }
         }
     }
     float* o = out + size_t(row) * D + lane * CPL;
