@@ -147,8 +147,8 @@ size_t kvq_decode_workspace_bytes(const kvq_layout* layout, int batch, int max_l
 /* Select the decode kernel family for subsequent kvq_decode_attention and
  * kvq_decode_workspace_bytes calls (process-wide):
  *   0  automatic (default): tensor-core kernel where the layout supports it
- *      (head_dim 128, key groups of 32, value groups of 128, bit pairs
- *      K/V in {4/2, 4/4, 8/8, 2/4, 2/2, 1/2}), CUDA-core kernel otherwise
+ *      (head_dim 128, key groups of 32, value groups of 128, any key and
+ *      value bit widths), CUDA-core kernel otherwise
  *   1  CUDA-core kernel for every layout
  *   2  same as 0 (tensor cores where supported)
  * Not thread-safe with concurrent calls; query workspace sizes after

@@ -231,6 +231,7 @@ __global__ void __launch_bounds__(128) append_small_kernel(Params p, const void*
             continue;
         }
         const int pos = q0 + job;
+        const int page = phys_page(p, b, pos / kPage);   // issued with the row loads below
         float kx[CPL], vx[CPL];
         if (p.W > 0) {                               // pos < L: the row is in the ring
             const size_t off = win_off(p, b, h, pos);
@@ -252,7 +253,6 @@ __global__ void __launch_bounds__(128) append_small_kernel(Params p, const void*
             load_row<D>(k_new, in_bf16, off, lane, kx);
             load_row<D>(v_new, in_bf16, off, lane, vx);
         }
-        const int page = phys_page(p, b, pos / kPage);
         if (page < 0) continue;
         if (p.rotate) rotate_warp<D>(kx, p.signs, lane);
         const int slot = pos % kPage;

@@ -3,6 +3,8 @@ library (through its C ABI) and the CPU oracle, and their outputs are
 compared.  No expected value comes from the CUDA side."""
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -103,6 +105,14 @@ class Pair:
     def check_decode(self, step: int = 0):
         qr, out, lse = self.decode(step)
         ref, ref_lse = self.oracle_decode(qr)
+        log = os.environ.get("KVQ_PARITY_LOG")
+        if log:                                   # optional record of the errors (max abs, max rel)
+            err = np.abs(np.asarray(out, np.float64) - ref)
+            rel = err / np.maximum(np.abs(ref), 1e-30)
+            with open(log, "a") as f:
+                f.write(f"{os.environ.get('PYTEST_CURRENT_TEST', '?').split(' ')[0]} step {step}: "
+                        f"max_abs {err.max() if err.size else 0.0:.3e} "
+                        f"max_rel(|ref|>1e-2) {rel[np.abs(ref) > 1e-2].max() if (np.abs(ref) > 1e-2).any() else 0.0:.3e}\n")
         check_close(out, ref, "out")
         finite = np.isfinite(ref_lse)
         assert np.array_equal(np.isfinite(lse), finite)
