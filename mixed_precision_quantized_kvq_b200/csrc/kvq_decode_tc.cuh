@@ -175,22 +175,6 @@ __device__ __forceinline__ float warp_sum(float v) {
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
     return v;
 }
-__device__ __forceinline__ uint32_t redux_max_u32(uint32_t v) {
-    uint32_t r;
-    asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
-    return r;
-}
-__device__ __forceinline__ int redux_max_s32(int v) {
-    int r;
-    asm volatile("redux.sync.max.s32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
-    return r;
-}
-// order-preserving map of floats onto signed integers, and back
-__device__ __forceinline__ int ord_key(float x) {
-    const int b = __float_as_int(x);
-    return b ^ ((b >> 31) & 0x7FFFFFFF);
-}
-__device__ __forceinline__ float ord_val(int k) { return __int_as_float(k ^ ((k >> 31) & 0x7FFFFFFF)); }
 __device__ __forceinline__ int rni(float x) {
     int r;
     asm("cvt.rni.s32.f32 %0, %1;" : "=r"(r) : "f"(x));
@@ -351,17 +335,11 @@ struct Unpack<8> {
     }
 };
 
-// position (along the MMA K dimension) of element i of a packed run, and
-// the element at a K position: inverse permutations of the unpack order
+// position (along the MMA K dimension) of element i of a packed run of value codes
 __host__ __device__ __forceinline__ int kpos_bf16(int i, int bits) {
     const int per = 32 / bits, half = per / 2;
     const int w = i / per, r = i % per;
     return w * per + 2 * (r % half) + r / half;
-}
-__host__ __device__ __forceinline__ int elem_at_bf16(int pos, int bits) {
-    const int per = 32 / bits, half = per / 2;
-    const int w = pos / per, r = pos % per;
-    return w * per + (r >> 1) + (r & 1) * half;
 }
 // byte offset of element (row n, K position pos) in a K-major B operand
 // stored as [k step][half][row][8 x bf16] with chunk stride cs
@@ -372,11 +350,6 @@ __device__ __forceinline__ int b_off_bf16(int n, int pos, int cs) {
 
 __device__ __forceinline__ uint16_t bf16_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
 
-template <int N>
-__device__ __forceinline__ void cp_wait_n() {
-    if constexpr (N <= 0) cp_wait<0>();
-    else cp_wait<N>();
-}
 
 static __device__ void write_empty_partial(int g, float* ws_o, float* ws_ml, size_t row0, int slots, int slot) {
     for (int i = threadIdx.x; i < g * D; i += blockDim.x) {
