@@ -116,10 +116,37 @@ def table(rows) -> str:
     return "\n".join(out)
 
 
+def grid(length: int = 4096):
+    """Errors of every (key bits >= value bits, key group, value group) setting
+    at head_dim 128 on the sweep workload's distribution: the table the
+    memory-budget planner reads."""
+    out = []
+    for kb in (8, 4, 2, 1):
+        for vb in (8, 4, 2, 1):
+            if vb > kb:
+                continue
+            for kg in (32, 64, 128):
+                for vg in (64, 128):
+                    r = measure(wl.SWEEP.with_(k_group=kg, v_group=vg), kb, vb, length=length)
+                    r.update(k_group=kg, v_group=vg)
+                    out.append(r)
+    return out
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--length", type=int, default=16384, help="tokens of the sequence")
+    ap.add_argument("--grid-json", help="write the planner's error table (JSON) to this path and exit")
     args = ap.parse_args(argv)
+    if args.grid_json:
+        import json
+        rows = grid(min(args.length, 4096))
+        keep = ("k_bits", "v_bits", "k_group", "v_group", "tokens", "max_abs", "mean_abs", "score_max_abs", "tv_max")
+        with open(args.grid_json, "w") as f:
+            json.dump({"source": "python -m oracle.error_report --grid-json (oracle quantizer, fp64 attention, "
+                                 "sweep workload distribution, one sequence, head_dim 128, 32/8 heads)",
+                       "rows": [{k: r[k] for k in keep} for r in rows]}, f, indent=1)
+        return
     rows = [measure(wl.SWEEP, kb, vb, length=args.length) for kb, vb in wl.SWEEP_BITS]
     print(f"sweep workload, one sequence of {args.length} tokens, 32/8 heads, d128, key groups 32, "
           "value groups 128; outlier key channels x10\n")
