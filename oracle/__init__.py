@@ -87,6 +87,8 @@ def lib():
         L.kvqo_attention_dense.argtypes = [P, P, P, C.c_int, C.c_int, C.c_double, P, P]
         L.kvqo_decode_attention.argtypes = [C.POINTER(_Layout), C.POINTER(_Cache), P, C.c_int,
                                             P, C.c_double, P, P]
+        L.kvqo_prefill_attention.argtypes = [C.POINTER(_Layout), C.POINTER(_Cache), P, C.c_int,
+                                             P, P, C.c_double, P, P]
         L.kvqo_num_threads.restype = C.c_int
         L.kvqo_set_num_threads.argtypes = [C.c_int]
         _lib = L
@@ -283,6 +285,25 @@ class Cache:
                                          float(sm_scale), _p(out), _p(lse))
         if rc != 0:
             raise ValueError(f"oracle attention failed: {rc}")
+        return out, lse
+
+    def prefill_attention(self, q, q_dtype: int, cu_q, lens, sm_scale: float):
+        """Causal attention of a chunk of new queries (rows cu_q[b]..cu_q[b+1]
+        of q [total_q][Hq][d]) whose keys and values are the newest positions
+        of each sequence; query i of sequence b sees positions
+        [0, lens[b] - n_b + i].  Returns out [total_q][Hq][d], lse [total_q][Hq]."""
+        lay, cache = self._structs()
+        q = np.ascontiguousarray(q)
+        cu = np.ascontiguousarray(cu_q, dtype=np.int32)
+        ln = np.ascontiguousarray(lens, dtype=np.int32)
+        Hq, d = self.layout.num_q_heads, self.layout.head_dim
+        total = int(cu[-1])
+        out = np.zeros((total, Hq, d), np.float64)
+        lse = np.zeros((total, Hq), np.float64)
+        rc = lib().kvqo_prefill_attention(C.byref(lay), C.byref(cache), _p(q), q_dtype, _p(cu), _p(ln),
+                                          float(sm_scale), _p(out), _p(lse))
+        if rc != 0:
+            raise ValueError(f"oracle prefill attention failed: {rc}")
         return out, lse
 
 

@@ -613,12 +613,70 @@ void kvqo_attention_dense(const double* q, const double* K, const double* V,
     free(s);
 }
 
+/* Softmax attention of one query over positions [0, n) of the reconstructed
+ * rows K, V [n][d] of one (sequence, kv-head), fp64 ([P1] "Error pada key
+ * masuk sebelum softmax": s = q K^T * sm_scale, a = softmax(s), o = a V,
+ * lse = log sum exp(s)).  Quantized keys of a rotating layout are in the
+ * rotated domain, so rows with quant[t] set are scored with the rotated
+ * query qr; the other rows (bf16 window) with the plain query qd. */
+static void attend_prefix(const kvqo_layout* l, const double* qd, const double* qr,
+                          const double* K, const double* V, const int* quant, int n,
+                          double sm_scale, double* o, double* lo)
+{
+    const int d = l->head_dim;
+    if (!l->rotate_keys) {
+        kvqo_attention_dense(qd, K, V, n, d, sm_scale, o, lo);
+        return;
+    }
+    for (int j = 0; j < d; ++j) o[j] = 0.0;
+    if (n <= 0) { *lo = -INFINITY; return; }
+    double* s = (double*)malloc(sizeof(double) * (size_t)n);
+    double mx = -INFINITY, sum = 0.0;
+    for (int t = 0; t < n; ++t) {
+        const double* qq = quant[t] ? qr : qd;
+        double acc = 0.0;
+        for (int j = 0; j < d; ++j) acc += qq[j] * K[(size_t)t * d + j];
+        s[t] = acc * sm_scale;
+        if (s[t] > mx) mx = s[t];
+    }
+    for (int t = 0; t < n; ++t) { s[t] = exp(s[t] - mx); sum += s[t]; }
+    for (int t = 0; t < n; ++t) {
+        double a = s[t] / sum;
+        for (int j = 0; j < d; ++j) o[j] += a * V[(size_t)t * d + j];
+    }
+    *lo = mx + log(sum);
+    free(s);
+}
+
+/* Reconstruct positions [0, L) of (b, kv-head h) into K, V [L][d] (fp64) and
+ * quant[L] (1 = from a page, 0 = from the bf16 window). */
+static void reconstruct_all(const kvqo_layout* l, const kvqo_cache* c, int b, int h, int L,
+                            double* K, double* V, int* quant)
+{
+    const int d = l->head_dim;
+    float kf[256], vf[256];
+    for (int pos = 0; pos < L; ++pos) {
+        quant[pos] = reconstruct(l, c, b, h, L, pos, kf, vf);
+        for (int j = 0; j < d; ++j) {
+            K[(size_t)pos * d + j] = kf[j];
+            V[(size_t)pos * d + j] = vf[j];
+        }
+    }
+}
+
+/* query row (fp64) of q-head hq of query row r of q [rows][Hq][d], and its
+ * rotation when the layout rotates keys */
+static void load_query(const kvqo_layout* l, const void* q, int q_dtype, size_t r, int hq,
+                       double* qd, double* qr)
+{
+    const int d = l->head_dim, Hq = l->num_q_heads;
+    for (int j = 0; j < d; ++j) qd[j] = load_in(q, q_dtype, (r * Hq + hq) * d + j);
+    if (l->rotate_keys) kvqo_rotate_f64(qd, l->rot_signs, d, qr);
+}
+
 /* Decode attention of one query token per sequence over the cache, fp64.
  * q [B][Hq][d] (q_dtype 0 = fp32, 1 = bf16); query head hq reads kv-head
- * hq / (Hq/Hkv).  Quantized keys of a rotating layout are in the rotated
- * domain, so those positions are scored with the rotated query (rotation
- * in fp64); window positions use the unrotated query.  out [B][Hq][d],
- * lse [B][Hq] (natural log). */
+ * hq / (Hq/Hkv).  out [B][Hq][d], lse [B][Hq] (natural log). */
 int kvqo_decode_attention(const kvqo_layout* l, const kvqo_cache* c, const void* q,
                           int q_dtype, const int32_t* lens, double sm_scale,
                           double* out, double* lse)
@@ -634,44 +692,59 @@ int kvqo_decode_attention(const kvqo_layout* l, const kvqo_cache* c, const void*
             double* K = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1) * d);
             double* V = (double*)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1) * d);
             int* quant = (int*)malloc(sizeof(int) * (size_t)(L > 0 ? L : 1));
-            float kf[256], vf[256];
-            for (int pos = 0; pos < L; ++pos) {
-                quant[pos] = reconstruct(l, c, b, h, L, pos, kf, vf);
-                for (int j = 0; j < d; ++j) {
-                    K[(size_t)pos * d + j] = kf[j];
-                    V[(size_t)pos * d + j] = vf[j];
-                }
-            }
+            reconstruct_all(l, c, b, h, L, K, V, quant);
             for (int r = 0; r < g; ++r) {
                 int hq = h * g + r;
                 double qd[256], qr[256];
-                for (int j = 0; j < d; ++j)
-                    qd[j] = load_in(q, q_dtype, ((size_t)b * Hq + hq) * d + j);
-                if (l->rotate_keys) kvqo_rotate_f64(qd, l->rot_signs, d, qr);
-                double* o = out + ((size_t)b * Hq + hq) * d;
-                double* lo = lse + (size_t)b * Hq + hq;
-                if (!l->rotate_keys) {
-                    kvqo_attention_dense(qd, K, V, L, d, sm_scale, o, lo);
-                } else {
-                    /* same softmax, with the query matched to each key's domain */
-                    for (int j = 0; j < d; ++j) o[j] = 0.0;
-                    if (L <= 0) { *lo = -INFINITY; continue; }
-                    double* s = (double*)malloc(sizeof(double) * (size_t)L);
-                    double mx = -INFINITY, sum = 0.0;
-                    for (int t = 0; t < L; ++t) {
-                        const double* qq = quant[t] ? qr : qd;
-                        double acc = 0.0;
-                        for (int j = 0; j < d; ++j) acc += qq[j] * K[(size_t)t * d + j];
-                        s[t] = acc * sm_scale;
-                        if (s[t] > mx) mx = s[t];
-                    }
-                    for (int t = 0; t < L; ++t) { s[t] = exp(s[t] - mx); sum += s[t]; }
-                    for (int t = 0; t < L; ++t) {
-                        double a = s[t] / sum;
-                        for (int j = 0; j < d; ++j) o[j] += a * V[(size_t)t * d + j];
-                    }
-                    *lo = mx + log(sum);
-                    free(s);
+                load_query(l, q, q_dtype, (size_t)b, hq, qd, qr);
+                attend_prefix(l, qd, qr, K, V, quant, L, sm_scale,
+                              out + ((size_t)b * Hq + hq) * d, lse + (size_t)b * Hq + hq);
+            }
+            free(K); free(V); free(quant);
+        }
+    return KVQO_OK;
+}
+
+/* Attention of a chunk of new query tokens over the cache (chunked prefill),
+ * causal, fp64.  The chunk's own keys and values were appended first, so
+ * sequence b holds lens[b] positions and its n_b = cu_q[b+1] - cu_q[b]
+ * queries are the newest n_b positions: query i sits at position
+ * p = lens[b] - n_b + i and attends to positions [0, p] as the cache holds
+ * them now (pages or bf16 window; [P1] "Pertumbuhan cache ...": the stored
+ * approximation is what later attention reads).  The pages describe one new
+ * query; extending it to a chunk with a causal mask is the plain reading.
+ * q [total_q][Hq][d] rows cu_q[b] + i; out [total_q][Hq][d],
+ * lse [total_q][Hq].  n_b < 0 or n_b > lens[b] is an argument error. */
+int kvqo_prefill_attention(const kvqo_layout* l, const kvqo_cache* c, const void* q,
+                           int q_dtype, const int32_t* cu_q, const int32_t* lens,
+                           double sm_scale, double* out, double* lse)
+{
+    int rc = check_layout(l);
+    if (rc) return rc;
+    const int d = l->head_dim, H = l->num_kv_heads, Hq = l->num_q_heads, B = c->batch;
+    const int g = Hq / H;
+    for (int b = 0; b < B; ++b) {
+        int n = cu_q[b + 1] - cu_q[b];
+        if (n < 0 || n > lens[b]) return KVQO_ERR_ARG;
+    }
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            int L = lens[b], n = cu_q[b + 1] - cu_q[b];
+            if (n == 0) continue;
+            double* K = (double*)malloc(sizeof(double) * (size_t)L * d);
+            double* V = (double*)malloc(sizeof(double) * (size_t)L * d);
+            int* quant = (int*)malloc(sizeof(int) * (size_t)L);
+            reconstruct_all(l, c, b, h, L, K, V, quant);
+            for (int i = 0; i < n; ++i) {
+                size_t row = (size_t)cu_q[b] + i;
+                int visible = L - n + i + 1;
+                for (int r = 0; r < g; ++r) {
+                    int hq = h * g + r;
+                    double qd[256], qr[256];
+                    load_query(l, q, q_dtype, row, hq, qd, qr);
+                    attend_prefix(l, qd, qr, K, V, quant, visible, sm_scale,
+                                  out + (row * Hq + hq) * d, lse + row * Hq + hq);
                 }
             }
             free(K); free(V); free(quant);

@@ -38,6 +38,7 @@ STREAM_PAGES = 6
 STREAM_SIGNS = 7
 STREAM_NEW_K = 8
 STREAM_NEW_V = 9
+STREAM_CHUNK_Q = 10
 
 PAGE_SIZE = 64
 
@@ -237,6 +238,13 @@ def query(w: Workload, step: int = 0):
     """One query token per sequence: [B][Hq][d] (raw, f32)."""
     q = rng(w.seed, STREAM_Q, step).standard_normal(
         (w.batch, w.num_q_heads, w.head_dim), dtype=np.float32)
+    return _finish(w, q)
+
+
+def chunk_queries(w: Workload, total: int, step: int = 0):
+    """Query rows of a chunk of new tokens, [total][Hq][d] (raw, f32)."""
+    q = rng(w.seed, STREAM_CHUNK_Q, step).standard_normal(
+        (total, w.num_q_heads, w.head_dim), dtype=np.float32)
     return _finish(w, q)
 
 
