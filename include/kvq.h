@@ -222,6 +222,33 @@ int kvq_decode_attention_static_scratch(const kvq_layout* layout, const kvq_cach
                                         int max_len, float sm_scale, float* out, float* lse,
                                         kvq_stream_t stream);
 
+/* Attention of a chunk of new query tokens over the cache (chunked
+ * prefill), causal, dequantization fused into the kernel.  The pages give
+ * attention for one new query ("Kuantisasi KV cache ...", "Error pada key
+ * masuk sebelum softmax": s = qK^T/sqrt(d), a = softmax(s), o = aV) over
+ * the stored approximation ("Pertumbuhan cache ..."); a chunk of n queries
+ * is read as n such queries under a causal mask.
+ * Call kvq_quantize_append with the chunk's keys and values first and
+ * advance lens; then sequence b holds lens[b] positions and its
+ * n_b = cu_q[b+1] - cu_q[b] queries are its newest n_b positions: query i
+ * sits at position lens[b] - n_b + i and attends to positions
+ * [0, lens[b] - n_b + i] (pages below lens[b] - W, the bf16 window above;
+ * with rotate_keys, page keys are scored with the rotated query).
+ * q         device [cu_q[batch]][Hq][d], q_dtype KVQ_BF16 or KVQ_F32
+ * cu_q      device int32 [batch+1], non-decreasing, cu_q[0] == 0
+ * lens      device int32 [batch], positions including the chunk
+ * max_q     host bound: max_q >= every n_b (launch size)
+ * sm_scale  score scale (1/sqrt(d) for standard attention)
+ * out       device fp32 [cu_q[batch]][Hq][d]; lse device fp32
+ *           [cu_q[batch]][Hq] (natural log) or NULL.
+ * Sequences with n_b = 0 are skipped.  A sequence with n_b > lens[b] or
+ * n_b > max_q is skipped too and its output rows are left untouched.
+ * Needs no workspace; allocates nothing. */
+int kvq_prefill_attention(const kvq_layout* layout, const kvq_cache* cache,
+                          const void* q, int q_dtype, const int32_t* cu_q,
+                          const int32_t* lens, int max_q, float sm_scale,
+                          float* out, float* lse, kvq_stream_t stream);
+
 /* Reconstruct the cache to fp32 [batch][Hkv][max_len][d] (check path;
  * "dequantization into temporary storage").  Quantized positions give
  * code*scale+zero (keys in the rotated domain when rotate_keys), window

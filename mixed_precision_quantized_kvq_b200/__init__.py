@@ -72,6 +72,7 @@ def lib() -> C.CDLL:
         L.kvq_decode_attention.argtypes = [LP, CP, P, I, P, I, C.c_float, P, P, P, S, P]
         L.kvq_decode_attention_static_scratch.argtypes = [LP, CP, P, I, P, I, C.c_float, P, P, P]
         L.kvq_dequantize.argtypes = [LP, CP, P, I, P, P, P]
+        L.kvq_prefill_attention.argtypes = [LP, CP, P, I, P, P, I, C.c_float, P, P, P]
         L.kvq_rotate_keys.argtypes = [LP, P, I, I, P, P]
         L.kvq_set_decode_path.argtypes = [I]
         L.kvq_set_decode_path.restype = I
@@ -221,6 +222,16 @@ def kvq_decode_attention_static_scratch(layout: Layout, cache: PagedCache, q: to
           _stream(stream))
 
 
+def kvq_prefill_attention(layout: Layout, cache: PagedCache, q: torch.Tensor, cu_q: torch.Tensor,
+                          lens: torch.Tensor, max_q: int, sm_scale: float, out: torch.Tensor,
+                          lse: Optional[torch.Tensor], stream=None) -> None:
+    """kvq.h kvq_prefill_attention: causal attention of each sequence's chunk
+    of new queries (rows cu_q[b]..cu_q[b+1] of q [total_q][Hq][d]), whose keys
+    and values are already appended, -> out fp32 [total_q][Hq][d], lse fp32."""
+    _call("kvq_prefill_attention", C.byref(layout.c()), C.byref(cache.c()), _ptr(q), _dtype_code(q),
+          _ptr(cu_q), _ptr(lens), int(max_q), C.c_float(sm_scale), _ptr(out), _ptr(lse), _stream(stream))
+
+
 def kvq_dequantize(layout: Layout, cache: PagedCache, lens: torch.Tensor, max_len: int,
                    k_out: torch.Tensor, v_out: torch.Tensor, stream=None) -> None:
     """kvq.h kvq_dequantize: fp32 [B][Hkv][max_len][d] reconstructions."""
@@ -272,5 +283,19 @@ def decode_attention(layout: Layout, cache: PagedCache, q: torch.Tensor, lens: t
     return out, lse
 
 
+def prefill_attention(layout: Layout, cache: PagedCache, q: torch.Tensor, cu_q: torch.Tensor,
+                      lens: torch.Tensor, max_q: int, sm_scale: Optional[float] = None,
+                      want_lse: bool = True):
+    """Allocating convenience wrapper around kvq_prefill_attention."""
+    T, Hq, d = q.shape
+    if sm_scale is None:
+        sm_scale = d ** -0.5
+    out = torch.empty((T, Hq, d), dtype=torch.float32, device=q.device)
+    lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device) if want_lse else None
+    kvq_prefill_attention(layout, cache, q, cu_q, lens, max_q, sm_scale, out, lse)
+    return out, lse
+
+
 __all__ = [n for n in dir() if n.startswith("kvq_")] + [
-    "Layout", "PagedCache", "KVQError", "lib", "decode_attention", "workspace_for", "LIB_PATH"]
+    "Layout", "PagedCache", "KVQError", "lib", "decode_attention", "prefill_attention", "workspace_for",
+    "LIB_PATH"]

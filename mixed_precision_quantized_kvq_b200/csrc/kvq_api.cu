@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "kvq_internal.cuh"
+#include "kvq_prefill.cuh"
 
 namespace {
 
@@ -189,6 +190,22 @@ int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache, const
         return KVQ_ERR_WORKSPACE;
     return cuda_status(kvq::launch_decode(p, q, q_dtype == KVQ_BF16, lens, max_len, sm_scale, out, lse,
                                           workspace, pl, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int kvq_prefill_attention(const kvq_layout* layout, const kvq_cache* cache, const void* q, int q_dtype,
+                          const int32_t* cu_q, const int32_t* lens, int max_q, float sm_scale, float* out,
+                          float* lse, kvq_stream_t stream) {
+    int rc = check_layout(layout);
+    if (rc) return rc;
+    if ((rc = check_cache(layout, cache))) return rc;
+    if (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+    if (!cu_q || !lens || max_q < 0 || !isfinite(sm_scale)) return KVQ_ERR_INVALID_ARG;
+    if (cache->batch > 65535 || layout->num_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
+    if (max_q == 0 || cache->batch == 0) return KVQ_OK;
+    if (!q || !out) return KVQ_ERR_INVALID_ARG;
+    Params p = make_params(layout, cache);
+    return cuda_status(kvq::launch_prefill_attention(p, q, q_dtype == KVQ_BF16, cu_q, lens, max_q, sm_scale, out,
+                                                     lse, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int kvq_dequantize(const kvq_layout* layout, const kvq_cache* cache, const int32_t* lens, int max_len,

@@ -1,0 +1,129 @@
+"""The chunked-prefill kernel body, run on the CPU, against the oracle.
+
+tests/emu/prefill_emu.cpp runs the CUDA kernel's own per-CTA body
+(csrc/kvq_prefill_body.cuh) as host C++: one thread per CUDA thread, real
+barriers, the GPU's warp-butterfly order.  It is built with AddressSanitizer
+and UndefinedBehaviorSanitizer and reads the oracle's cache arrays (the
+library's storage format) from exact-size allocations, so these tests check
+the kernel's indexing, masking and online softmax, and that it stays inside
+every buffer, before it runs on a GPU.  They are not the GPU parity tests
+(tests/test_gpu_prefill.py): the emulator is neither the oracle nor a
+fallback of the library.
+"""
+import os
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads as wl
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+SRC = os.path.join(HERE, "emu", "prefill_emu.cpp")
+CSRC = os.path.join(ROOT, "mixed_precision_quantized_kvq_b200", "csrc")
+ATOL = RTOL = 1e-3
+
+
+def _cuda_include():
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.realpath(nvcc))), "include")
+    return inc if os.path.exists(os.path.join(inc, "cuda_fp16.h")) else None
+
+
+@pytest.fixture(scope="module")
+def emu(tmp_path_factory):
+    inc = _cuda_include()
+    gxx = shutil.which("g++")
+    if not inc or not gxx:
+        pytest.skip("g++ or the CUDA headers are missing")
+    exe = str(tmp_path_factory.mktemp("emu") / "prefill_emu")
+    cmd = [gxx, "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=all",
+           "-fno-omit-frame-pointer", "-I", inc, "-I", CSRC, SRC, "-o", exe, "-pthread"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr[-4000:]
+    return exe
+
+
+def _run(exe, tmp, c: oracle.Cache, q, q_bf16, cu_q, lens, max_q, sm_scale, signs=None):
+    lay = c.layout
+    params = dict(d=lay.head_dim, hq=lay.num_q_heads, hkv=lay.num_kv_heads, kb=lay.k_bits, vb=lay.v_bits,
+                  kg=lay.k_group, vg=lay.v_group, W=lay.window, rotate=int(lay.rotate_keys), batch=c.batch,
+                  max_pages=c.page_table.shape[1], num_pages=c.num_pages, q_bf16=int(q_bf16), max_q=max_q,
+                  sm_scale=repr(float(sm_scale)))
+    with open(os.path.join(tmp, "params.txt"), "w") as f:
+        for k, v in params.items():
+            f.write(f"{k} {v}\n")
+    arrays = dict(k_codes=c.k_codes, v_codes=c.v_codes, k_meta=c.k_meta, v_meta=c.v_meta, k_win=c.k_win,
+                  v_win=c.v_win, page_table=c.page_table, q=q, cu_q=np.asarray(cu_q, np.int32),
+                  lens=np.asarray(lens, np.int32))
+    if signs is not None:
+        arrays["signs"] = np.asarray(signs, np.int8)
+    for k, a in arrays.items():
+        np.ascontiguousarray(a).tofile(os.path.join(tmp, k + ".bin"))
+    env = dict(os.environ, ASAN_OPTIONS="detect_leaks=0")
+    r = subprocess.run([exe, str(tmp)], capture_output=True, text=True, timeout=600, env=env)
+    assert r.returncode == 0, (r.stdout + r.stderr)[-4000:]
+    total = int(cu_q[-1])
+    out = np.fromfile(os.path.join(tmp, "out.bin"), np.float32).reshape(total, lay.num_q_heads, lay.head_dim)
+    lse = np.fromfile(os.path.join(tmp, "lse.bin"), np.float32).reshape(total, lay.num_q_heads)
+    return out, lse
+
+
+CASES = {
+    # name: (workload overrides, chunk cap)
+    "d64_g3_w16_k4v2": (dict(head_dim=64, num_q_heads=6, num_kv_heads=2, k_group=32, v_group=64, window=16), 70),
+    "d128_g4_w0_whole_f32": (dict(window=0, in_dtype=wl.DT_F32), 10 ** 6),
+    "d128_g5_allwindow": (dict(num_q_heads=10, num_kv_heads=2, window=1000), 30),
+    "d128_g4_rot_w16": (dict(window=16, rotate_keys=True, outliers=("student_t", 2, 10.0, 3)), 70),
+    "d64_g1_k8v8_w16": (dict(head_dim=64, num_q_heads=2, num_kv_heads=2, k_bits=8, v_bits=8, k_group=64,
+                             v_group=64, window=16), 50),
+    "d64_g2_k1v1_w8": (dict(head_dim=64, num_q_heads=4, num_kv_heads=2, k_bits=1, v_bits=1, k_group=32,
+                            v_group=32, window=8), 65),
+}
+
+BASE = wl.Workload(name="prefill_emu", batch=3, num_q_heads=8, num_kv_heads=2, head_dim=128, seq_len=0,
+                   k_bits=4, v_bits=2, k_group=32, v_group=128, window=16, ragged=(1, 200),
+                   shuffle_pages=True, outliers=("random", 2, 10.0), seed=5)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_emulated_kernel_matches_oracle(emu, tmp_path, name):
+    over, cap = CASES[name]
+    w = BASE.with_(**over)
+    lens = wl.lengths(w)
+    lens[-1] = max(int(lens[-1]), 130)             # at least three position tiles in one sequence
+    signs = wl.rotation_signs(w) if w.rotate_keys else None
+    pt = wl.page_table(w, np.maximum(0, lens - w.window))
+    c = oracle.Cache(oracle.Layout.from_workload(w, signs), w.batch, pt, max(1, int((pt >= 0).sum())))
+    kr, vr, _, _, cu, _ = wl.prefill(w, lens, with_f32=False)
+    dt = oracle.IN_BF16 if w.in_dtype == wl.DT_BF16 else oracle.IN_F32
+    c.append(kr, vr, dt, cu, np.zeros(w.batch, np.int32))
+    n = np.minimum(lens, cap).astype(np.int32)
+    cu_q = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    q, _ = wl.chunk_queries(w, int(cu_q[-1]))
+    sc = 1 / np.sqrt(w.head_dim)
+    ref_o, ref_l = c.prefill_attention(q, dt, cu_q, lens, sc)
+    out, lse = _run(emu, tmp_path, c, q, dt == oracle.IN_BF16, cu_q, lens, int(n.max()), sc, signs)
+    np.testing.assert_allclose(out, ref_o, atol=ATOL, rtol=RTOL)
+    np.testing.assert_allclose(lse, ref_l, atol=ATOL, rtol=RTOL)
+
+
+def test_emulated_kernel_skips_empty_and_oversized_chunks(emu, tmp_path):
+    w = BASE.with_(window=8)
+    lens = np.array([70, 0, 5], np.int32)
+    pt = wl.page_table(w, np.maximum(0, lens - w.window))
+    c = oracle.Cache(oracle.Layout.from_workload(w), w.batch, pt, max(1, int((pt >= 0).sum())))
+    kr, vr, _, _, cu, _ = wl.prefill(w, lens, with_f32=False)
+    c.append(kr, vr, oracle.IN_BF16, cu, np.zeros(w.batch, np.int32))
+    # sequence 1 sends nothing; sequence 2 sends 7 queries for 5 positions (skipped, rows untouched)
+    cu_q = np.array([0, 20, 20, 27], np.int32)
+    q, _ = wl.chunk_queries(w, 27)
+    out, lse = _run(emu, tmp_path, c, q, True, cu_q, lens, 20, 0.125)
+    ref_o, ref_l = c.prefill_attention(q[:20], oracle.IN_BF16, np.array([0, 20, 20, 20], np.int32),
+                                       np.array([70, 0, 5], np.int32), 0.125)
+    np.testing.assert_allclose(out[:20], ref_o, atol=ATOL, rtol=RTOL)
+    np.testing.assert_allclose(lse[:20], ref_l, atol=ATOL, rtol=RTOL)
+    assert np.all(out[20:] == 0) and np.all(lse[20:] == 0)
