@@ -38,7 +38,7 @@ class _Layout(C.Structure):
     _fields_ = [("head_dim", C.c_int), ("num_q_heads", C.c_int), ("num_kv_heads", C.c_int),
                 ("k_bits", C.c_int), ("v_bits", C.c_int), ("k_group", C.c_int),
                 ("v_group", C.c_int), ("page_size", C.c_int), ("window", C.c_int),
-                ("rotate_keys", C.c_int), ("rot_signs", C.c_void_p)]
+                ("rotate_keys", C.c_int), ("rot_signs", C.c_void_p), ("k_per_channel", C.c_int)]
 
 
 class _Cache(C.Structure):
@@ -215,12 +215,19 @@ class Layout:
     window: int = 0
     rotate_keys: bool = False
     rot_signs: Optional[np.ndarray] = None
+    k_per_channel: bool = False        # key groups of k_group positions of one channel
 
     @classmethod
     def from_workload(cls, w, signs=None):
         return cls(w.head_dim, w.num_q_heads, w.num_kv_heads, w.k_bits, w.v_bits,
                    w.k_group, w.v_group, w.page_size, w.window, bool(w.rotate_keys),
-                   signs)
+                   signs, bool(getattr(w, "k_per_channel", False)))
+
+    @property
+    def ring_slots(self) -> int:
+        """bf16 ring rows per (sequence, kv-head): W, plus k_group - 1 when key
+        groups run along positions (a group waits there until complete)."""
+        return self.window + (self.k_group - 1 if self.k_per_channel else 0)
 
 
 class Cache:
@@ -233,12 +240,15 @@ class Cache:
         d, H, P = layout.head_dim, layout.num_kv_heads, layout.page_size
         self.num_pages = num_pages
         self.k_codes = np.zeros((num_pages, H, P, d * layout.k_bits // 8), np.uint8)
-        self.k_meta = np.zeros((num_pages, H, P, d // layout.k_group, 2), np.uint16)
+        if layout.k_per_channel:
+            self.k_meta = np.zeros((num_pages, H, P // layout.k_group, d, 2), np.uint16)
+        else:
+            self.k_meta = np.zeros((num_pages, H, P, d // layout.k_group, 2), np.uint16)
         self.v_codes = np.zeros((num_pages, H, d, P * layout.v_bits // 8), np.uint8)
         self.v_meta = np.zeros((num_pages, H, P, d // layout.v_group, 2), np.uint16)
-        W = max(layout.window, 0)
-        self.k_win = np.zeros((batch, H, max(W, 1), d), np.uint16)
-        self.v_win = np.zeros((batch, H, max(W, 1), d), np.uint16)
+        R = max(layout.ring_slots, 0)
+        self.k_win = np.zeros((batch, H, max(R, 1), d), np.uint16)
+        self.v_win = np.zeros((batch, H, max(R, 1), d), np.uint16)
         self._signs = (np.ascontiguousarray(layout.rot_signs, dtype=np.int8)
                        if layout.rot_signs is not None else None)
 
@@ -246,7 +256,7 @@ class Cache:
         l = self.layout
         lay = _Layout(l.head_dim, l.num_q_heads, l.num_kv_heads, l.k_bits, l.v_bits,
                       l.k_group, l.v_group, l.page_size, l.window, int(l.rotate_keys),
-                      _p(self._signs) if self._signs is not None else None)
+                      _p(self._signs) if self._signs is not None else None, int(l.k_per_channel))
         cache = _Cache(_p(self.k_codes), _p(self.v_codes), _p(self.k_meta), _p(self.v_meta),
                        _p(self.k_win), _p(self.v_win), _p(self.page_table), self.batch,
                        self.page_table.shape[1])
@@ -310,7 +320,7 @@ class Cache:
 def page_bytes(layout: Layout):
     lay = _Layout(layout.head_dim, layout.num_q_heads, layout.num_kv_heads, layout.k_bits,
                   layout.v_bits, layout.k_group, layout.v_group, layout.page_size,
-                  layout.window, int(layout.rotate_keys), None)
+                  layout.window, int(layout.rotate_keys), None, int(layout.k_per_channel))
     vals = [C.c_size_t() for _ in range(4)]
     rc = lib().kvqo_page_bytes(C.byref(lay), *[C.byref(v) for v in vals])
     if rc != 0:

@@ -304,12 +304,25 @@ void kvqo_rotate(const float* x, const int8_t* signs, int d, float* y)
  * Positions [0, L-W) live in pages (position p in logical page p/P, slot
  * p%P); the last min(W, L) positions live in the ring ([P1] "Pertumbuhan
  * cache ...": recent tokens kept at higher precision).
+ *
+ * Per-channel key groups (k_per_channel = 1; [P1] "Granularitas ...": the
+ * grouping axis may run along token positions): a key group is k_group
+ * consecutive positions of one channel, aligned to k_group inside a page.
+ * Key codes are then stored like value codes (channel runs of P*kb/8 bytes,
+ * chunk-major) and key metadata as
+ *   k_meta  [pages][Hkv][P/kg][d] {u16 scale, u16 zero}.
+ * A group is quantized only when complete and out of the W newest
+ * positions, so positions [0, Q) live in pages with
+ * Q = kg * floor(max(0, L-W) / kg), the rest (at most W + kg - 1
+ * positions) in a ring of W + kg - 1 slots (slot = position mod (W + kg - 1)):
+ * the bf16 window is the residual buffer.
  * ---------------------------------------------------------------------- */
 typedef struct {
     int head_dim, num_q_heads, num_kv_heads;
     int k_bits, v_bits, k_group, v_group, page_size, window;
     int rotate_keys;
     const int8_t* rot_signs;       /* host [head_dim] */
+    int k_per_channel;             /* 1: key groups run along positions */
 } kvqo_layout;
 
 typedef struct {
@@ -327,8 +340,14 @@ static int check_layout(const kvqo_layout* l)
     if (l->head_dim <= 0 || l->head_dim > 256) return KVQO_ERR_UNSUPPORTED;
     if (!valid_bits(l->k_bits) || !valid_bits(l->v_bits)) return KVQO_ERR_UNSUPPORTED;
     if (l->k_group <= 0 || l->v_group <= 0) return KVQO_ERR_UNSUPPORTED;
-    if (l->head_dim % l->k_group || l->head_dim % l->v_group) return KVQO_ERR_UNSUPPORTED;
-    if ((l->head_dim * l->k_bits) % 32) return KVQO_ERR_UNSUPPORTED;
+    if (l->head_dim % l->v_group) return KVQO_ERR_UNSUPPORTED;
+    if (l->k_per_channel) {
+        if (l->page_size <= 0 || l->page_size % l->k_group || l->k_group > 64) return KVQO_ERR_UNSUPPORTED;
+        if ((l->page_size * l->k_bits) % 32 || l->rotate_keys) return KVQO_ERR_UNSUPPORTED;
+    } else {
+        if (l->head_dim % l->k_group) return KVQO_ERR_UNSUPPORTED;
+        if ((l->head_dim * l->k_bits) % 32) return KVQO_ERR_UNSUPPORTED;
+    }
     if (l->page_size <= 0 || (l->page_size * l->v_bits) % 32) return KVQO_ERR_UNSUPPORTED;
     if (l->num_kv_heads <= 0 || l->num_q_heads % l->num_kv_heads) return KVQO_ERR_UNSUPPORTED;
     if (l->window < 0) return KVQO_ERR_ARG;
@@ -344,7 +363,9 @@ int kvqo_page_bytes(const kvqo_layout* l, size_t* kc, size_t* km, size_t* vc, si
     if (rc) return rc;
     size_t per = (size_t)l->num_kv_heads * l->page_size;
     *kc = per * (size_t)(l->head_dim * l->k_bits / 8);
-    *km = per * (size_t)(l->head_dim / l->k_group) * 4;
+    *km = l->k_per_channel
+              ? (size_t)l->num_kv_heads * (size_t)(l->page_size / l->k_group) * (size_t)l->head_dim * 4
+              : per * (size_t)(l->head_dim / l->k_group) * 4;
     *vc = per * (size_t)(l->head_dim * l->v_bits / 8);
     *vm = per * (size_t)(l->head_dim / l->v_group) * 4;
     return KVQO_OK;
@@ -352,6 +373,17 @@ int kvqo_page_bytes(const kvqo_layout* l, size_t* kc, size_t* km, size_t* vc, si
 
 static size_t krow_bytes(const kvqo_layout* l) { return (size_t)l->head_dim * l->k_bits / 8; }
 static size_t vrow_bytes(const kvqo_layout* l) { return (size_t)l->page_size * l->v_bits / 8; }
+static size_t kchan_bytes(const kvqo_layout* l) { return (size_t)l->page_size * l->k_bits / 8; }
+
+/* ring slots of the bf16 window, and the number of positions of a length-L
+ * sequence that live in pages */
+static int ring_slots(const kvqo_layout* l) { return l->window + (l->k_per_channel ? l->k_group - 1 : 0); }
+static int paged_len(const kvqo_layout* l, int L)
+{
+    int q = L - l->window > 0 ? L - l->window : 0;
+    if (l->k_per_channel) q -= q % l->k_group;
+    return q;
+}
 
 /* Code rows longer than 16 bytes are stored in 16-byte chunks, chunk-major
  * inside the (page, kv-head) block: chunk i of token slot t of a key block
@@ -391,6 +423,24 @@ static void v_chan_io(const kvqo_layout* l, const kvqo_cache* c, int page, int h
         else memcpy(run + i * ch, at, ch);
     }
 }
+/* per-channel keys: gather or scatter the packed token run of key channel j */
+static void k_chan_io(const kvqo_layout* l, const kvqo_cache* c, int page, int h, int j,
+                      uint8_t* run, int put)
+{
+    size_t rb = kchan_bytes(l), ch = chunk_of(rb);
+    uint8_t* base = k_block(l, c, page, h);
+    for (size_t i = 0; i < rb / ch; ++i) {
+        uint8_t* at = base + i * (size_t)l->head_dim * ch + (size_t)j * ch;
+        if (put) memcpy(at, run + i * ch, ch);
+        else memcpy(run + i * ch, at, ch);
+    }
+}
+/* per-channel keys: metadata of group grp (slots grp*kg ..) of channel j */
+static uint8_t* k_meta_chan(const kvqo_layout* l, const kvqo_cache* c, int page, int h, int grp, int j)
+{
+    return c->k_meta + ((((size_t)page * l->num_kv_heads + h) * (size_t)(l->page_size / l->k_group) + grp) *
+                            (size_t)l->head_dim + j) * 4;
+}
 static uint8_t* k_meta_row(const kvqo_layout* l, const kvqo_cache* c, int page, int h, int slot)
 {
     return c->k_meta + (((size_t)page * l->num_kv_heads + h) * l->page_size + slot) *
@@ -403,7 +453,8 @@ static uint8_t* v_meta_row(const kvqo_layout* l, const kvqo_cache* c, int page, 
 }
 static uint16_t* win_row(const kvqo_layout* l, uint16_t* win, int b, int h, int pos)
 {
-    return win + (((size_t)b * l->num_kv_heads + h) * l->window + (size_t)(pos % l->window)) * l->head_dim;
+    const int R = ring_slots(l);
+    return win + (((size_t)b * l->num_kv_heads + h) * R + (size_t)(pos % R)) * l->head_dim;
 }
 
 static void put_meta(uint8_t* m, uint16_t scale, uint16_t zero)
@@ -417,29 +468,15 @@ static void get_meta(const uint8_t* m, uint16_t* scale, uint16_t* zero)
     *zero = (uint16_t)(m[2] | (m[3] << 8));
 }
 
-/* quantize one token of one kv-head (fp32 k, v) into its page slot */
-static void quantize_token(const kvqo_layout* l, const kvqo_cache* c, int b, int h,
-                           int pos, const float* k, const float* v)
+/* quantize the value row of one token of one kv-head into its page slot:
+ * groups of v_group channels, codes stored per channel */
+static void quantize_token_values(const kvqo_layout* l, const kvqo_cache* c, int b, int h,
+                                  int pos, const float* v)
 {
     int d = l->head_dim;
     int page = c->page_table[(size_t)b * c->max_pages_per_seq + pos / l->page_size];
     int slot = pos % l->page_size;
-    float kr[256];
     uint8_t codes[256];
-    if (l->rotate_keys) kvqo_rotate(k, l->rot_signs, d, kr);
-    else memcpy(kr, k, sizeof(float) * d);
-    /* keys: groups of k_group channels */
-    uint8_t* km = k_meta_row(l, c, page, h, slot);
-    for (int g = 0; g < d / l->k_group; ++g) {
-        uint16_t s, z;
-        kvqo_quantize_group(kr + g * l->k_group, l->k_group, l->k_bits, &s, &z,
-                            codes + g * l->k_group);
-        put_meta(km + 4 * g, s, z);
-    }
-    uint8_t row[256];
-    kvqo_pack(codes, d, l->k_bits, row);
-    k_row_io(l, c, page, h, slot, row, 1);
-    /* values: groups of v_group channels; codes stored per channel */
     uint8_t* vm = v_meta_row(l, c, page, h, slot);
     for (int g = 0; g < d / l->v_group; ++g) {
         uint16_t s, z;
@@ -452,6 +489,52 @@ static void quantize_token(const kvqo_layout* l, const kvqo_cache* c, int b, int
         v_chan_io(l, c, page, h, j, run, 0);
         set_packed(run, slot, l->v_bits, codes[j]);
         v_chan_io(l, c, page, h, j, run, 1);
+    }
+}
+
+/* quantize one token of one kv-head (fp32 k, v) into its page slot; keys in
+ * groups of k_group channels (rotated first when the layout rotates keys) */
+static void quantize_token(const kvqo_layout* l, const kvqo_cache* c, int b, int h,
+                           int pos, const float* k, const float* v)
+{
+    int d = l->head_dim;
+    int page = c->page_table[(size_t)b * c->max_pages_per_seq + pos / l->page_size];
+    int slot = pos % l->page_size;
+    float kr[256];
+    uint8_t codes[256];
+    if (l->rotate_keys) kvqo_rotate(k, l->rot_signs, d, kr);
+    else memcpy(kr, k, sizeof(float) * d);
+    uint8_t* km = k_meta_row(l, c, page, h, slot);
+    for (int g = 0; g < d / l->k_group; ++g) {
+        uint16_t s, z;
+        kvqo_quantize_group(kr + g * l->k_group, l->k_group, l->k_bits, &s, &z,
+                            codes + g * l->k_group);
+        put_meta(km + 4 * g, s, z);
+    }
+    uint8_t row[256];
+    kvqo_pack(codes, d, l->k_bits, row);
+    k_row_io(l, c, page, h, slot, row, 1);
+    quantize_token_values(l, c, b, h, pos, v);
+}
+
+/* per-channel keys: quantize the keys of positions [g0, g0 + k_group) of
+ * (b, kv-head h), K [k_group][d] fp32; one group per channel */
+static void quantize_key_group(const kvqo_layout* l, const kvqo_cache* c, int b, int h,
+                               int g0, const float* K)
+{
+    const int d = l->head_dim, G = l->k_group;
+    int page = c->page_table[(size_t)b * c->max_pages_per_seq + g0 / l->page_size];
+    int slot0 = g0 % l->page_size;
+    for (int j = 0; j < d; ++j) {
+        float x[64];
+        uint8_t codes[64], run[64];
+        uint16_t s, z;
+        for (int t = 0; t < G; ++t) x[t] = K[(size_t)t * d + j];
+        kvqo_quantize_group(x, G, l->k_bits, &s, &z, codes);
+        put_meta(k_meta_chan(l, c, page, h, slot0 / G, j), s, z);
+        k_chan_io(l, c, page, h, j, run, 0);
+        for (int t = 0; t < G; ++t) set_packed(run, slot0 + t, l->k_bits, codes[t]);
+        k_chan_io(l, c, page, h, j, run, 1);
     }
 }
 
@@ -474,36 +557,59 @@ int kvqo_quantize_append(const kvqo_layout* l, const kvqo_cache* c,
     int rc = check_layout(l);
     if (rc) return rc;
     if (!c || !k_new || !v_new || !cu_new || !lens) return KVQO_ERR_ARG;
-    const int d = l->head_dim, H = l->num_kv_heads, W = l->window;
+    const int d = l->head_dim, H = l->num_kv_heads;
     int B = c->batch;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int b = 0; b < B; ++b) {
         int L = lens[b];
         int n = cu_new[b + 1] - cu_new[b];
-        int q0 = L - W > 0 ? L - W : 0;
-        int q1 = L + n - W > 0 ? L + n - W : 0;
-        float k[256], v[256];
-        for (int pos = q0; pos < q1; ++pos) {
-            for (int h = 0; h < H; ++h) {
-                if (pos < L) {            /* leaving the ring */
-                    uint16_t* kw = win_row(l, c->k_win, b, h, pos);
-                    uint16_t* vw = win_row(l, c->v_win, b, h, pos);
-                    for (int j = 0; j < d; ++j) {
-                        k[j] = kvqo_bf16_to_f32(kw[j]);
-                        v[j] = kvqo_bf16_to_f32(vw[j]);
-                    }
-                } else {                  /* straight from the input */
-                    size_t row = ((size_t)(cu_new[b] + pos - L) * H + h) * d;
-                    for (int j = 0; j < d; ++j) {
-                        k[j] = load_in(k_new, in_dtype, row + j);
-                        v[j] = load_in(v_new, in_dtype, row + j);
-                    }
+        int q0 = paged_len(l, L), q1 = paged_len(l, L + n);
+        /* fp32 row of position pos (< L + n) of (b, h): the ring when older than L */
+        #define KVQO_ROW(pos, h, kdst, vdst)                                              \
+            do {                                                                          \
+                if ((pos) < L) {                                                          \
+                    uint16_t* kw_ = win_row(l, c->k_win, b, (h), (pos));                  \
+                    uint16_t* vw_ = win_row(l, c->v_win, b, (h), (pos));                  \
+                    for (int j_ = 0; j_ < d; ++j_) {                                      \
+                        (kdst)[j_] = kvqo_bf16_to_f32(kw_[j_]);                           \
+                        (vdst)[j_] = kvqo_bf16_to_f32(vw_[j_]);                           \
+                    }                                                                     \
+                } else {                                                                  \
+                    size_t row_ = ((size_t)(cu_new[b] + (pos) - L) * H + (h)) * d;       \
+                    for (int j_ = 0; j_ < d; ++j_) {                                      \
+                        (kdst)[j_] = load_in(k_new, in_dtype, row_ + j_);                 \
+                        (vdst)[j_] = load_in(v_new, in_dtype, row_ + j_);                 \
+                    }                                                                     \
+                }                                                                         \
+            } while (0)
+        if (!l->k_per_channel) {
+            /* every position that leaves the window (or never enters it) */
+            float k[256], v[256];
+            for (int pos = q0; pos < q1; ++pos)
+                for (int h = 0; h < H; ++h) {
+                    KVQO_ROW(pos, h, k, v);
+                    quantize_token(l, c, b, h, pos, k, v);
                 }
-                quantize_token(l, c, b, h, pos, k, v);
-            }
+        } else {
+            /* every key group that became complete and left the window */
+            const int G = l->k_group;
+            float* K = (float*)malloc(sizeof(float) * (size_t)G * d);
+            float v[256];
+            for (int g0 = q0; g0 < q1; g0 += G)
+                for (int h = 0; h < H; ++h) {
+                    for (int t = 0; t < G; ++t) {
+                        KVQO_ROW(g0 + t, h, K + (size_t)t * d, v);
+                        quantize_token_values(l, c, b, h, g0 + t, v);
+                    }
+                    quantize_key_group(l, c, b, h, g0, K);
+                }
+            free(K);
         }
-        if (W > 0) {
-            int w0 = L + n - W > L ? L + n - W : L;
+        #undef KVQO_ROW
+        /* the new positions that stay in the window go to the ring (after
+         * the reads above: a slot may be reused) */
+        if (ring_slots(l) > 0) {
+            int w0 = q1 > L ? q1 : L;
             for (int pos = w0; pos < L + n; ++pos) {
                 for (int h = 0; h < H; ++h) {
                     size_t row = ((size_t)(cu_new[b] + pos - L) * H + h) * d;
@@ -532,7 +638,7 @@ static int reconstruct(const kvqo_layout* l, const kvqo_cache* c, int b, int h,
                        int L, int pos, float* k, float* v)
 {
     int d = l->head_dim;
-    if (pos >= L - l->window) {
+    if (pos >= paged_len(l, L)) {
         const uint16_t* kw = win_row(l, c->k_win, b, h, pos);
         const uint16_t* vw = win_row(l, c->v_win, b, h, pos);
         for (int j = 0; j < d; ++j) {
@@ -543,14 +649,20 @@ static int reconstruct(const kvqo_layout* l, const kvqo_cache* c, int b, int h,
     }
     int page = c->page_table[(size_t)b * c->max_pages_per_seq + pos / l->page_size];
     int slot = pos % l->page_size;
-    uint8_t kc[256], vrun[64];
-    k_row_io(l, c, page, h, slot, kc, 0);
+    uint8_t kc[256], vrun[64], krun[64];
+    if (!l->k_per_channel) k_row_io(l, c, page, h, slot, kc, 0);
     const uint8_t* km = k_meta_row(l, c, page, h, slot);
     const uint8_t* vm = v_meta_row(l, c, page, h, slot);
     for (int j = 0; j < d; ++j) {
         uint16_t s, z;
-        get_meta(km + 4 * (j / l->k_group), &s, &z);
-        k[j] = kvqo_dequant_code(kvqo_unpack_one(kc, j, l->k_bits), s, z);
+        if (l->k_per_channel) {
+            k_chan_io(l, c, page, h, j, krun, 0);
+            get_meta(k_meta_chan(l, c, page, h, slot / l->k_group, j), &s, &z);
+            k[j] = kvqo_dequant_code(kvqo_unpack_one(krun, slot, l->k_bits), s, z);
+        } else {
+            get_meta(km + 4 * (j / l->k_group), &s, &z);
+            k[j] = kvqo_dequant_code(kvqo_unpack_one(kc, j, l->k_bits), s, z);
+        }
         get_meta(vm + 4 * (j / l->v_group), &s, &z);
         v_chan_io(l, c, page, h, j, vrun, 0);
         v[j] = kvqo_dequant_code(kvqo_unpack_one(vrun, slot, l->v_bits), s, z);

@@ -61,6 +61,7 @@ class Workload:
     window: int = 0
     page_size: int = PAGE_SIZE
     rotate_keys: bool = False
+    k_per_channel: bool = False        # key groups of k_group positions of one channel
     in_dtype: str = DT_BF16
     # key outliers: ("fixed", (channels...), factor) | ("random", count, factor)
     #               | ("student_t", count, scale, nu)
