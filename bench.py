@@ -44,6 +44,9 @@ METRIC = "quantized-KV decode attention µs/step and HBM GB/s (% of B200 peak), 
 WORKLOADS = {"llama8b": wl.LLAMA8B, "sweep_k4v2": wl.SWEEP, "ragged": wl.RAGGED,
              "rotation": wl.ROTATION, "tiny": wl.TINY}
 FALLBACK_HBM_GBS = 6650.0
+# chunked-prefill attention: (cache shape, queries per sequence in the chunk)
+PREFILL_WORKLOADS = {"prefill_llama8b": (wl.LLAMA8B, 512)}
+PREFILL_METRIC = "chunked-prefill attention over the quantized cache, µs/step (fp32 TFLOP/s)"
 
 
 # ------------------------------------------------------------------ shared
@@ -504,13 +507,160 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def prefill_flops(lens, n, d: int, hq: int) -> float:
+    """Algorithmic flops of a chunked-prefill attention call: per (query,
+    head, visible position) 2d for q.k and 2d for p.v; query i of a chunk of
+    n at the end of L positions sees L - n + i + 1 of them."""
+    vis = 0
+    for L, m in zip(lens, n):
+        L, m = int(L), int(m)
+        vis += m * (L - m) + m * (m + 1) // 2
+    return 4.0 * d * hq * vis
+
+
+def oracle_prefill_timer(w: wl.Workload, chunk: int):
+    """Oracle (fp64, all host threads) on one sequence of the workload:
+    quantize its cache, then the chunk's causal attention; returns (seconds,
+    threads, sample description)."""
+    import oracle
+    L = w.seq_len
+    w1 = w.with_(batch=1, ragged=None)
+    lens = np.array([L], np.int32)
+    pt = wl.page_table(w1, np.maximum(0, lens - w1.window))
+    c = oracle.Cache(oracle.Layout.from_workload(w1), 1, pt, max(1, int((pt >= 0).sum())))
+    kr, vr, _, _, cu, _ = wl.prefill(w1, lens, with_f32=False)
+    c.append(kr, vr, oracle.IN_BF16, cu, np.zeros(1, np.int32))
+    q, _ = wl.chunk_queries(w1, chunk)
+    cu_q = np.array([0, chunk], np.int32)
+    t0 = time.perf_counter()
+    c.prefill_attention(q, oracle.IN_BF16, cu_q, lens, 1.0 / np.sqrt(w.head_dim))
+    dt = time.perf_counter() - t0
+    return dt, oracle.num_threads(), f"1 of {w.batch} sequences (chunk {chunk} at the end of {L} positions)"
+
+
+def run_prefill(args):
+    """Chunked-prefill attention (kvq_prefill_attention): every sequence holds
+    seq_len positions whose newest `chunk` are the chunk being prefilled; one
+    step is one call over the whole batch.  L2 is flushed (a 256 MB write)
+    before every timed call; each call is timed with events on its stream."""
+    import torch
+
+    import mixed_precision_quantized_kvq_b200 as kvq
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist("nccl")
+    w, chunk = PREFILL_WORKLOADS[args.workload]
+    B, L = w.batch, w.seq_len
+    lens = np.full(B, L, np.int32)
+    n = np.full(B, chunk, np.int32)
+    pt = wl.page_table(w, np.maximum(0, lens - w.window))
+    lay = kvq.Layout(w.head_dim, w.num_q_heads, w.num_kv_heads, w.k_bits, w.v_bits, w.k_group,
+                     w.v_group, w.page_size, w.window, False, None)
+    cache = kvq.PagedCache.allocate(lay, torch.from_numpy(pt).to(dev), max(1, int((pt >= 0).sum())))
+
+    def raw(a):
+        return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).to(dev)
+
+    kr, vr, _, _, cu, _ = wl.prefill(w, lens, with_f32=False)
+    glens = torch.zeros(B, dtype=torch.int32, device=dev)
+    kvq.kvq_quantize_append(lay, cache, raw(kr), raw(vr), torch.from_numpy(cu).to(dev), glens, L)
+    del kr, vr
+    glens.copy_(torch.from_numpy(lens))
+    cu_q = torch.from_numpy(np.concatenate([[0], np.cumsum(n)]).astype(np.int32)).to(dev)
+    q = raw(wl.chunk_queries(w, int(n.sum()))[0])
+    out = torch.empty((int(n.sum()), w.num_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+    lse = torch.empty((int(n.sum()), w.num_q_heads), dtype=torch.float32, device=dev)
+    scale = 1.0 / np.sqrt(w.head_dim)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+
+    def call():
+        kvq.kvq_prefill_attention(lay, cache, q, cu_q, glens, chunk, scale, out, lse, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            call()
+    stream.synchronize()
+    if dist is not None:
+        dist.barrier()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    with torch.cuda.stream(stream):
+        for e0, e1 in evs:
+            flush.fill_(1)
+            e0.record(stream)
+            call()
+            e1.record(stream)
+    stream.synchronize()
+    wall1 = time.time()
+    sampler.stop()
+    us = float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs])) * 1e3
+    us_max = reduce_max(dist, us, dev)
+
+    # e2e: the chunk's queries from pinned host memory, outputs back, every step
+    hq_ = q.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq = torch.empty_like(q)
+    k_e2e = max(1, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(k_e2e):
+            dq.copy_(hq_, non_blocking=True)
+            kvq.kvq_prefill_attention(lay, cache, dq, cu_q, glens, chunk, scale, out, lse, stream)
+            hout.copy_(out, non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    e2e_us = reduce_max(dist, e0.elapsed_time(e1) * 1e3 / k_e2e, dev)
+
+    flops = prefill_flops(lens, n, w.head_dim, w.num_q_heads)
+    props = torch.cuda.get_device_properties(dev)
+    clocks = sampler.summary(wall0, wall1)
+    sm_max = float((clocks or {}).get("sm_max_mhz") or 1965.0)
+    peak = props.multi_processor_count * 128 * 2 * sm_max * 1e6 / 1e12   # fp32 FMA lanes x 2 flops x clock
+    achieved = flops / (us * 1e-6) / 1e12
+    line = {
+        "metric": PREFILL_METRIC, "value": us_max, "unit": "us/step", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": us_max / 1e3, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; bf16 N(0,1) with key outlier channels)",
+        "config": {"workload": f"{args.workload}: batch {B}, {L} positions, chunk {chunk} (causal), "
+                               f"{w.num_q_heads}/{w.num_kv_heads} heads, d{w.head_dim}, K{w.k_bits}V{w.v_bits}, "
+                               f"window {w.window}", "l2": "flushed (256 MB write) before every call"},
+        "tflops": achieved, "flops_per_step": flops,
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "kvq_prefill_attention (CUDA cores)",
+                     "peak_source": f"{props.multi_processor_count} SMs x 128 fp32 lanes x 2 flops x {sm_max:.0f} MHz"},
+        "e2e": {"value": e2e_us, "unit": "us/step", "h2d_bytes_per_step": q.numel() * q.element_size(),
+                "d2h_bytes_per_step": out.numel() * out.element_size(),
+                "api": "python binding -> C ABI, eager calls, pinned host buffers"},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        dt, cores, sample = oracle_prefill_timer(w, chunk)
+        line["cpu_baseline"] = {"value": dt * 1e6 * B, "unit": "us/step", "cores": cores, "kind": "oracle",
+                                "sample": sample + f", scaled x{B} to the batch"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama8b")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(PREFILL_WORKLOADS), default="llama8b")
     ap.add_argument("--copies", type=int, default=0, help="cache copies to rotate (0 = auto from L2 size)")
     ap.add_argument("--graph-rounds", type=int, default=4)
     ap.add_argument("--e2e-steps", type=int, default=300)
@@ -520,7 +670,11 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.workload in PREFILL_WORKLOADS:
+        if args.impl == "reference":
+            ap.error("the prefill workloads time the CUDA path only (cpu_baseline carries the oracle)")
+        run_prefill(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
