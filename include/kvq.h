@@ -59,6 +59,21 @@
  *  Position p of sequence b lives in page page_table[b][p / P], slot p % P,
  *  when p < len - window, and in ring slot p % window otherwise.  All
  *  buffers must be 16-byte aligned.
+ *
+ * Per-channel key groups (k_per_channel = 1; "Granularitas kuantisasi
+ * ...": the grouping axis may run along token positions): a key group is
+ * k_group consecutive positions of ONE channel, aligned to k_group inside
+ * a page, quantized with the same min/max rule.  Then
+ *    k_codes [num_pages][Hkv][d][P*k_bits/8]  channel runs, stored like
+ *            v_codes (token slot t in bits k_bits*(t mod (32/k_bits)) of
+ *            word floor(t*k_bits/32); chunk-major above 16 bytes)
+ *    k_meta  [num_pages][Hkv][P/k_group][d] x {uint16 scale, uint16 zero}
+ *    k_win, v_win [batch][Hkv][window + k_group - 1][d] bf16 ring, slot =
+ *            position % (window + k_group - 1)
+ *  A key group is quantized once it is complete and out of the window
+ *  newest positions, so positions below Q = k_group*floor(max(0, len -
+ *  window)/k_group) live in pages and the rest (window to window +
+ *  k_group - 1 positions) in the ring.  Values keep per-token groups.
  */
 #ifndef KVQ_H_
 #define KVQ_H_
@@ -89,6 +104,8 @@ enum { KVQ_F32 = 0, KVQ_BF16 = 1 }; /* element types of inputs */
  * k_bits, v_bits  1, 2, 4 or 8 ("more for keys": k_bits >= v_bits is the
  *                 intended use, not a requirement)
  * k_group,v_group channels per group: 16, 32, 64 or 128, dividing d
+ *                 (with k_per_channel, k_group counts positions: 16, 32
+ *                 or 64)
  * page_size       tokens per page: 64
  * window          W >= 0 newest positions kept in bf16 (0 = none)
  * rotate_keys     1 = keys are multiplied by (diag(rot_signs) H / sqrt(d))
@@ -96,6 +113,10 @@ enum { KVQ_F32 = 0, KVQ_BF16 = 1 }; /* element types of inputs */
  *                 query is rotated the same way when scoring quantized
  *                 positions; window keys stay unrotated.
  * rot_signs       device int8 [d] of +1/-1, required when rotate_keys
+ * k_per_channel   1 = key groups run along positions of one channel (see
+ *                 the storage layout above); not combined with
+ *                 rotate_keys.  Decode and prefill attention then run on
+ *                 CUDA cores and need no workspace.
  */
 typedef struct kvq_layout {
     int head_dim;
@@ -109,6 +130,7 @@ typedef struct kvq_layout {
     int window;
     int rotate_keys;
     const int8_t* rot_signs;
+    int k_per_channel;
 } kvq_layout;
 
 /* Device buffers of one layer's cache (layout in the file header). */

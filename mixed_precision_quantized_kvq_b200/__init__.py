@@ -38,7 +38,7 @@ class kvq_layout(C.Structure):
     _fields_ = [("head_dim", C.c_int), ("num_q_heads", C.c_int), ("num_kv_heads", C.c_int),
                 ("k_bits", C.c_int), ("v_bits", C.c_int), ("k_group", C.c_int),
                 ("v_group", C.c_int), ("page_size", C.c_int), ("window", C.c_int),
-                ("rotate_keys", C.c_int), ("rot_signs", C.c_void_p)]
+                ("rotate_keys", C.c_int), ("rot_signs", C.c_void_p), ("k_per_channel", C.c_int)]
 
 
 class kvq_cache(C.Structure):
@@ -135,11 +135,12 @@ class Layout:
     window: int = 0
     rotate_keys: bool = False
     rot_signs: Optional[torch.Tensor] = None     # device int8 [head_dim]
+    k_per_channel: bool = False                  # key groups of k_group positions of one channel
 
     def c(self) -> kvq_layout:
         return kvq_layout(self.head_dim, self.num_q_heads, self.num_kv_heads, self.k_bits,
                           self.v_bits, self.k_group, self.v_group, self.page_size, self.window,
-                          int(self.rotate_keys), _ptr(self.rot_signs))
+                          int(self.rotate_keys), _ptr(self.rot_signs), int(self.k_per_channel))
 
 
 @dataclass
@@ -165,7 +166,7 @@ class PagedCache:
         batch = int(page_table.shape[0])
         wb = kvq_window_bytes(layout, batch)
         z = lambda n: torch.zeros(max(int(n), 16), dtype=torch.uint8, device=dev)
-        win = (z(wb), z(wb)) if layout.window > 0 else (None, None)
+        win = (z(wb), z(wb)) if wb > 0 else (None, None)
         return cls(z(kc * num_pages), z(vc * num_pages), z(km * num_pages), z(vm * num_pages),
                    win[0], win[1], page_table.to(torch.int32).contiguous(), num_pages)
 

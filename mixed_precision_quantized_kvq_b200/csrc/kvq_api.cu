@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "kvq_internal.cuh"
+#include "kvq_channel.cuh"
 #include "kvq_prefill.cuh"
 
 namespace {
@@ -42,12 +43,24 @@ int check_layout(const kvq_layout* l) {
     const int g = l->num_q_heads / l->num_kv_heads;
     if (g > kvq::kMaxGqa) return KVQ_ERR_UNSUPPORTED;
     if (!bits_ok(l->k_bits) || !bits_ok(l->v_bits)) return KVQ_ERR_UNSUPPORTED;
-    if (!group_ok(l->k_group, l->head_dim) || !group_ok(l->v_group, l->head_dim)) return KVQ_ERR_UNSUPPORTED;
+    if (l->k_per_channel != 0 && l->k_per_channel != 1) return KVQ_ERR_INVALID_ARG;
+    if (l->k_per_channel) {
+        // key groups of 16, 32 or 64 positions of one channel; rotation mixes channels per token
+        if (l->k_group != 16 && l->k_group != 32 && l->k_group != 64) return KVQ_ERR_UNSUPPORTED;
+        if (l->rotate_keys) return KVQ_ERR_UNSUPPORTED;
+    } else if (!group_ok(l->k_group, l->head_dim)) {
+        return KVQ_ERR_UNSUPPORTED;
+    }
+    if (!group_ok(l->v_group, l->head_dim)) return KVQ_ERR_UNSUPPORTED;
     if (l->page_size != kvq::kPage) return KVQ_ERR_UNSUPPORTED;
     if (l->window < 0) return KVQ_ERR_INVALID_ARG;
     if (l->rotate_keys && !l->rot_signs) return KVQ_ERR_INVALID_ARG;
     return KVQ_OK;
 }
+
+// bf16 ring slots per (sequence, kv-head): the window, plus kg - 1 positions
+// of an incomplete key group when key groups run along positions
+int ring_slots(const kvq_layout* l) { return l->window + (l->k_per_channel ? l->k_group - 1 : 0); }
 
 int check_cache(const kvq_layout* l, const kvq_cache* c) {
     if (!c) return KVQ_ERR_INVALID_ARG;
@@ -56,7 +69,7 @@ int check_cache(const kvq_layout* l, const kvq_cache* c) {
     if (!aligned16(c->k_codes) || !aligned16(c->v_codes) || !aligned16(c->k_meta) || !aligned16(c->v_meta) ||
         !aligned16(c->page_table))
         return KVQ_ERR_INVALID_ARG;
-    if (l->window > 0) {
+    if (ring_slots(l) > 0) {
         if (!c->k_win || !c->v_win || !aligned16(c->k_win) || !aligned16(c->v_win)) return KVQ_ERR_INVALID_ARG;
     }
     return KVQ_OK;
@@ -117,7 +130,7 @@ const char* kvq_status_string(int status) {
     }
 }
 
-int kvq_version(void) { return 100; }
+int kvq_version(void) { return 200; }
 
 int kvq_page_bytes(const kvq_layout* layout, size_t* k_codes, size_t* k_meta, size_t* v_codes,
                    size_t* v_meta) {
@@ -125,7 +138,10 @@ int kvq_page_bytes(const kvq_layout* layout, size_t* k_codes, size_t* k_meta, si
     if (rc) return rc;
     const size_t per = size_t(layout->num_kv_heads) * kvq::kPage;
     if (k_codes) *k_codes = per * size_t(layout->head_dim * layout->k_bits / 8);
-    if (k_meta) *k_meta = per * size_t(layout->head_dim / layout->k_group) * 4;
+    if (k_meta)
+        *k_meta = layout->k_per_channel
+                      ? size_t(layout->num_kv_heads) * (kvq::kPage / layout->k_group) * layout->head_dim * 4
+                      : per * size_t(layout->head_dim / layout->k_group) * 4;
     if (v_codes) *v_codes = per * size_t(layout->head_dim * layout->v_bits / 8);
     if (v_meta) *v_meta = per * size_t(layout->head_dim / layout->v_group) * 4;
     return KVQ_OK;
@@ -135,12 +151,13 @@ int kvq_window_bytes(const kvq_layout* layout, int batch, size_t* bytes) {
     int rc = check_layout(layout);
     if (rc) return rc;
     if (batch < 0 || !bytes) return KVQ_ERR_INVALID_ARG;
-    *bytes = size_t(batch) * layout->num_kv_heads * layout->window * layout->head_dim * 2;
+    *bytes = size_t(batch) * layout->num_kv_heads * ring_slots(layout) * layout->head_dim * 2;
     return KVQ_OK;
 }
 
 size_t kvq_decode_workspace_bytes(const kvq_layout* layout, int batch, int max_len) {
     if (check_layout(layout) || batch < 0 || max_len < 0) return 0;
+    if (layout->k_per_channel) return 0;   // one pass per (sequence, kv-head), no partials
     Params p = make_params(layout, nullptr);
     kvq::DecodePlan pl = kvq::plan_decode(p, batch, max_len, device_sm_count());
     return kvq::decode_workspace_bytes(p, batch, pl);
@@ -155,6 +172,7 @@ int kvq_set_decode_path(int path) {
 int kvq_get_decode_path(const kvq_layout* layout) {
     int rc = check_layout(layout);
     if (rc) return rc;
+    if (layout->k_per_channel) return 1;
     Params p = make_params(layout, nullptr);
     return (kvq::g_decode_path != 1 && kvq::tc_supported(p)) ? 2 : 1;
 }
@@ -170,6 +188,9 @@ int kvq_quantize_append(const kvq_layout* layout, const kvq_cache* cache, const 
     if (max_new > 0 && (!k_new || !v_new)) return KVQ_ERR_INVALID_ARG;
     if (max_new == 0 || cache->batch == 0) return KVQ_OK;
     Params p = make_params(layout, cache);
+    if (layout->k_per_channel)
+        return cuda_status(kvq::launch_append_per_channel(p, k_new, v_new, in_dtype == KVQ_BF16, cu_new, lens,
+                                                          max_new, reinterpret_cast<cudaStream_t>(stream)));
     return cuda_status(kvq::launch_quantize_append(p, k_new, v_new, in_dtype == KVQ_BF16, cu_new, lens, max_new,
                                                    reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -183,7 +204,12 @@ int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache, const
     if (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
     if (!q || !lens || !out || max_len < 0 || !isfinite(sm_scale)) return KVQ_ERR_INVALID_ARG;
     if (cache->batch == 0) return KVQ_OK;
+    if (cache->batch > 65535 || layout->num_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
     Params p = make_params(layout, cache);
+    if (layout->k_per_channel)   // one query per sequence through the chunked-prefill kernel
+        return cuda_status(kvq::launch_prefill_attention(p, 1, 1, q, q_dtype == KVQ_BF16, nullptr, lens, max_len,
+                                                         1, sm_scale, out, lse,
+                                                         reinterpret_cast<cudaStream_t>(stream)));
     kvq::DecodePlan pl = kvq::plan_decode(p, cache->batch, max_len, device_sm_count());
     const size_t need = kvq::decode_workspace_bytes(p, cache->batch, pl);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -204,8 +230,9 @@ int kvq_prefill_attention(const kvq_layout* layout, const kvq_cache* cache, cons
     if (max_q == 0 || cache->batch == 0) return KVQ_OK;
     if (!q || !out) return KVQ_ERR_INVALID_ARG;
     Params p = make_params(layout, cache);
-    return cuda_status(kvq::launch_prefill_attention(p, q, q_dtype == KVQ_BF16, cu_q, lens, max_q, sm_scale, out,
-                                                     lse, reinterpret_cast<cudaStream_t>(stream)));
+    return cuda_status(kvq::launch_prefill_attention(p, layout->k_per_channel, 0, q, q_dtype == KVQ_BF16, cu_q, lens,
+                                                     INT32_MAX, max_q, sm_scale, out, lse,
+                                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int kvq_dequantize(const kvq_layout* layout, const kvq_cache* cache, const int32_t* lens, int max_len,
@@ -216,6 +243,9 @@ int kvq_dequantize(const kvq_layout* layout, const kvq_cache* cache, const int32
     if (!lens || !k_out || !v_out || max_len < 0) return KVQ_ERR_INVALID_ARG;
     if (cache->batch == 0 || max_len == 0) return KVQ_OK;
     Params p = make_params(layout, cache);
+    if (layout->k_per_channel)
+        return cuda_status(kvq::launch_dequantize_per_channel(p, lens, max_len, k_out, v_out,
+                                                              reinterpret_cast<cudaStream_t>(stream)));
     return cuda_status(kvq::launch_dequantize(p, lens, max_len, k_out, v_out,
                                               reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -273,7 +303,12 @@ extern "C" int kvq_decode_attention_static_scratch(const kvq_layout* layout, con
     if (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
     if (!q || !lens || !out || max_len < 0 || !isfinite(sm_scale)) return KVQ_ERR_INVALID_ARG;
     if (cache->batch == 0) return KVQ_OK;
+    if (cache->batch > 65535 || layout->num_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
     Params p = make_params(layout, cache);
+    if (layout->k_per_channel)   // needs no scratch
+        return cuda_status(kvq::launch_prefill_attention(p, 1, 1, q, q_dtype == KVQ_BF16, nullptr, lens, max_len,
+                                                         1, sm_scale, out, lse,
+                                                         reinterpret_cast<cudaStream_t>(stream)));
     kvq::DecodePlan pl = kvq::plan_decode(p, cache->batch, max_len, device_sm_count());
     if (kvq::decode_workspace_bytes(p, cache->batch, pl) > KVQ_STATIC_SCRATCH_BYTES) return KVQ_ERR_WORKSPACE;
     void* scratch = nullptr;

@@ -52,9 +52,9 @@ cudaError_t launch_d(const prefill::View& v, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_prefill_attention(const Params& p, const void* q, int q_bf16, const int32_t* cu_q,
-                                     const int32_t* lens, int max_q, float sm_scale, float* out, float* lse,
-                                     cudaStream_t s) {
+cudaError_t launch_prefill_attention(const Params& p, int k_per_channel, int one_query, const void* q,
+                                     int q_bf16, const int32_t* cu_q, const int32_t* lens, int len_cap,
+                                     int max_q, float sm_scale, float* out, float* lse, cudaStream_t s) {
     prefill::View v{};
     v.d = p.d;
     v.hq = p.hq;
@@ -68,6 +68,11 @@ cudaError_t launch_prefill_attention(const Params& p, const void* q, int q_bf16,
     v.nvg = p.nvg;
     v.W = p.W;
     v.rotate = p.rotate;
+    v.kpc = k_per_channel;
+    v.R = k_per_channel ? p.W + p.kg - 1 : p.W;
+    v.kchan_bytes = prefill::kTile * p.kb / 8;
+    v.kchc = v.kchan_bytes < 16 ? v.kchan_bytes : 16;
+    v.one_query = one_query;
     v.signs = p.signs;
     v.k_codes = p.k_codes;
     v.v_codes = p.v_codes;
@@ -87,6 +92,7 @@ cudaError_t launch_prefill_attention(const Params& p, const void* q, int q_bf16,
     v.q_bf16 = q_bf16;
     v.cu_q = cu_q;
     v.lens = lens;
+    v.len_cap = len_cap;
     v.max_q = max_q;
     v.scale_log2 = sm_scale * 1.4426950408889634f;
     v.out = out;

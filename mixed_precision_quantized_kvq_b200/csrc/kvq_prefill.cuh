@@ -6,8 +6,12 @@
 
 namespace kvq {
 
-cudaError_t launch_prefill_attention(const Params& p, const void* q, int q_bf16, const int32_t* cu_q,
-                                     const int32_t* lens, int max_q, float sm_scale, float* out, float* lse,
-                                     cudaStream_t s);
+// k_per_channel: key groups run along positions (ring of W + kg - 1 slots).
+// one_query: decode (q [B][Hq][d], one query per sequence at its newest
+// position, cu_q unused, max_q = 1; empty sequences get out = 0, lse = -inf).
+// len_cap: device lengths above it are clamped to it.
+cudaError_t launch_prefill_attention(const Params& p, int k_per_channel, int one_query, const void* q,
+                                     int q_bf16, const int32_t* cu_q, const int32_t* lens, int len_cap,
+                                     int max_q, float sm_scale, float* out, float* lse, cudaStream_t s);
 
 }  // namespace kvq

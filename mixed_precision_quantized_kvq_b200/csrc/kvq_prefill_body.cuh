@@ -50,6 +50,8 @@ struct View {
     int d, hq, hkv, g;
     int kb, vb, kg, vg, nkg, nvg;
     int W, rotate;
+    int kpc;                           // 1: key groups of kg positions of one channel
+    int R;                             // ring slots: W, or W + kg - 1 with kpc
     const int8_t* signs;               // [d] +-1, when rotating
     const uint8_t* k_codes;
     const uint8_t* v_codes;
@@ -60,10 +62,14 @@ struct View {
     const int32_t* page_table;         // [B][max_pages]
     int batch, max_pages, num_pages;
     int krow_bytes, vchan_bytes, kch, vch;
+    int kchan_bytes, kchc;             // kpc: key channel run bytes and chunk bytes
     const void* q;                     // [total_q][Hq][d], bf16 or fp32
     int q_bf16;
+    int one_query;                     // decode: one query per sequence, q row b, cu_q unused;
+                                       // an empty sequence gets out = 0, lse = -inf
     const int32_t* cu_q;               // [B+1] query row offsets
     const int32_t* lens;               // [B] positions, the chunk included
+    int len_cap;                       // lengths above it are clamped to it
     int max_q;                         // >= every chunk length
     float scale_log2;                  // softmax scale * log2(e)
     float* out;                        // [total_q][Hq][d]
@@ -98,8 +104,23 @@ KVQ_HD float half_bits_f32(uint16_t b) {
     return __half2float(__half(r));
 }
 
+// positions of a length-L sequence that live in pages: below L - W, rounded
+// down to whole key groups when key groups run along positions
+KVQ_HD int paged_len(const View& v, int L) {
+    const int q = L - v.W > 0 ? L - v.W : 0;
+    return v.kpc ? q - q % v.kg : q;
+}
+
 // key of channel j at token slot t of page pg (fp32 reconstruction)
 KVQ_HD float key_at(const View& v, int pg, int h, int t, int j) {
+    if (v.kpc) {   // channel runs, metadata [64/kg][d]
+        const int bit = t * v.kb, byte = bit >> 3;
+        const uint8_t* blk = v.k_codes + (size_t(pg) * v.hkv + h) * size_t(v.d) * v.kchan_bytes;
+        const uint8_t c8 = blk[(byte / v.kchc) * (v.d * v.kchc) + j * v.kchc + (byte % v.kchc)];
+        const uint32_t code = (uint32_t(c8) >> (bit & 7)) & ((1u << v.kb) - 1u);
+        const uint32_t m = v.k_meta[((size_t(pg) * v.hkv + h) * size_t(kTile / v.kg) + t / v.kg) * v.d + j];
+        return fmaf(float(code), half_bits_f32(uint16_t(m & 0xffffu)), half_bits_f32(uint16_t(m >> 16)));
+    }
     const int bit = j * v.kb, byte = bit >> 3;
     const uint8_t* blk = v.k_codes + (size_t(pg) * v.hkv + h) * size_t(kTile) * v.krow_bytes;
     const uint8_t c8 = blk[(byte / v.kch) * (kTile * v.kch) + t * v.kch + (byte % v.kch)];
@@ -129,15 +150,25 @@ KVQ_HD void body(Ctx& cx, const View& v) {
     const int qt = cx.bx(), h = cx.by(), b = cx.bz();
     const int tid = cx.tid();
     const int g = v.g, QT = kRows / g, R = QT * g;
-    const int L = v.lens[b];
-    const int q0 = v.cu_q[b], n = v.cu_q[b + 1] - q0;
+    const int L = imin(v.lens[b], v.len_cap);
+    if (v.one_query && L <= 0) {                           // empty sequence: o = 0, lse = -inf
+        if (qt == 0)
+            for (int e = tid; e < g * D; e += kThreads) {
+                const size_t orow = size_t(b) * v.hq + size_t(h) * g + e / D;
+                v.out[orow * D + e % D] = 0.f;
+                if (v.lse && e % D == 0) v.lse[orow] = -INFINITY;
+            }
+        return;
+    }
+    const int q0 = v.one_query ? b : v.cu_q[b];
+    const int n = v.one_query ? 1 : v.cu_q[b + 1] - q0;
     if (n <= 0 || n > L || n > v.max_q) return;           // uniform over the CTA
     const int i0 = qt * QT;
     if (i0 >= n) return;
     const int nq = imin(QT, n - i0);                       // queries of this CTA
     const int base = L - n;                                // position of query 0 of the chunk
     const int p_max = base + i0 + nq - 1;                  // newest position any row sees
-    const int Lq = L - v.W > 0 ? L - v.W : 0;              // positions below Lq live in pages
+    const int Lq = paged_len(v, L);                        // positions below Lq live in pages
 
     float* sQ = cx.smem();
     float* sQr = sQ + kRows * LD;
@@ -212,7 +243,7 @@ KVQ_HD void body(Ctx& cx, const View& v) {
                         vx = value_at(v, pg, h, t, j);
                     }
                 } else {
-                    const size_t w = ((size_t(b) * v.hkv + h) * v.W + size_t(pos % v.W)) * D + j;
+                    const size_t w = ((size_t(b) * v.hkv + h) * v.R + size_t(pos % v.R)) * D + j;
                     kx = bf16_bits_f32(v.k_win[w]);
                     vx = bf16_bits_f32(v.v_win[w]);
                 }

@@ -43,7 +43,8 @@ class Pair:
         self.ocache = oracle.Cache(self.olay, w.batch, self.pt, self.num_pages)
         self.glay = kvq.Layout(w.head_dim, w.num_q_heads, w.num_kv_heads, w.k_bits, w.v_bits,
                                w.k_group, w.v_group, w.page_size, w.window, w.rotate_keys,
-                               torch.from_numpy(self.signs).to(device) if self.signs is not None else None)
+                               torch.from_numpy(self.signs).to(device) if self.signs is not None else None,
+                               w.k_per_channel)
         self.gcache = kvq.PagedCache.allocate(self.glay, torch.from_numpy(self.pt).to(device),
                                               self.num_pages)
         self.glens = torch.from_numpy(self.lens).to(device)
@@ -81,7 +82,7 @@ class Pair:
     def compare_cache(self):
         """Codes, metadata and window are bit-identical to the oracle's."""
         names = ["k_codes", "k_meta", "v_codes", "v_meta"]
-        if self.w.window > 0:
+        if self.olay.ring_slots > 0:
             names += ["k_win", "v_win"]
         for name in names:
             want = getattr(self.ocache, name).view(np.uint8).ravel()

@@ -140,3 +140,37 @@ def test_workspace_size_monotone():
     assert kvq.kvq_decode_workspace_bytes(lay, 0, 4096) >= 0
     assert kvq.kvq_decode_workspace_bytes(L(k_bits=3), 16, 4096) == 0
     assert kvq.kvq_decode_workspace_bytes(lay, 16, -1) == 0
+
+
+@pytest.mark.parametrize("kb,vb,kg,vg,d,w", [(4, 2, 64, 128, 128, 128), (4, 2, 32, 128, 128, 0),
+                                             (2, 4, 16, 64, 64, 8), (1, 1, 16, 32, 64, 3)])
+def test_per_channel_sizes_agree_with_oracle(kb, vb, kg, vg, d, w):
+    """Key groups along positions: page bytes as the oracle's layout, a ring
+    of window + k_group - 1 slots, no decode workspace, CUDA-core decode."""
+    lay = L(head_dim=d, k_bits=kb, v_bits=vb, k_group=kg, v_group=vg, window=w, k_per_channel=True)
+    olay = oracle.Layout(d, 32, 8, kb, vb, kg, vg, 64, w, k_per_channel=True)
+    assert kvq.kvq_page_bytes(lay) == oracle.page_bytes(olay)
+    assert kvq.kvq_window_bytes(lay, 16) == 16 * 8 * (w + kg - 1) * d * 2 == 16 * 8 * olay.ring_slots * d * 2
+    assert kvq.kvq_decode_workspace_bytes(lay, 16, 4096) == 0
+    assert kvq.kvq_get_decode_path(lay) == kvq.DECODE_CUDA_CORES
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k_group=128), kvq.KVQ_ERR_UNSUPPORTED),             # a group must fit in a 64-position page
+    (dict(k_group=48), kvq.KVQ_ERR_UNSUPPORTED),
+    (dict(rotate_keys=True), kvq.KVQ_ERR_UNSUPPORTED),        # checked before the missing signs
+])
+def test_per_channel_layout_rejected(kw, code):
+    with pytest.raises(kvq.KVQError) as e:
+        kvq.kvq_page_bytes(L(k_per_channel=True, **kw))
+    assert e.value.status == code
+
+
+def test_per_channel_ring_required_without_window():
+    """With key groups along positions the ring exists even at window 0."""
+    lib = kvq.lib()
+    lay = L(window=0, k_per_channel=True)
+    c, keep = _fake_cache(window=False)
+    buf = C.create_string_buffer(1024)
+    p = C.c_void_p((C.addressof(buf) + 255) & ~255)
+    assert lib.kvq_quantize_append(C.byref(lay.c()), C.byref(c), p, p, 1, p, p, 4, None) == kvq.KVQ_ERR_INVALID_ARG

@@ -1,7 +1,7 @@
 """The chunked-prefill kernel body, run on the CPU, against the oracle.
 
-tests/emu/prefill_emu.cpp runs the CUDA kernel's own per-CTA body
-(csrc/kvq_prefill_body.cuh) as host C++: one thread per CUDA thread, real
+tests/emu/kernel_emu.cpp (driven by tests/emu_harness.py) runs the CUDA
+kernel's own per-CTA body (csrc/kvq_prefill_body.cuh) as host C++: one thread per CUDA thread, real
 barriers, the GPU's warp-butterfly order.  It is built with AddressSanitizer
 and UndefinedBehaviorSanitizer and reads the oracle's cache arrays (the
 library's storage format) from exact-size allocations, so these tests check
@@ -10,66 +10,33 @@ every buffer, before it runs on a GPU.  They are not the GPU parity tests
 (tests/test_gpu_prefill.py): the emulator is neither the oracle nor a
 fallback of the library.
 """
-import os
-import shutil
-import subprocess
-
 import numpy as np
 import pytest
 
+import emu_harness as emu
 import oracle
 import workloads as wl
 
-HERE = os.path.dirname(os.path.abspath(__file__))
-ROOT = os.path.dirname(HERE)
-SRC = os.path.join(HERE, "emu", "prefill_emu.cpp")
-CSRC = os.path.join(ROOT, "mixed_precision_quantized_kvq_b200", "csrc")
 ATOL = RTOL = 1e-3
 
 
-def _cuda_include():
-    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
-    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.realpath(nvcc))), "include")
-    return inc if os.path.exists(os.path.join(inc, "cuda_fp16.h")) else None
-
-
 @pytest.fixture(scope="module")
-def emu(tmp_path_factory):
-    inc = _cuda_include()
-    gxx = shutil.which("g++")
-    if not inc or not gxx:
+def emu_exe(tmp_path_factory):
+    exe = emu.build(str(tmp_path_factory.mktemp("emu")))
+    if exe is None:
         pytest.skip("g++ or the CUDA headers are missing")
-    exe = str(tmp_path_factory.mktemp("emu") / "prefill_emu")
-    cmd = [gxx, "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=all",
-           "-fno-omit-frame-pointer", "-I", inc, "-I", CSRC, SRC, "-o", exe, "-pthread"]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    assert r.returncode == 0, r.stderr[-4000:]
     return exe
 
 
 def _run(exe, tmp, c: oracle.Cache, q, q_bf16, cu_q, lens, max_q, sm_scale, signs=None):
-    lay = c.layout
-    params = dict(d=lay.head_dim, hq=lay.num_q_heads, hkv=lay.num_kv_heads, kb=lay.k_bits, vb=lay.v_bits,
-                  kg=lay.k_group, vg=lay.v_group, W=lay.window, rotate=int(lay.rotate_keys), batch=c.batch,
-                  max_pages=c.page_table.shape[1], num_pages=c.num_pages, q_bf16=int(q_bf16), max_q=max_q,
-                  sm_scale=repr(float(sm_scale)))
-    with open(os.path.join(tmp, "params.txt"), "w") as f:
-        for k, v in params.items():
-            f.write(f"{k} {v}\n")
-    arrays = dict(k_codes=c.k_codes, v_codes=c.v_codes, k_meta=c.k_meta, v_meta=c.v_meta, k_win=c.k_win,
-                  v_win=c.v_win, page_table=c.page_table, q=q, cu_q=np.asarray(cu_q, np.int32),
-                  lens=np.asarray(lens, np.int32))
-    if signs is not None:
-        arrays["signs"] = np.asarray(signs, np.int8)
-    for k, a in arrays.items():
-        np.ascontiguousarray(a).tofile(os.path.join(tmp, k + ".bin"))
-    env = dict(os.environ, ASAN_OPTIONS="detect_leaks=0")
-    r = subprocess.run([exe, str(tmp)], capture_output=True, text=True, timeout=600, env=env)
-    assert r.returncode == 0, (r.stdout + r.stderr)[-4000:]
-    total = int(cu_q[-1])
-    out = np.fromfile(os.path.join(tmp, "out.bin"), np.float32).reshape(total, lay.num_q_heads, lay.head_dim)
-    lse = np.fromfile(os.path.join(tmp, "lse.bin"), np.float32).reshape(total, lay.num_q_heads)
-    return out, lse
+    params, arrays = emu.cache_params(c)
+    params.update(mode=emu.MODE_ATTENTION, q_bf16=int(q_bf16), max_q=max_q, sm_scale=sm_scale)
+    arrays.update(q=q, cu_q=np.asarray(cu_q, np.int32), lens=np.asarray(lens, np.int32),
+                  signs=None if signs is None else np.asarray(signs, np.int8))
+    total, lay = int(cu_q[-1]), c.layout
+    r = emu.run(exe, tmp, params, arrays, {"out": (np.float32, (total, lay.num_q_heads, lay.head_dim)),
+                                           "lse": (np.float32, (total, lay.num_q_heads))})
+    return r["out"], r["lse"]
 
 
 CASES = {
@@ -90,7 +57,7 @@ BASE = wl.Workload(name="prefill_emu", batch=3, num_q_heads=8, num_kv_heads=2, h
 
 
 @pytest.mark.parametrize("name", list(CASES))
-def test_emulated_kernel_matches_oracle(emu, tmp_path, name):
+def test_emulated_kernel_matches_oracle(emu_exe, tmp_path, name):
     over, cap = CASES[name]
     w = BASE.with_(**over)
     lens = wl.lengths(w)
@@ -106,12 +73,12 @@ def test_emulated_kernel_matches_oracle(emu, tmp_path, name):
     q, _ = wl.chunk_queries(w, int(cu_q[-1]))
     sc = 1 / np.sqrt(w.head_dim)
     ref_o, ref_l = c.prefill_attention(q, dt, cu_q, lens, sc)
-    out, lse = _run(emu, tmp_path, c, q, dt == oracle.IN_BF16, cu_q, lens, int(n.max()), sc, signs)
+    out, lse = _run(emu_exe, tmp_path, c, q, dt == oracle.IN_BF16, cu_q, lens, int(n.max()), sc, signs)
     np.testing.assert_allclose(out, ref_o, atol=ATOL, rtol=RTOL)
     np.testing.assert_allclose(lse, ref_l, atol=ATOL, rtol=RTOL)
 
 
-def test_emulated_kernel_skips_empty_and_oversized_chunks(emu, tmp_path):
+def test_emulated_kernel_skips_empty_and_oversized_chunks(emu_exe, tmp_path):
     w = BASE.with_(window=8)
     lens = np.array([70, 0, 5], np.int32)
     pt = wl.page_table(w, np.maximum(0, lens - w.window))
@@ -121,7 +88,7 @@ def test_emulated_kernel_skips_empty_and_oversized_chunks(emu, tmp_path):
     # sequence 1 sends nothing; sequence 2 sends 7 queries for 5 positions (skipped, rows untouched)
     cu_q = np.array([0, 20, 20, 27], np.int32)
     q, _ = wl.chunk_queries(w, 27)
-    out, lse = _run(emu, tmp_path, c, q, True, cu_q, lens, 20, 0.125)
+    out, lse = _run(emu_exe, tmp_path, c, q, True, cu_q, lens, 20, 0.125)
     ref_o, ref_l = c.prefill_attention(q[:20], oracle.IN_BF16, np.array([0, 20, 20, 20], np.int32),
                                        np.array([70, 0, 5], np.int32), 0.125)
     np.testing.assert_allclose(out[:20], ref_o, atol=ATOL, rtol=RTOL)
