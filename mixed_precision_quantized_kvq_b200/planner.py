@@ -4,9 +4,12 @@
 Bijdragen, Resultaten) argues that bits belong to the keys first: at a fixed
 memory budget a key-heavy split (K4V2) beats an even one.  This module turns
 that rule into a choice.  Given a budget in bytes per token and kv-head, it
-picks the setting (key bits, value bits, key group, value group), with key
-bits >= value bits, that fits the budget and has the smallest measured
-attention error.
+picks the setting (key bits, value bits, key grouping, value group), with
+key bits >= value bits, that fits the budget and has the smallest measured
+attention error.  Key groups run either over channels of one token or over
+positions of one channel ("Kuantisasi KV cache ...", section "Granularitas
+kuantisasi menentukan nilai yang berbagi scale": the grouping axis is an
+implementation choice).
 
 * Bytes come from the library's own accounting (`kvq_page_bytes`: packed
   codes plus fp16 scale and zero point per group, "Kuantisasi KV cache ...",
@@ -33,9 +36,11 @@ TABLE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "data", "error_
 METRICS = ("mean_abs", "max_abs", "score_max_abs", "tv_max")
 
 
-def bytes_per_token_head(k_bits: int, v_bits: int, k_group: int, v_group: int, head_dim: int = 128) -> float:
-    """Cache bytes of one token of one kv-head: codes and metadata of keys and values."""
-    lay = Layout(head_dim, 1, 1, k_bits, v_bits, k_group, v_group, PAGE_SIZE, 0)
+def bytes_per_token_head(k_bits: int, v_bits: int, k_group: int, v_group: int, head_dim: int = 128,
+                         k_per_channel: bool = False) -> float:
+    """Cache bytes of one token of one kv-head: codes and metadata of keys and
+    values (k_per_channel: key groups of k_group positions of one channel)."""
+    lay = Layout(head_dim, 1, 1, k_bits, v_bits, k_group, v_group, PAGE_SIZE, 0, k_per_channel=k_per_channel)
     kc, km, vc, vm = kvq_page_bytes(lay)
     return (kc + km + vc + vm) / PAGE_SIZE
 
@@ -52,8 +57,9 @@ def frontier(table: Optional[List[Dict]] = None, metric: str = "mean_abs", head_
     for r in (table if table is not None else load_table()):
         if r["v_bits"] > r["k_bits"]:
             continue
-        b = bytes_per_token_head(r["k_bits"], r["v_bits"], r["k_group"], r["v_group"], head_dim)
-        rows.append(dict(r, bytes=b))
+        pc = bool(r.get("k_per_channel", False))
+        b = bytes_per_token_head(r["k_bits"], r["v_bits"], r["k_group"], r["v_group"], head_dim, pc)
+        rows.append(dict(r, bytes=b, k_per_channel=pc))
     rows.sort(key=lambda r: (r["bytes"], r[metric]))
     out, best = [], float("inf")
     for r in rows:
@@ -81,12 +87,15 @@ def main(argv=None):
     ap.add_argument("--metric", default="mean_abs", choices=METRICS)
     args = ap.parse_args(argv)
     r = plan(args.budget, args.metric)
-    print(f"K{r['k_bits']} g{r['k_group']} / V{r['v_bits']} g{r['v_group']}: {r['bytes']:.1f} B per token-head, "
-          f"{args.metric} {r[args.metric]:.5f}")
+    print(f"{describe(r)}: {r['bytes']:.1f} B per token-head, {args.metric} {r[args.metric]:.5f}")
     print("\nfrontier (bytes -> error):")
     for f in frontier(metric=args.metric):
-        print(f"  {f['bytes']:6.1f} B  K{f['k_bits']} g{f['k_group']} / V{f['v_bits']} g{f['v_group']}  "
-              f"{args.metric} {f[args.metric]:.5f}")
+        print(f"  {f['bytes']:6.1f} B  {describe(f)}  {args.metric} {f[args.metric]:.5f}")
+
+
+def describe(r: Dict) -> str:
+    kgrp = f"{r['k_group']} positions" if r.get("k_per_channel") else f"g{r['k_group']}"
+    return f"K{r['k_bits']} {kgrp} / V{r['v_bits']} g{r['v_group']}"
 
 
 if __name__ == "__main__":

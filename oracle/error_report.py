@@ -47,6 +47,14 @@ def _quantized_rows(x: np.ndarray, group: int, bits: int) -> np.ndarray:
     return oracle.dequantize_rows(c, s, z, group).astype(np.float64)
 
 
+def _quantized_columns(x: np.ndarray, group: int, bits: int) -> np.ndarray:
+    """Columns of x [L][d] through the oracle's group quantizer in groups of
+    `group` consecutive rows (positions) of one column (channel), and back."""
+    L, d = x.shape
+    assert L % group == 0
+    return _quantized_rows(np.ascontiguousarray(x.T), group, bits).T
+
+
 def _attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, g: int, scale: float):
     """q [Hq][d], K and V [L][Hkv][d] -> scores s [Hq][L], weights a, output o [Hq][d] (fp64)."""
     Hq = q.shape[0]
@@ -59,8 +67,11 @@ def _attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, g: int, scale: float
 
 
 def measure(w: wl.Workload, k_bits: int, v_bits: int, rotate_keys: bool = False,
-            rotate_values: bool = False, length: int | None = None) -> dict:
-    """Error of attention over the quantized cache for one sequence of `w`."""
+            rotate_values: bool = False, length: int | None = None, k_per_channel: bool = False) -> dict:
+    """Error of attention over the quantized cache for one sequence of `w`.
+    k_per_channel: key groups of w.k_group positions of one channel (the
+    sequence length must be a multiple of it) instead of w.k_group channels
+    of one token."""
     w1 = w.with_(batch=1, window=0, seq_len=length or w.seq_len or w.ragged[1], ragged=None,
                  rotate_keys=False, k_bits=k_bits, v_bits=v_bits)
     lens = wl.lengths(w1)
@@ -77,10 +88,12 @@ def measure(w: wl.Workload, k_bits: int, v_bits: int, rotate_keys: bool = False,
     # keys: quantize (rotated rows when asked), score against the matching query
     if rotate_keys:
         Kr = (K.reshape(-1, d) @ R).astype(np.float32)
-        Khat = _quantized_rows(Kr, w1.k_group, k_bits) @ R.T          # back to the original basis
+        Khat = (_quantized_rows(Kr, w1.k_group, k_bits) @ R.T).reshape(L, Hkv, d)   # back to the original basis
+    elif k_per_channel:
+        Khat = np.stack([_quantized_columns(K[:, h].astype(np.float32), w1.k_group, k_bits)
+                         for h in range(Hkv)], axis=1)
     else:
-        Khat = _quantized_rows(K.reshape(-1, d), w1.k_group, k_bits)
-    Khat = Khat.reshape(L, Hkv, d)
+        Khat = _quantized_rows(K.reshape(-1, d), w1.k_group, k_bits).reshape(L, Hkv, d)
     if rotate_values:
         Vr = (V.reshape(-1, d) @ R).astype(np.float32)
         Vhat = _quantized_rows(Vr, w1.v_group, v_bits) @ R.T
@@ -95,6 +108,7 @@ def measure(w: wl.Workload, k_bits: int, v_bits: int, rotate_keys: bool = False,
     err = np.abs(o1 - o0)
     return {
         "k_bits": k_bits, "v_bits": v_bits, "rotate_keys": rotate_keys, "rotate_values": rotate_values,
+        "k_per_channel": k_per_channel, "k_group": w1.k_group,
         "tokens": L, "max_abs": float(err.max()), "mean_abs": float(err.mean()),
         "score_max_abs": float(np.abs(s1 - s0).max()),
         "tv_max": float(0.5 * np.abs(a1 - a0).sum(axis=1).max()),
@@ -110,26 +124,30 @@ def table(rows) -> str:
     out = [head]
     for r in rows:
         rot = "+".join(n for n, f in (("keys", r["rotate_keys"]), ("values", r["rotate_values"])) if f) or "none"
-        out.append(f"| {r['k_bits']} | {r['v_bits']} | {rot} | {r['max_abs']:.4f} | {r['mean_abs']:.5f} | "
+        kb = f"{r['k_bits']} ({r['k_group']} positions)" if r.get("k_per_channel") else f"{r['k_bits']}"
+        out.append(f"| {kb} | {r['v_bits']} | {rot} | {r['max_abs']:.4f} | {r['mean_abs']:.5f} | "
                    f"{r['score_max_abs']:.4f} | {r['tv_max']:.4f} | {r['key_only_max_abs']:.4f} | "
                    f"{r['value_only_max_abs']:.4f} |")
     return "\n".join(out)
 
 
 def grid(length: int = 4096):
-    """Errors of every (key bits >= value bits, key group, value group) setting
-    at head_dim 128 on the sweep workload's distribution: the table the
-    memory-budget planner reads."""
+    """Errors of every (key bits >= value bits, key grouping, value group)
+    setting at head_dim 128 on the sweep workload's distribution: the table
+    the memory-budget planner reads.  Key groupings: 32, 64 or 128 channels
+    of one token, or 32 or 64 positions of one channel."""
     out = []
     for kb in (8, 4, 2, 1):
         for vb in (8, 4, 2, 1):
             if vb > kb:
                 continue
-            for kg in (32, 64, 128):
-                for vg in (64, 128):
-                    r = measure(wl.SWEEP.with_(k_group=kg, v_group=vg), kb, vb, length=length)
-                    r.update(k_group=kg, v_group=vg)
-                    out.append(r)
+            for pc, kgs in ((False, (32, 64, 128)), (True, (32, 64))):
+                for kg in kgs:
+                    for vg in (64, 128):
+                        r = measure(wl.SWEEP.with_(k_group=kg, v_group=vg), kb, vb, length=length,
+                                    k_per_channel=pc)
+                        r.update(k_group=kg, v_group=vg)
+                        out.append(r)
     return out
 
 
@@ -141,7 +159,8 @@ def main(argv=None):
     if args.grid_json:
         import json
         rows = grid(min(args.length, 4096))
-        keep = ("k_bits", "v_bits", "k_group", "v_group", "tokens", "max_abs", "mean_abs", "score_max_abs", "tv_max")
+        keep = ("k_bits", "v_bits", "k_group", "v_group", "k_per_channel", "tokens", "max_abs", "mean_abs",
+                "score_max_abs", "tv_max")
         with open(args.grid_json, "w") as f:
             json.dump({"source": "python -m oracle.error_report --grid-json (oracle quantizer, fp64 attention, "
                                  "sweep workload distribution, one sequence, head_dim 128, 32/8 heads)",
@@ -155,6 +174,11 @@ def main(argv=None):
            for rk, rv in ((False, False), (True, False), (False, True), (True, True))]
     print(f"\nrotation workload (outlier key channels 10 * t(3)), K4V2, one sequence of {args.length} tokens\n")
     print(table(rot))
+    pc = [measure(wl.SWEEP.with_(k_group=g), kb, 2, length=args.length, k_per_channel=per)
+          for kb in (4, 2) for per, g in ((False, 32), (True, 32), (True, 64))]
+    print(f"\nsweep workload, key groups of 32 channels of one token vs groups of 32 / 64 positions of one "
+          f"channel, values 2-bit in groups of 128, one sequence of {args.length} tokens\n")
+    print(table(pc))
 
 
 if __name__ == "__main__":

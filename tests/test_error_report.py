@@ -41,3 +41,24 @@ def test_lossless_limit():
     r = er.measure(wl.SWEEP, 8, 8, length=256)
     assert r["max_abs"] < 0.05 * max(1.0, r["o_abs_mean"] * 10)
     assert np.isfinite(r["tv_max"])
+
+
+def test_per_channel_report_matches_the_cache():
+    """The report's key groups along positions are the oracle cache's
+    per-channel groups (window 0, length a multiple of the group)."""
+    import numpy as np
+
+    import oracle
+    import workloads as wl
+    from oracle import error_report as er
+
+    w = wl.SWEEP.with_(batch=1, num_kv_heads=2, num_q_heads=8, window=0, k_group=32, k_per_channel=True)
+    L = 256
+    lens = np.array([L], np.int32)
+    kr, vr, kf, _, cu, _ = wl.prefill(w, lens)
+    pt = wl.page_table(w, lens)
+    c = oracle.Cache(oracle.Layout.from_workload(w), 1, pt, int((pt >= 0).sum()))
+    c.append(kr, vr, oracle.IN_BF16, cu, np.zeros(1, np.int32))
+    kh, _ = c.dequantize(lens, L)
+    for h in range(w.num_kv_heads):
+        np.testing.assert_array_equal(er._quantized_columns(kf[:, h], 32, w.k_bits), kh[0, h])

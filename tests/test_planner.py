@@ -25,6 +25,24 @@ def test_bytes_match_memory_golden():
     assert planner.bytes_per_token_head(4, 4, 32, 128) == g["token_head_bytes_k4v4_g32_g128_d128"]
 
 
+def test_per_channel_bytes_match_golden():
+    g = {}
+    for line in open(os.path.join(os.path.dirname(GOLD), "memory_per_channel_keys.txt")):
+        if "=" in line and not line.startswith("#"):
+            k, v = line.split("=")
+            g[k.strip()] = float(v)
+    assert planner.bytes_per_token_head(4, 2, 64, 128, k_per_channel=True) == g["token_head_bytes_k4_pc64_v2_g128_d128"]
+    assert planner.bytes_per_token_head(4, 2, 32, 128, k_per_channel=True) == g["token_head_bytes_k4_pc32_v2_g128_d128"]
+    assert planner.bytes_per_token_head(2, 2, 64, 128, k_per_channel=True) == g["token_head_bytes_k2_pc64_v2_g128_d128"]
+
+
+def test_table_has_both_key_grouping_axes():
+    rows = planner.load_table()
+    axes = {(r["k_bits"], r["v_bits"], bool(r.get("k_per_channel"))) for r in rows if r["k_group"] == 32}
+    for kb in (1, 2, 4, 8):
+        assert (kb, 1, False) in axes and (kb, 1, True) in axes
+
+
 def test_table_covers_key_heavy_settings():
     rows = planner.load_table()
     keys = {(r["k_bits"], r["v_bits"], r["k_group"], r["v_group"]) for r in rows}
@@ -40,7 +58,8 @@ def test_table_covers_key_heavy_settings():
 def test_plan_is_the_best_fitting_setting(budget, metric):
     rows = planner.load_table()
     fitting = [r for r in rows if r["v_bits"] <= r["k_bits"] and
-               planner.bytes_per_token_head(r["k_bits"], r["v_bits"], r["k_group"], r["v_group"]) <= budget]
+               planner.bytes_per_token_head(r["k_bits"], r["v_bits"], r["k_group"], r["v_group"],
+                                            k_per_channel=r.get("k_per_channel", False)) <= budget]
     if not fitting:
         with pytest.raises(ValueError):
             planner.plan(budget, metric)
