@@ -163,7 +163,8 @@ int kvq_page_bytes(const kvq_layout* layout, size_t* k_codes, size_t* k_meta,
 int kvq_window_bytes(const kvq_layout* layout, int batch, size_t* bytes);
 
 /* Workspace that kvq_decode_attention needs for this batch and bound on
- * lengths on the current device (split partials); 0 on invalid input. */
+ * lengths on the current device (split partials); 0 on invalid input, and
+ * 0 for k_per_channel layouts (no split partials: workspace may be NULL). */
 size_t kvq_decode_workspace_bytes(const kvq_layout* layout, int batch, int max_len);
 
 /* Select the decode kernel family for subsequent kvq_decode_attention and
@@ -178,7 +179,8 @@ size_t kvq_decode_workspace_bytes(const kvq_layout* layout, int batch, int max_l
 int kvq_set_decode_path(int path);
 
 /* Decode kernel family the current setting picks for this layout:
- * 2 = tensor cores, 1 = CUDA cores, or a negative KVQ_ERR_* code. */
+ * 2 = tensor cores, 1 = CUDA cores (always for k_per_channel layouts), or a
+ * negative KVQ_ERR_* code. */
 int kvq_get_decode_path(const kvq_layout* layout);
 
 /* Append new tokens and quantize what leaves the bf16 window.
@@ -210,7 +212,11 @@ int kvq_quantize_append(const kvq_layout* layout, const kvq_cache* cache,
  *           log of sum exp(scores)) or NULL.  A sequence of length 0 gets
  *           out = 0 and lse = -inf.
  * workspace device, >= kvq_decode_workspace_bytes(layout, batch, max_len)
- *           bytes, 256-byte aligned; its contents need no initialisation. */
+ *           bytes, 256-byte aligned; its contents need no initialisation.
+ *           Not read for k_per_channel layouts (may be NULL): those run the
+ *           chunked-prefill kernel with one query per sequence, one CTA per
+ *           (sequence, kv-head), no split-K.
+ * Returns KVQ_ERR_UNSUPPORTED for batch or num_kv_heads above 65535. */
 int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache,
                          const void* q, int q_dtype, const int32_t* lens, int max_len,
                          float sm_scale, float* out, float* lse,
