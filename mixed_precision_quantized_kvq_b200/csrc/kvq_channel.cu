@@ -85,9 +85,18 @@ cudaError_t launch_append_per_channel(const Params& p, const void* k_new, const 
     v.in_bf16 = in_bf16;
     v.cu_new = cu_new;
     v.lens = lens;
+    // opt in once per device, for the largest size (d 128, groups of 64)
+    static bool configured[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    cudaError_t e;
+    if (!configured[dev]) {
+        e = cudaFuncSetAttribute(append_groups_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(chan::append_smem_bytes(128, 64)));
+        if (e != cudaSuccess) return e;
+        configured[dev] = true;
+    }
     const size_t sm = chan::append_smem_bytes(p.d, p.kg);
-    cudaError_t e = cudaFuncSetAttribute(append_groups_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm));
-    if (e != cudaSuccess) return e;
     const int groups = (max_new + p.kg - 1) / p.kg;
     append_groups_kernel<<<dim3(groups, p.hkv, p.batch), chan::kThreads, sm, s>>>(v);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

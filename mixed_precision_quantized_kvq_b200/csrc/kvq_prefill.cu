@@ -40,10 +40,18 @@ __global__ void __launch_bounds__(prefill::kThreads) prefill_attention_kernel(pr
 
 template <int D>
 cudaError_t launch_d(const prefill::View& v, cudaStream_t s) {
+    // opt in once per device, for the largest size (with rotation)
+    static bool configured[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
+        const cudaError_t e = cudaFuncSetAttribute(prefill_attention_kernel<D>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   int(prefill::smem_bytes(D, 1)));
+        if (e != cudaSuccess) return e;
+        configured[dev] = true;
+    }
     const size_t sm = prefill::smem_bytes(D, v.rotate);
-    cudaError_t e = cudaFuncSetAttribute(prefill_attention_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(sm));
-    if (e != cudaSuccess) return e;
     const int qpc = prefill::queries_per_cta(v.g);
     dim3 grid((v.max_q + qpc - 1) / qpc, v.hkv, v.batch);
     prefill_attention_kernel<D><<<grid, prefill::kThreads, sm, s>>>(v);
