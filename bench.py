@@ -42,7 +42,10 @@ import workloads as wl  # noqa: E402
 
 METRIC = "quantized-KV decode attention µs/step and HBM GB/s (% of B200 peak), K4V2"
 WORKLOADS = {"llama8b": wl.LLAMA8B, "sweep_k4v2": wl.SWEEP, "ragged": wl.RAGGED,
-             "rotation": wl.ROTATION, "tiny": wl.TINY}
+             "rotation": wl.ROTATION, "tiny": wl.TINY,
+             # the memory-budget planner's pick at 116 B per token-head: key groups of 64 positions
+             "per_channel_llama8b": wl.LLAMA8B.with_(name="llama3_8b_layer_b16_l4096_k4pc64v2g64_w128",
+                                                     k_group=64, v_group=64, k_per_channel=True)}
 FALLBACK_HBM_GBS = 6650.0
 # chunked-prefill attention: (cache shape, queries per sequence in the chunk)
 PREFILL_WORKLOADS = {"prefill_llama8b": (wl.LLAMA8B, 512)}
@@ -51,15 +54,25 @@ PREFILL_METRIC = "chunked-prefill attention over the quantized cache, µs/step (
 
 # ------------------------------------------------------------------ shared
 
+def paged_positions(w: wl.Workload, L: int) -> int:
+    """Positions of a length-L sequence that live in pages: below L - W, and
+    whole key groups only when key groups run along positions."""
+    q = max(0, L - w.window)
+    return q - q % w.k_group if w.k_per_channel else q
+
+
 def algorithmic_bytes(w: wl.Workload, lens) -> int:
     """Bytes the decode attention must read: packed codes + fp16 metadata of
-    every quantized token and bf16 K/V of every window token, per kv-head."""
+    every quantized token and bf16 K/V of every window token, per kv-head.
+    (Key metadata per token and kv-head is 4*d/k_group bytes for groups of
+    k_group channels and for groups of k_group positions alike.)"""
     d = w.head_dim
     t = d * w.k_bits // 8 + 4 * d // w.k_group + d * w.v_bits // 8 + 4 * d // w.v_group
     total = 0
     for L in lens:
         L = int(L)
-        total += (max(0, L - w.window) * t + min(w.window, L) * 4 * d) * w.num_kv_heads
+        q = paged_positions(w, L)
+        total += (q * t + (L - q) * 4 * d) * w.num_kv_heads
     return total
 
 
@@ -264,7 +277,7 @@ def workload_config(w: wl.Workload, lens1) -> dict:
     cfg = {"workload": w.name, "batch": w.batch, "q_heads": w.num_q_heads, "kv_heads": w.num_kv_heads,
            "head_dim": w.head_dim, "k_bits": w.k_bits, "v_bits": w.v_bits, "k_group": w.k_group,
            "v_group": w.v_group, "window": w.window, "page_size": w.page_size,
-           "rotate_keys": bool(w.rotate_keys),
+           "rotate_keys": bool(w.rotate_keys), "k_per_channel": bool(w.k_per_channel),
            "tokens_attended": int(lens1[0]) if w.ragged is None else "ragged",
            "total_tokens": int(np.sum(lens1)),
            "step": "append 1 token per sequence + decode attention (1 query token per sequence)",
@@ -316,7 +329,7 @@ def run_ours(args):
     npages = max(1, int((pt >= 0).sum()))
     signs = torch.from_numpy(wl.rotation_signs(w)).to(dev) if w.rotate_keys else None
     lay = kvq.Layout(w.head_dim, w.num_q_heads, w.num_kv_heads, w.k_bits, w.v_bits, w.k_group,
-                     w.v_group, w.page_size, w.window, w.rotate_keys, signs)
+                     w.v_group, w.page_size, w.window, w.rotate_keys, signs, w.k_per_channel)
 
     def raw(a):
         if a.dtype == np.uint16:
@@ -355,7 +368,8 @@ def run_ours(args):
     lse = torch.empty((w.batch, w.num_q_heads), dtype=torch.float32, device=dev)
     scale = 1.0 / math.sqrt(w.head_dim)
     # kernels per step: one append launch (a single token per sequence takes the
-    # one-launch append path) and the decode kernel plus its combine
+    # one-launch append path) and the decode kernel plus its combine; with key
+    # groups along positions, the group and ring kernels and one attention kernel
     launches_per_step = 3
 
     def step(i, ev=None):
@@ -487,7 +501,8 @@ def run_ours(args):
         "algorithmic_bytes_per_step": step_bytes,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "kvq_decode_attention (split-K decode + combine)",
+                     "kernel": "kvq_decode_attention (chunked-prefill kernel, one query per sequence)"
+                     if w.k_per_channel else "kvq_decode_attention (split-K decode + combine)",
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
                      else "fallback 6650 GB/s"},
         "e2e": {"value": e2e_us, "unit": "us/step", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

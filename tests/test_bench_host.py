@@ -95,3 +95,18 @@ def test_reference_arm_two_ranks_prints_once():
     lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1
     assert json.loads(lines[0])["n_gpus"] == 2
+
+
+def test_algorithmic_bytes_per_channel_counts_whole_groups():
+    """With key groups along positions the pages hold whole groups only; the
+    rest of the sequence is read from the bf16 ring."""
+    import bench
+    import workloads as wl
+    w = bench.WORKLOADS["per_channel_llama8b"]
+    d, H = w.head_dim, w.num_kv_heads
+    t = d * 4 // 8 + 4 * d // 64 + d * 2 // 8 + 4 * d // 64          # 64 + 8 + 32 + 8 = 112
+    assert t == 112
+    for L in (0, 100, 128, 191, 192, 193, 4096):
+        q = max(0, L - 128) // 64 * 64
+        assert bench.algorithmic_bytes(w, [L]) == (q * t + (L - q) * 4 * d) * H
+    assert bench.algorithmic_bytes(wl.LLAMA8B, [4096]) == (3968 * 116 + 128 * 512) * 8
