@@ -219,6 +219,41 @@ def oracle_step_timer(w: wl.Workload, budget_s: float):
     return us, oracle.num_threads(), f"{i} full steps of {w.name} (append + fp64 attention, all heads)"
 
 
+def oracle_tiny_single_thread(steps: int = 20):
+    """The oracle on one thread, on the tiny configuration (1 sequence of 256
+    tokens, 4/4 heads, d64, K4V2, fp32 inputs): mean microseconds of a full
+    step (append one token, fp64 attention of every head)."""
+    import oracle
+    before = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        us, _, _ = _tiny_steps(steps)
+    finally:
+        oracle.set_num_threads(before)
+    return us
+
+
+def _tiny_steps(steps: int):
+    import oracle
+    w = wl.TINY
+    lens0, lens1 = cache_lens(w)
+    kr, vr, _, _, cu, _ = wl.prefill(w, lens0, with_f32=False)
+    pt = wl.page_table(w, np.maximum(0, lens1 - w.window))
+    c = oracle.Cache(oracle.Layout.from_workload(w), w.batch, pt, max(1, int((pt >= 0).sum())))
+    in_dt = oracle.IN_BF16 if w.in_dtype == wl.DT_BF16 else oracle.IN_F32
+    c.append(kr, vr, in_dt, cu, np.zeros(w.batch, np.int32))
+    cu1 = np.arange(w.batch + 1, dtype=np.int32)
+    times = []
+    for i in range(steps):
+        k1, v1, _, _ = wl.new_tokens(w, i)
+        qr, _ = wl.query(w, i)
+        t = time.perf_counter()
+        c.append(k1, v1, in_dt, cu1, lens0)
+        c.decode_attention(qr, in_dt, lens1, 1.0 / math.sqrt(w.head_dim))
+        times.append(time.perf_counter() - t)
+    return float(np.median(times)) * 1e6, 1, ""
+
+
 def run_reference(args):
     ws, rank, local = dist_env()
     dist = init_dist("gloo")
@@ -265,7 +300,8 @@ def run_reference(args):
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(w, lens1),
             "cpu_baseline": {"value": us, "unit": "us/step", "cores": oracle.num_threads(),
-                             "kind": "oracle", "sample": sample},
+                             "kind": "oracle", "sample": sample,
+                             "tiny_single_thread_us": oracle_tiny_single_thread()},
             "e2e": {"value": us, "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     if dist is not None:
@@ -513,7 +549,7 @@ def run_ours(args):
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         us_cpu, cores, sample = oracle_step_timer(w, args.cpu_budget)
         line["cpu_baseline"] = {"value": us_cpu, "unit": "us/step", "cores": cores, "kind": "oracle",
-                                "sample": sample}
+                                "sample": sample, "tiny_single_thread_us": oracle_tiny_single_thread()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     del g_big, g_one

@@ -110,3 +110,11 @@ def test_algorithmic_bytes_per_channel_counts_whole_groups():
         q = max(0, L - 128) // 64 * 64
         assert bench.algorithmic_bytes(w, [L]) == (q * t + (L - q) * 4 * d) * H
     assert bench.algorithmic_bytes(wl.LLAMA8B, [4096]) == (3968 * 116 + 128 * 512) * 8
+
+
+def test_tiny_single_thread_oracle_timer_restores_threads():
+    import bench
+    import oracle
+    before = oracle.num_threads()
+    us = bench.oracle_tiny_single_thread(steps=3)
+    assert us > 0 and oracle.num_threads() == before
