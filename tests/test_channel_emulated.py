@@ -162,3 +162,31 @@ def test_emulated_dequantize_and_attention(emu_exe, tmp_path):
     ref, ref_lse = ec.oc.prefill_attention(qc, oracle.IN_BF16, cu_q, lens, sc)
     np.testing.assert_allclose(r["out"], ref, atol=ATOL, rtol=RTOL)
     np.testing.assert_allclose(r["lse"], ref_lse, atol=ATOL, rtol=RTOL)
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_emulated_append_random_sequences(emu_exe, tmp_path, seed):
+    """Random per-channel layouts and random append sizes (0 to 69 tokens per
+    sequence per call); bytes equal the oracle's after every call."""
+    r = np.random.default_rng([seed, 78])
+    d = int(r.choice([64, 128]))
+    hkv = int(r.choice([1, 2]))
+    w = wl.Workload(name="random", batch=int(r.integers(1, 4)), num_q_heads=2 * hkv, num_kv_heads=hkv, head_dim=d,
+                    seq_len=0, k_bits=int(r.choice([1, 2, 4, 8])), v_bits=int(r.choice([1, 2, 4, 8])),
+                    k_group=int(r.choice([16, 32, 64])), v_group=int(r.choice([x for x in (16, 32, 64, 128) if x <= d])),
+                    window=int(r.choice([0, 1, 7, 16, 64, 100])), k_per_channel=True,
+                    ragged=(0, int(r.integers(1, 200))), shuffle_pages=True, outliers=("random", 1, 10.0),
+                    seed=int(r.integers(0, 1 << 30)), in_dtype=wl.DT_BF16 if r.integers(0, 3) else wl.DT_F32)
+    lens0 = wl.lengths(w)
+    steps = [r.integers(0, 70, w.batch).astype(np.int32) for _ in range(3)]
+    ec = EmuCache(emu_exe, str(tmp_path), w, lens0 + sum(steps))
+    kr, vr, _, _, cu, _ = wl.prefill(w, lens0, with_f32=False)
+    if cu[-1] > 0:
+        ec.append(kr, vr, cu)
+        ec.compare()
+    for n in steps:
+        if n.sum() == 0:
+            continue
+        k, v = _chunk_rows(w, ec.lens, n)
+        ec.append(k, v, np.concatenate([[0], np.cumsum(n)]).astype(np.int32))
+        ec.compare()

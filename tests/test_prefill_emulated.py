@@ -94,3 +94,46 @@ def test_emulated_kernel_skips_empty_and_oversized_chunks(emu_exe, tmp_path):
     np.testing.assert_allclose(out[:20], ref_o, atol=ATOL, rtol=RTOL)
     np.testing.assert_allclose(lse[:20], ref_l, atol=ATOL, rtol=RTOL)
     assert np.all(out[20:] == 0) and np.all(lse[20:] == 0)
+
+
+def _random_case(seed):
+    """A random layout (d, GQA ratio, bits, grouping axis, groups, window,
+    rotation, input type), ragged lengths including empty sequences, and a
+    ragged chunk; seeded."""
+    r = np.random.default_rng([seed, 77])
+    d = int(r.choice([64, 128]))
+    hkv, g = int(r.choice([1, 2])), int(r.choice([1, 2, 3, 4, 5, 8]))
+    pc = bool(r.integers(0, 2))
+    kg = int(r.choice([16, 32, 64])) if pc else int(r.choice([x for x in (16, 32, 64, 128) if x <= d]))
+    w = wl.Workload(name="random", batch=int(r.integers(1, 4)), num_q_heads=hkv * g, num_kv_heads=hkv,
+                    head_dim=d, seq_len=0, k_bits=int(r.choice([1, 2, 4, 8])), v_bits=int(r.choice([1, 2, 4, 8])),
+                    k_group=kg, v_group=int(r.choice([x for x in (16, 32, 64, 128) if x <= d])),
+                    window=int(r.choice([0, 1, 5, 16, 64, 200])), k_per_channel=pc,
+                    rotate_keys=(not pc) and bool(r.integers(0, 4) == 0), ragged=(0, int(r.integers(1, 260))),
+                    shuffle_pages=True, outliers=("random", 2, 10.0), seed=int(r.integers(0, 1 << 30)),
+                    in_dtype=wl.DT_BF16 if r.integers(0, 3) else wl.DT_F32)
+    cap = int(r.integers(1, 150))
+    return w, r, cap
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_emulated_kernel_random_layouts(emu_exe, tmp_path, seed):
+    w, r, cap = _random_case(seed)
+    lens = wl.lengths(w)
+    signs = wl.rotation_signs(w) if w.rotate_keys else None
+    pt = wl.page_table(w, np.maximum(0, lens - w.window))
+    c = oracle.Cache(oracle.Layout.from_workload(w, signs), w.batch, pt, max(1, int((pt >= 0).sum())))
+    kr, vr, _, _, cu, _ = wl.prefill(w, lens, with_f32=False)
+    dt = oracle.IN_BF16 if w.in_dtype == wl.DT_BF16 else oracle.IN_F32
+    c.append(kr, vr, dt, cu, np.zeros(w.batch, np.int32))
+    n = np.minimum(lens, r.integers(0, cap + 1, w.batch)).astype(np.int32)
+    n[0] = min(int(lens[0]), max(1, int(n[0])))
+    cu_q = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    if cu_q[-1] == 0:
+        pytest.skip("every sequence of this draw is empty")
+    q, _ = wl.chunk_queries(w, int(cu_q[-1]))
+    sc = float(r.uniform(0.05, 0.2))
+    ref_o, ref_l = c.prefill_attention(q, dt, cu_q, lens, sc)
+    out, lse = _run(emu_exe, tmp_path, c, q, dt == oracle.IN_BF16, cu_q, lens, int(n.max()), sc, signs)
+    np.testing.assert_allclose(out, ref_o, atol=ATOL, rtol=RTOL)
+    np.testing.assert_allclose(lse, ref_l, atol=ATOL, rtol=RTOL)
