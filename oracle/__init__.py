@@ -16,13 +16,18 @@ import numpy as np
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "kvq_oracle.c")
-LIB = os.path.join(HERE, "libkvq_oracle.so")
+# KVQO_SANITIZE=1 builds and loads a separate copy under AddressSanitizer and
+# UBSan (the process must preload libasan); the arithmetic flags are the same.
+SANITIZE = os.environ.get("KVQO_SANITIZE") == "1"
+LIB = os.path.join(HERE, "libkvq_oracle_sanitized.so" if SANITIZE else "libkvq_oracle.so")
 
 RN, RD, RU = 0, -1, 1
 IN_F32, IN_BF16 = 0, 1
 
 CFLAGS = ["-O2", "-fPIC", "-shared", "-frounding-math", "-ffp-contract=off",
           "-fno-fast-math", "-fopenmp", "-Wall"]
+if SANITIZE:
+    CFLAGS += ["-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=all", "-fno-omit-frame-pointer"]
 
 
 def build(force: bool = False) -> str:

@@ -284,7 +284,8 @@ void kvqo_rotate_f64(const double* x, const int8_t* signs, int d, double* y)
 
 void kvqo_rotate(const float* x, const int8_t* signs, int d, float* y)
 {
-    double xd[256], yd[256];
+    double xd[256] = {0}, yd[256];
+    if (d <= 0 || d > 256) return;      /* head_dim is at most 256 (check_layout) */
     for (int j = 0; j < d; ++j) xd[j] = x[j];
     kvqo_rotate_f64(xd, signs, d, yd);
     for (int i = 0; i < d; ++i) y[i] = (float)yd[i];
