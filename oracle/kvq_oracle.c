@@ -102,6 +102,7 @@ static double round_to_format(double x, int p, int emin, double maxf, int mode)
 /* binary16: p = 11, emin = -14, max 65504; bits = sign | exp(5) | frac(10) */
 uint16_t kvqo_f32_to_f16(float x, int mode)
 {
+    if (isnan(x)) return (uint16_t)(signbit(x) ? 0xFE00u : 0x7E00u);   /* NaN stays NaN (quiet) */
     double v = round_to_format((double)x, 11, -14, 65504.0, mode);
     uint16_t s = signbit(v) ? 0x8000u : 0u;
     double a = fabs(v);
