@@ -195,3 +195,32 @@ def test_unsupported_per_channel_layouts():
     with pytest.raises(ValueError):                       # rotation is a per-token channel mix
         oracle.page_bytes(oracle.Layout(128, 8, 2, 4, 2, 32, 128, 64, 0, rotate_keys=True,
                                         k_per_channel=True))
+
+
+def test_storage_positions_hand_derived():
+    """Per-channel key storage, derived by hand from the layout: key codes are
+    channel runs of 64*kb/8 bytes stored like value runs (16-byte chunks,
+    chunk-major), key metadata [64/kg][d] words.  K4 at head_dim 128: token
+    slot 37 of channel 9 is the high nibble of run byte 18 = chunk 1, byte 2
+    -> block offset 1*(128*16) + 9*16 + 2 = 2194.  With groups of 16
+    positions, slot 37 is in group 2, so channel 9's metadata word is word
+    2*128 + 9 = 265 of the block, bytes 1060..1063."""
+    d = 128
+    lay = oracle.Layout(d, 1, 1, 4, 4, 16, 128, 64, 0, k_per_channel=True)
+    pt = np.zeros((1, 1), np.int32)
+    c = oracle.Cache(lay, 1, pt, 1)
+    # each channel's groups range over 0..15 (scale 1, zero 0): code == value
+    k = np.zeros((64, 1, d), np.float32)
+    v = np.zeros((64, 1, d), np.float32)
+    k[15::16, 0, :] = 15.0                   # the last slot of every 16-position group
+    k[37, 0, 9] = 6.0
+    v[:, 0, 127] = 15.0
+    c.append(k, v, oracle.IN_F32, np.array([0, 64], np.int32), np.zeros(1, np.int32))
+    kb = c.k_codes.ravel()
+    assert (kb[2194] >> 4) == 6
+    assert (kb[2194] & 0x0F) == 0            # slot 36 of channel 9
+    assert (kb[2194 + 16] >> 4) == 0         # slot 37 of channel 10
+    meta = c.k_meta.view(np.uint8).ravel()
+    scale = int(meta[1060]) | (int(meta[1061]) << 8)
+    zero = int(meta[1062]) | (int(meta[1063]) << 8)
+    assert (scale, zero) == (0x3C00, 0x0000)    # fp16 1.0 and +0
