@@ -705,6 +705,34 @@ def run_prefill(args):
         dist.destroy_process_group()
 
 
+def run_prefill_reference(args):
+    """The oracle (as it stands, all host threads) on the chunked-prefill
+    workload: each step times one sequence's chunk (cache quantization not
+    timed) and scales it to the batch.  Rank 0 only."""
+    ws, rank, local = dist_env()
+    dist = init_dist("gloo")
+    if rank == 0:
+        w, chunk = PREFILL_WORKLOADS[args.workload]
+        times, cores, sample = [], 1, ""          # no warm-up: the oracle keeps no state between steps
+        for _ in range(max(1, args.steps)):
+            dt, cores, sample = oracle_prefill_timer(w, chunk)
+            times.append(dt * 1e6 * w.batch)
+        us = float(np.mean(times))
+        line = {"impl": "reference", "metric": PREFILL_METRIC, "value": us, "unit": "us/step", "n_gpus": ws,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": f"{args.workload}: batch {w.batch}, {w.seq_len} positions, chunk {chunk} "
+                                       f"(causal), {w.num_q_heads}/{w.num_kv_heads} heads, d{w.head_dim}, "
+                                       f"K{w.k_bits}V{w.v_bits}, window {w.window}"},
+                "cpu_baseline": {"value": us, "unit": "us/step", "cores": cores, "kind": "oracle",
+                                 "sample": sample + f", scaled x{w.batch} to the batch"},
+                "e2e": {"value": us, "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -723,8 +751,9 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.workload in PREFILL_WORKLOADS:
         if args.impl == "reference":
-            ap.error("the prefill workloads time the CUDA path only (cpu_baseline carries the oracle)")
-        run_prefill(args)
+            run_prefill_reference(args)
+        else:
+            run_prefill(args)
     elif args.impl == "reference":
         run_reference(args)
     else:
