@@ -66,6 +66,31 @@ def _attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, g: int, scale: float
     return s, a, o
 
 
+def reconstruct(K: np.ndarray, V: np.ndarray, k_group: int, k_bits: int, v_group: int, v_bits: int,
+                Rk: np.ndarray | None = None, Rv: np.ndarray | None = None, k_per_channel: bool = False):
+    """Keys and values [L][Hkv][d] (fp64) as the quantized cache holds them,
+    in the original basis.  Rk / Rv: an orthogonal rotation applied to the
+    rows before quantization ("Quantize What Counts", Resultaten: rotation of
+    keys, and as an ablation of values); the quantized rows x^ R^T map back,
+    since R R^T = I.  k_per_channel: key groups of k_group positions of one
+    channel."""
+    L, Hkv, d = K.shape
+    if Rk is not None:
+        Kr = (K.reshape(-1, d) @ Rk).astype(np.float32)
+        Khat = (_quantized_rows(Kr, k_group, k_bits) @ Rk.T).reshape(L, Hkv, d)
+    elif k_per_channel:
+        Khat = np.stack([_quantized_columns(K[:, h].astype(np.float32), k_group, k_bits)
+                         for h in range(Hkv)], axis=1)
+    else:
+        Khat = _quantized_rows(K.reshape(-1, d), k_group, k_bits).reshape(L, Hkv, d)
+    if Rv is not None:
+        Vr = (V.reshape(-1, d) @ Rv).astype(np.float32)
+        Vhat = _quantized_rows(Vr, v_group, v_bits) @ Rv.T
+    else:
+        Vhat = _quantized_rows(V.reshape(-1, d), v_group, v_bits)
+    return Khat, Vhat.reshape(L, Hkv, d)
+
+
 def measure(w: wl.Workload, k_bits: int, v_bits: int, rotate_keys: bool = False,
             rotate_values: bool = False, length: int | None = None, k_per_channel: bool = False) -> dict:
     """Error of attention over the quantized cache for one sequence of `w`.
@@ -84,22 +109,8 @@ def measure(w: wl.Workload, k_bits: int, v_bits: int, rotate_keys: bool = False,
     scale = 1.0 / np.sqrt(d)
     g = w1.num_q_heads // Hkv
     R = _rotation_matrix(wl.rotation_signs(w.with_(rotate_keys=True))) if (rotate_keys or rotate_values) else None
-
-    # keys: quantize (rotated rows when asked), score against the matching query
-    if rotate_keys:
-        Kr = (K.reshape(-1, d) @ R).astype(np.float32)
-        Khat = (_quantized_rows(Kr, w1.k_group, k_bits) @ R.T).reshape(L, Hkv, d)   # back to the original basis
-    elif k_per_channel:
-        Khat = np.stack([_quantized_columns(K[:, h].astype(np.float32), w1.k_group, k_bits)
-                         for h in range(Hkv)], axis=1)
-    else:
-        Khat = _quantized_rows(K.reshape(-1, d), w1.k_group, k_bits).reshape(L, Hkv, d)
-    if rotate_values:
-        Vr = (V.reshape(-1, d) @ R).astype(np.float32)
-        Vhat = _quantized_rows(Vr, w1.v_group, v_bits) @ R.T
-    else:
-        Vhat = _quantized_rows(V.reshape(-1, d), w1.v_group, v_bits)
-    Vhat = Vhat.reshape(L, Hkv, d)
+    Khat, Vhat = reconstruct(K, V, w1.k_group, k_bits, w1.v_group, v_bits, R if rotate_keys else None,
+                             R if rotate_values else None, k_per_channel)
 
     s0, a0, o0 = _attention(q, K, V, g, scale)
     s1, a1, o1 = _attention(q, Khat, Vhat, g, scale)
