@@ -129,6 +129,25 @@ class Pair:
         return k.cpu().numpy(), v.cpu().numpy()
 
 
+    def check_dequantize(self, max_len=None):
+        """kvq_dequantize is bit-identical to the oracle's reconstruction:
+        code*scale+zero in one fp32 fma for quantized positions (keys in the
+        rotated domain when the layout rotates them), widened bf16 for window
+        positions; positions at or past a sequence's length are not written
+        (zeros here)."""
+        max_len = int(self.lens.max()) if max_len is None else max_len
+        k, v = self.dequantize(max_len)
+        ko, vo = self.ocache.dequantize(self.lens, max_len)
+        for name, got, want in (("keys", k, ko), ("values", v, vo)):
+            for b in range(self.w.batch):
+                L = int(min(self.lens[b], max_len))
+                g, o = got[b, :, :L], want[b, :, :L]
+                if not np.array_equal(g.view(np.uint32), o.view(np.uint32)):
+                    bad = np.argwhere(g.view(np.uint32) != o.view(np.uint32))
+                    raise AssertionError(f"{name} of sequence {b}: {len(bad)} values differ, first {bad[:4].tolist()}")
+                assert not got[b, :, L:].any(), f"{name} of sequence {b} written past its length"
+
+
 def check_close(got, want, what="value"):
     got = np.asarray(got, np.float64)
     want = np.asarray(want, np.float64)
