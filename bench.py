@@ -41,11 +41,13 @@ if ROOT not in sys.path:
 import workloads as wl  # noqa: E402
 
 METRIC = "quantized-KV decode attention µs/step and HBM GB/s (% of B200 peak), K4V2"
-WORKLOADS = {"llama8b": wl.LLAMA8B, "sweep_k4v2": wl.SWEEP, "ragged": wl.RAGGED,
+WORKLOADS = {"llama8b": wl.LLAMA8B, "ragged": wl.RAGGED,
              "rotation": wl.ROTATION, "tiny": wl.TINY,
              # the memory-budget planner's pick at 116 B per token-head: key groups of 64 positions
              "per_channel_llama8b": wl.LLAMA8B.with_(name="llama3_8b_layer_b16_l4096_k4pc64v2g64_w128",
                                                      k_group=64, v_group=64, k_per_channel=True)}
+# the long-context bit-allocation sweep: one workload per (key bits, value bits)
+WORKLOADS.update({f"sweep_k{v.k_bits}v{v.v_bits}": v for v in wl.sweep_variants()})
 FALLBACK_HBM_GBS = 6650.0
 # chunked-prefill attention: (cache shape, queries per sequence in the chunk)
 PREFILL_WORKLOADS = {"prefill_llama8b": (wl.LLAMA8B, 512)}
@@ -203,6 +205,7 @@ def oracle_step_timer(w: wl.Workload, budget_s: float):
     del kr, vr
     cu1 = np.arange(w.batch + 1, dtype=np.int32)
     times = []
+    first = None
     t_all = time.perf_counter()
     i = 0
     while True:
@@ -210,13 +213,15 @@ def oracle_step_timer(w: wl.Workload, budget_s: float):
         qr, _ = wl.query(w, i)
         t = time.perf_counter()
         c.append(k1, v1, in_dt, cu1, lens0)
-        c.decode_attention(qr, in_dt, lens1, 1.0 / math.sqrt(w.head_dim))
+        o, _ = c.decode_attention(qr, in_dt, lens1, 1.0 / math.sqrt(w.head_dim))
         times.append(time.perf_counter() - t)
+        if first is None:
+            first = np.array(o, np.float64)
         i += 1
         if (time.perf_counter() - t_all >= budget_s and i >= 2) or i >= 1000:
             break
     us = float(np.mean(times)) * 1e6
-    return us, oracle.num_threads(), f"{i} full steps of {w.name} (append + fp64 attention, all heads)"
+    return us, oracle.num_threads(), f"{i} full steps of {w.name} (append + fp64 attention, all heads)", first
 
 
 def oracle_tiny_single_thread(steps: int = 20):
@@ -349,6 +354,20 @@ def profile_traffic(workload: str):
         return None
 
 
+def timed_replays(graph_list, reps: int, stream):
+    """Median microseconds of one replay: `reps` replays (cycling through the
+    graphs), each bracketed by events on `stream`."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        for r, (e0, e1) in enumerate(evs):
+            e0.record(stream)
+            graph_list[r % len(graph_list)].replay()
+            e1.record(stream)
+    stream.synchronize()
+    return float(np.median([e0.elapsed_time(e1) for e0, e1 in evs])) * 1e3
+
+
 def run_ours(args):
     import torch
 
@@ -403,42 +422,47 @@ def run_ours(args):
     out = torch.empty((w.batch, w.num_q_heads, w.head_dim), dtype=torch.float32, device=dev)
     lse = torch.empty((w.batch, w.num_q_heads), dtype=torch.float32, device=dev)
     scale = 1.0 / math.sqrt(w.head_dim)
-    # kernels per step: one append launch (a single token per sequence takes the
-    # one-launch append path) and the decode kernel plus its combine; with key
-    # groups along positions, the group and ring kernels and one attention kernel
-    launches_per_step = 3
+    # kernels per step: the append (one launch for one token per sequence; the
+    # per-channel layout adds its ring write), then the decode: one persistent
+    # kernel, or a split kernel and its combine
+    path = kvq.kvq_get_decode_path(lay)
+    if w.k_per_channel:
+        launches_per_step, decode_kernel = 3, "kvq_decode_attention (chunked-prefill kernel, one query per sequence)"
+    elif path == kvq.DECODE_TENSOR_CORES:
+        launches_per_step, decode_kernel = 2, "kvq_decode_attention (persistent tensor-core kernel, merge fused)"
+    else:
+        launches_per_step, decode_kernel = 3, "kvq_decode_attention (split-K kernel + combine)"
 
-    def step(i, ev=None):
+    def append(i):
         c = caches[i % n_copies]
-        if ev is not None:
-            ev[0].record()
         kvq.kvq_quantize_append(lay, c, knew[i % n_copies], vnew[i % n_copies], cu1, glens0, 1)
-        if ev is not None:
-            ev[1].record()
-        kvq.kvq_decode_attention(lay, c, qs[i % n_copies], glens1, max_len, scale, out, lse, wsp)
-        if ev is not None:
-            ev[2].record()
+
+    def decode(i, qq=None):
+        c = caches[i % n_copies]
+        kvq.kvq_decode_attention(lay, c, qs[i % n_copies] if qq is None else qq, glens1, max_len, scale, out,
+                                 lse, wsp)
+
+    def step(i):
+        append(i)
+        decode(i)
 
     stream = torch.cuda.Stream(device=dev)
     S = n_copies * max(1, args.graph_rounds)
-    # per-launch times: events around the first step of every cache round of
-    # the S-step graph (a sample, so that event nodes stay off most steps)
-    timed = list(range(0, S, n_copies))
-    evs = {i: [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for i in timed}
     with torch.cuda.stream(stream):
         for i in range(2 * n_copies):          # eager warm-up before capture
             step(i)
     stream.synchronize()
-    g_big = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_big, stream=stream):
-        for i in range(S):
-            step(i, evs.get(i))
-    g_one = []
-    for c in range(n_copies):
+
+    def capture(fn):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            step(c)
-        g_one.append(g)
+            fn()
+        return g
+
+    g_big = capture(lambda: [step(i) for i in range(S)])
+    g_one = [capture(lambda c=c: step(c)) for c in range(n_copies)]
+    g_dec = [capture(lambda c=c: decode(c)) for c in range(n_copies)]
+    g_app = [capture(lambda c=c: append(c)) for c in range(n_copies)]
 
     def run_steps(k, start=0):
         """k steps through graph replays; returns the next step index."""
@@ -473,51 +497,56 @@ def run_ours(args):
         t_end.record(stream)
     stream.synchronize()
     torch.cuda.synchronize()
-    wall1 = time.time()
     if dist is not None:
         dist.barrier()
     ms = t_start.elapsed_time(t_end)
     ms_max = reduce_max(dist, ms, dev)
     us_step = ms_max * 1e3 / max(1, args.steps)
-    # per-launch times from the last replay of the S-step graph in the timed region
-    if args.steps < S:
-        with torch.cuda.stream(stream):
-            g_big.replay()
-        stream.synchronize()
-    app = [evs[i][0].elapsed_time(evs[i][1]) * 1e3 for i in timed]
-    dec = [evs[i][1].elapsed_time(evs[i][2]) * 1e3 for i in timed]
-    dec_us = float(np.mean(dec))
-    app_us = float(np.mean(app))
+    # medians over single-graph replays (each bracketed by events; every replay
+    # reads the next cache copy, so each reads HBM)
+    reps = max(200, args.median_reps)
+    med_step = reduce_max(dist, timed_replays(g_one, reps, stream), dev)
+    dec_us = reduce_max(dist, timed_replays(g_dec, reps, stream), dev)
+    app_us = reduce_max(dist, timed_replays(g_app, reps, stream), dev)
+    wall1 = time.time()
 
-    # e2e through the public API: host inputs in, host result out, every step
-    pin = lambda t: t.cpu().pin_memory()
-    hq = [pin(t) for t in qs]
-    hk = [pin(t) for t in knew]
-    hv = [pin(t) for t in vnew]
+    # e2e through the public API: each step copies its inputs (q, new k, new v
+    # packed in one pinned host buffer) to the device in one copy, appends,
+    # decodes and reads the output back; captured in a CUDA graph per cache copy
+    qn, kn = qs[0].numel() * qs[0].element_size(), knew[0].numel() * knew[0].element_size()
+    total = qn + 2 * kn
+    hstage = []
+    for c in range(n_copies):
+        hb = torch.empty(total, dtype=torch.uint8).pin_memory()
+        hb[:qn].copy_(qs[c].view(torch.uint8).reshape(-1).cpu())
+        hb[qn:qn + kn].copy_(knew[c].view(torch.uint8).reshape(-1).cpu())
+        hb[qn + kn:].copy_(vnew[c].view(torch.uint8).reshape(-1).cpu())
+        hstage.append(hb)
+    dstage = torch.empty(total, dtype=torch.uint8, device=dev)
+    dq = dstage[:qn].view(qs[0].dtype).view(qs[0].shape)
+    dk = dstage[qn:qn + kn].view(knew[0].dtype).view(knew[0].shape)
+    dv = dstage[qn + kn:].view(vnew[0].dtype).view(vnew[0].shape)
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    dq, dk, dv = torch.empty_like(qs[0]), torch.empty_like(knew[0]), torch.empty_like(vnew[0])
+
+    def e2e_step(c):
+        dstage.copy_(hstage[c], non_blocking=True)
+        kvq.kvq_quantize_append(lay, caches[c], dk, dv, cu1, glens0, 1)
+        kvq.kvq_decode_attention(lay, caches[c], dq, glens1, max_len, scale, out, lse, wsp)
+        hout.copy_(out, non_blocking=True)
+
+    g_e2e = [capture(lambda c=c: e2e_step(c)) for c in range(n_copies)]
     k_e2e = max(1, min(args.steps, args.e2e_steps))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
-        for rep in range(2):
-            n = min(3, k_e2e) if rep == 0 else k_e2e
-            if rep == 1:
-                e0.record(stream)
-            for i in range(n):
-                j = i % n_copies
-                dq.copy_(hq[j], non_blocking=True)
-                dk.copy_(hk[j], non_blocking=True)
-                dv.copy_(hv[j], non_blocking=True)
-                c = caches[j]
-                kvq.kvq_quantize_append(lay, c, dk, dv, cu1, glens0, 1)
-                kvq.kvq_decode_attention(lay, c, dq, glens1, max_len, scale, out, lse, wsp)
-                hout.copy_(out, non_blocking=True)
-            if rep == 1:
-                e1.record(stream)
+        for c in range(n_copies):
+            g_e2e[c].replay()
+        e0.record(stream)
+        for i in range(k_e2e):
+            g_e2e[i % n_copies].replay()
+        e1.record(stream)
     stream.synchronize()
     e2e_us = reduce_max(dist, e0.elapsed_time(e1) * 1e3 / k_e2e, dev)
-    h2d = qs[0].numel() * qs[0].element_size() + 2 * knew[0].numel() * knew[0].element_size()
-    d2h = out.numel() * out.element_size()
+    e2e_med = reduce_max(dist, timed_replays(g_e2e, reps, stream), dev)
 
     sampler.stop()
     clocks = sampler.summary(wall0, wall1)
@@ -533,26 +562,43 @@ def run_ours(args):
                        l2=f"{n_copies} rotating cache copies ({n_copies * step_bytes / 1e6:.0f} MB of "
                           f"decode reads) > 2x L2 ({l2 / 1e6:.0f} MB)"),
         "hbm_gbs": achieved, "pct_hbm_peak": 100.0 * achieved / peak,
+        "median_us": {"step": med_step, "decode_attention": dec_us, "append": app_us, "e2e_step": e2e_med,
+                      "replays": reps,
+                      "method": "median of single-graph replays, each bracketed by CUDA events on the stream"},
         "breakdown_us": {"append": app_us, "decode_attention": dec_us},
         "algorithmic_bytes_per_step": step_bytes,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "kvq_decode_attention (chunked-prefill kernel, one query per sequence)"
-                     if w.k_per_channel else "kvq_decode_attention (split-K decode + combine)",
+                     "frac": achieved / peak, "traffic": traffic, "kernel": decode_kernel,
+                     "duration_us": dec_us,
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
                      else "fallback 6650 GB/s"},
-        "e2e": {"value": e2e_us, "unit": "us/step", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "api": "python binding -> C ABI, eager calls, pinned host buffers"},
+        "e2e": {"value": e2e_us, "unit": "us/step", "h2d_bytes_per_step": total,
+                "d2h_bytes_per_step": out.numel() * out.element_size(),
+                "api": "python binding -> C ABI; one H2D copy of the packed step inputs from pinned memory, "
+                       "append, decode and the D2H read of the output captured in one CUDA graph per step"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        us_cpu, cores, sample = oracle_step_timer(w, args.cpu_budget)
+        # the oracle's first step has the inputs of cache copy 0: compare outputs
+        with torch.cuda.stream(stream):
+            step(0)
+        stream.synchronize()
+        got = out.cpu().numpy()
+        us_cpu, cores, sample, ref = oracle_step_timer(w, args.cpu_budget)
+        err = np.abs(got.astype(np.float64) - ref)
+        lim = 1e-3 + 1e-3 * np.abs(ref)
         line["cpu_baseline"] = {"value": us_cpu, "unit": "us/step", "cores": cores, "kind": "oracle",
-                                "sample": sample, "tiny_single_thread_us": oracle_tiny_single_thread()}
+                                "sample": sample, "tiny_single_thread_us": oracle_tiny_single_thread(),
+                                "oracle_check": {"what": "decode output of the first step (all sequences and "
+                                                         "heads) against the fp64 oracle on the same cache",
+                                                 "max_abs": float(err.max()),
+                                                 "max_rel_ref_gt_1e-2": float((err / np.maximum(np.abs(ref), 1e-30))
+                                                                              [np.abs(ref) > 1e-2].max()),
+                                                 "within_1e-3_plus_1e-3_rel": bool(np.all(err <= lim))}}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del g_big, g_one
+    del g_big, g_one, g_dec, g_app, g_e2e
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -743,6 +789,7 @@ def main():
     ap.add_argument("--copies", type=int, default=0, help="cache copies to rotate (0 = auto from L2 size)")
     ap.add_argument("--graph-rounds", type=int, default=4)
     ap.add_argument("--e2e-steps", type=int, default=300)
+    ap.add_argument("--median-reps", type=int, default=200, help="replays per median (at least 200)")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-sample-seqs", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -169,19 +169,36 @@ size_t kvq_decode_workspace_bytes(const kvq_layout* layout, int batch, int max_l
 
 /* Select the decode kernel family for subsequent kvq_decode_attention and
  * kvq_decode_workspace_bytes calls (process-wide):
- *   0  automatic (default): tensor-core kernel where the layout supports it
- *      (head_dim 128, key groups of 32, value groups of 128, any key and
- *      value bit widths), CUDA-core kernel otherwise
+ *   0  automatic (default): the persistent tensor-core kernel where the
+ *      layout supports it (head_dim 128, key groups of 32, value groups of
+ *      128, any key and value bit widths, batch <= 4096), the CUDA-core
+ *      kernel otherwise
  *   1  CUDA-core kernel for every layout
  *   2  same as 0 (tensor cores where supported)
+ *   3  the two-phase tcgen05 kernel with a separate combine launch where the
+ *      layout supports it (same layouts, any batch), CUDA cores otherwise
  * Not thread-safe with concurrent calls; query workspace sizes after
  * changing it.  Returns KVQ_ERR_INVALID_ARG for other values. */
 int kvq_set_decode_path(int path);
 
-/* Decode kernel family the current setting picks for this layout:
- * 2 = tensor cores, 1 = CUDA cores (always for k_per_channel layouts), or a
- * negative KVQ_ERR_* code. */
+/* Decode kernel family the current setting picks for this layout (at batch
+ * 1): 2 = persistent tensor-core kernel, 3 = two-phase tcgen05 kernel,
+ * 1 = CUDA cores (always for k_per_channel layouts), or a negative KVQ_ERR_*
+ * code. */
 int kvq_get_decode_path(const kvq_layout* layout);
+
+/* Decode diagnostics of the current device, counted by the decode kernels
+ * since the library was loaded (or last cleared):
+ *   wait_timeouts  bounded waits inside a decode kernel that gave up (the
+ *                  kernel then writes NaN for the outputs it could not
+ *                  finish; 0 in normal operation)
+ *   bad_tickets    merge tickets found above their count, i.e. a workspace
+ *                  that was not zero-filled before its first use (those
+ *                  outputs are not written)
+ * Either pointer may be NULL; clear != 0 resets both counters.  This call
+ * reads device memory synchronously (it waits for the device), unlike every
+ * other entry point; use it for checking, not inside a timed loop. */
+int kvq_decode_status(unsigned int* wait_timeouts, unsigned int* bad_tickets, int clear);
 
 /* Append new tokens and quantize what leaves the bf16 window.
  * ("Granularitas kuantisasi ..." group quantizer; "Pertumbuhan cache ..."
@@ -212,7 +229,12 @@ int kvq_quantize_append(const kvq_layout* layout, const kvq_cache* cache,
  *           log of sum exp(scores)) or NULL.  A sequence of length 0 gets
  *           out = 0 and lse = -inf.
  * workspace device, >= kvq_decode_workspace_bytes(layout, batch, max_len)
- *           bytes, 256-byte aligned; its contents need no initialisation.
+ *           bytes, 256-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE (for
+ *           example cudaMemsetAsync after allocating it).  It holds split
+ *           partials and one merge ticket per (sequence, kv-head); every
+ *           call leaves the tickets at zero again, so the zero fill is needed
+ *           once per allocation, not per call.  Calls that overlap on the GPU
+ *           need separate workspaces.
  *           Not read for k_per_channel layouts (may be NULL): those run the
  *           chunked-prefill kernel with one query per sequence, one CTA per
  *           (sequence, kv-head), no split-K.
@@ -235,16 +257,21 @@ int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache,
  * Arguments, output and error behaviour are those of kvq_decode_attention,
  * plus one case: KVQ_ERR_WORKSPACE, with nothing enqueued, when
  * kvq_decode_workspace_bytes(layout, cache->batch, max_len) exceeds
- * KVQ_STATIC_SCRATCH_BYTES.  For scale: batch 64 at lengths up to 16384
- * with 40/8 heads needs 12 MB.
- * Nothing needs to start at zero: each call writes every partial before
- * its combine step reads it.
+ * KVQ_STATIC_SCRATCH_BYTES.  For scale: the persistent tensor-core kernel
+ * needs about 1.3 MB on 148 SMs plus 4 bytes per (sequence, kv-head); the
+ * two-phase tcgen05 kernel needs 12 MB for batch 64 at lengths up to 16384
+ * with 40/8 heads.
+ * The array starts at zero when the library's module is loaded in a
+ * device context, which is what the merge tickets inside it need; each call
+ * writes every partial before reading it and leaves the tickets at zero.
  * One scratch array serves every call on a device.  Calls whose GPU
  * execution overlaps (different streams without ordering between them, or
  * several host threads) race on it and give undefined results.  Order them
  * on one stream, or use kvq_decode_attention with a workspace per stream.
- * The cached address belongs to the device's current context: do not call
- * this after cudaDeviceReset. */
+ * The cached address belongs to the context that was current on the device
+ * at the first call: do not call this after cudaDeviceReset, nor from
+ * another context on the same device (for example one made current with
+ * the driver API), since the address is not looked up again. */
 int kvq_decode_attention_static_scratch(const kvq_layout* layout, const kvq_cache* cache,
                                         const void* q, int q_dtype, const int32_t* lens,
                                         int max_len, float sm_scale, float* out, float* lse,

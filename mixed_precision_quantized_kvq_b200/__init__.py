@@ -78,6 +78,8 @@ def lib() -> C.CDLL:
         L.kvq_set_decode_path.restype = I
         L.kvq_get_decode_path.argtypes = [LP]
         L.kvq_get_decode_path.restype = I
+        L.kvq_decode_status.argtypes = [C.POINTER(C.c_uint), C.POINTER(C.c_uint), I]
+        L.kvq_decode_status.restype = I
         for n in ("kvq_page_bytes", "kvq_window_bytes", "kvq_quantize_append",
                   "kvq_decode_attention", "kvq_decode_attention_static_scratch", "kvq_dequantize",
                   "kvq_rotate_keys"):
@@ -100,6 +102,38 @@ def _ptr(t: Optional[torch.Tensor]):
     if not t.is_contiguous():
         raise ValueError("tensor must be contiguous")
     return C.c_void_p(t.data_ptr())
+
+
+def _check(t: Optional[torch.Tensor], name: str, dtypes, numel: Optional[int] = None,
+           at_least: bool = False, optional: bool = False) -> None:
+    """Argument checks before a C call: a CUDA tensor on the current device,
+    contiguous, of one of `dtypes`, with exactly (or at least) `numel`
+    elements.  A wrong buffer would otherwise be read or written past its end
+    by a kernel."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor, got {t.device}")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, not on the current CUDA device "
+                         f"cuda:{torch.cuda.current_device()}")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} must have dtype {' or '.join(str(d) for d in dtypes)}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if numel is not None:
+        n = t.numel()
+        if (n < numel) if at_least else (n != numel):
+            raise ValueError(f"{name} has {n} elements, expected {'at least ' if at_least else ''}{numel}")
+
+
+_FLOAT_IN = (torch.bfloat16, torch.float32)
+_I32 = (torch.int32,)
+_F32 = (torch.float32,)
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -198,14 +232,32 @@ def kvq_quantize_append(layout: Layout, cache: PagedCache, k_new: torch.Tensor, 
     """kvq.h kvq_quantize_append: k_new/v_new [total_new][Hkv][d] (bf16 or fp32)."""
     if k_new.dtype != v_new.dtype:
         raise ValueError("k_new and v_new must share a dtype")
+    B, row = cache.batch, layout.num_kv_heads * layout.head_dim
+    _check(k_new, "k_new", _FLOAT_IN)
+    if k_new.numel() % row:
+        raise ValueError(f"k_new must hold whole rows of {row} elements ([total_new][Hkv][d])")
+    _check(v_new, "v_new", _FLOAT_IN, k_new.numel())
+    _check(cu_new, "cu_new", _I32, B + 1)
+    _check(lens, "lens", _I32, B)
     _call("kvq_quantize_append", C.byref(layout.c()), C.byref(cache.c()), _ptr(k_new), _ptr(v_new),
           _dtype_code(k_new), _ptr(cu_new), _ptr(lens), int(max_new), _stream(stream))
+
+
+def _check_decode_args(layout, cache, q, lens, out, lse):
+    B, Hq, d = cache.batch, layout.num_q_heads, layout.head_dim
+    _check(q, "q", _FLOAT_IN, B * Hq * d)
+    _check(lens, "lens", _I32, B)
+    _check(out, "out", _F32, B * Hq * d)
+    _check(lse, "lse", _F32, B * Hq, optional=True)
 
 
 def kvq_decode_attention(layout: Layout, cache: PagedCache, q: torch.Tensor, lens: torch.Tensor,
                          max_len: int, sm_scale: float, out: torch.Tensor,
                          lse: Optional[torch.Tensor], workspace: torch.Tensor, stream=None) -> None:
     """kvq.h kvq_decode_attention: q [B][Hq][d] -> out fp32 [B][Hq][d], lse fp32 [B][Hq]."""
+    _check_decode_args(layout, cache, q, lens, out, lse)
+    _check(workspace, "workspace", (torch.uint8,), kvq_decode_workspace_bytes(layout, cache.batch, max_len),
+           at_least=True)
     _call("kvq_decode_attention", C.byref(layout.c()), C.byref(cache.c()), _ptr(q), _dtype_code(q),
           _ptr(lens), int(max_len), C.c_float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace),
           C.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
@@ -218,6 +270,7 @@ def kvq_decode_attention_static_scratch(layout: Layout, cache: PagedCache, q: to
     """kvq.h kvq_decode_attention_static_scratch: kvq_decode_attention with the
     library's static per-device scratch (KVQ_STATIC_SCRATCH_BYTES) instead of a
     workspace; calls overlapping on the GPU race on that scratch."""
+    _check_decode_args(layout, cache, q, lens, out, lse)
     _call("kvq_decode_attention_static_scratch", C.byref(layout.c()), C.byref(cache.c()), _ptr(q),
           _dtype_code(q), _ptr(lens), int(max_len), C.c_float(sm_scale), _ptr(out), _ptr(lse),
           _stream(stream))
@@ -229,6 +282,15 @@ def kvq_prefill_attention(layout: Layout, cache: PagedCache, q: torch.Tensor, cu
     """kvq.h kvq_prefill_attention: causal attention of each sequence's chunk
     of new queries (rows cu_q[b]..cu_q[b+1] of q [total_q][Hq][d]), whose keys
     and values are already appended, -> out fp32 [total_q][Hq][d], lse fp32."""
+    B, Hq, d = cache.batch, layout.num_q_heads, layout.head_dim
+    _check(q, "q", _FLOAT_IN)
+    if q.numel() % (Hq * d):
+        raise ValueError(f"q must hold whole rows of {Hq * d} elements ([total_q][Hq][d])")
+    T = q.numel() // (Hq * d)
+    _check(cu_q, "cu_q", _I32, B + 1)
+    _check(lens, "lens", _I32, B)
+    _check(out, "out", _F32, T * Hq * d)
+    _check(lse, "lse", _F32, T * Hq, optional=True)
     _call("kvq_prefill_attention", C.byref(layout.c()), C.byref(cache.c()), _ptr(q), _dtype_code(q),
           _ptr(cu_q), _ptr(lens), int(max_q), C.c_float(sm_scale), _ptr(out), _ptr(lse), _stream(stream))
 
@@ -236,23 +298,40 @@ def kvq_prefill_attention(layout: Layout, cache: PagedCache, q: torch.Tensor, cu
 def kvq_dequantize(layout: Layout, cache: PagedCache, lens: torch.Tensor, max_len: int,
                    k_out: torch.Tensor, v_out: torch.Tensor, stream=None) -> None:
     """kvq.h kvq_dequantize: fp32 [B][Hkv][max_len][d] reconstructions."""
+    n = cache.batch * layout.num_kv_heads * int(max_len) * layout.head_dim
+    _check(lens, "lens", _I32, cache.batch)
+    _check(k_out, "k_out", _F32, n)
+    _check(v_out, "v_out", _F32, n)
     _call("kvq_dequantize", C.byref(layout.c()), C.byref(cache.c()), _ptr(lens), int(max_len),
           _ptr(k_out), _ptr(v_out), _stream(stream))
 
 
 def kvq_rotate_keys(layout: Layout, k: torch.Tensor, out: torch.Tensor, stream=None) -> None:
     """kvq.h kvq_rotate_keys: rows [rows][d] -> fp32 rotated rows."""
+    _check(k, "k", _FLOAT_IN)
+    if k.numel() % layout.head_dim:
+        raise ValueError(f"k must hold whole rows of {layout.head_dim} elements")
     rows = k.numel() // layout.head_dim
+    _check(out, "out", _F32, rows * layout.head_dim)
     _call("kvq_rotate_keys", C.byref(layout.c()), _ptr(k), _dtype_code(k), int(rows), _ptr(out),
           _stream(stream))
 
 
-DECODE_AUTO, DECODE_CUDA_CORES, DECODE_TENSOR_CORES = 0, 1, 2
+DECODE_AUTO, DECODE_CUDA_CORES, DECODE_TENSOR_CORES, DECODE_TCGEN05 = 0, 1, 2, 3
 
 
 def kvq_set_decode_path(path: int) -> None:
-    """kvq.h kvq_set_decode_path: 0 automatic, 1 CUDA cores, 2 tensor cores."""
+    """kvq.h kvq_set_decode_path: 0 automatic, 1 CUDA cores, 2 tensor cores
+    (persistent kernel), 3 the two-phase tcgen05 kernel."""
     _call("kvq_set_decode_path", int(path))
+
+
+def kvq_decode_status(clear: bool = False) -> Tuple[int, int]:
+    """kvq.h kvq_decode_status: (expired bounded waits, bad merge tickets) on
+    the current device; blocking."""
+    t, b = C.c_uint(), C.c_uint()
+    _call("kvq_decode_status", C.byref(t), C.byref(b), int(bool(clear)))
+    return int(t.value), int(b.value)
 
 
 def kvq_get_decode_path(layout: Layout) -> int:
@@ -265,8 +344,10 @@ def kvq_get_decode_path(layout: Layout) -> int:
 # ---------------------------------------------------------------- helpers
 
 def workspace_for(layout: Layout, batch: int, max_len: int, device) -> torch.Tensor:
+    """A decode workspace, zero-filled as kvq_decode_attention requires before
+    its first use (each call leaves it ready for the next)."""
     n = max(kvq_decode_workspace_bytes(layout, batch, max_len), 256)
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def decode_attention(layout: Layout, cache: PagedCache, q: torch.Tensor, lens: torch.Tensor,

@@ -164,7 +164,7 @@ size_t kvq_decode_workspace_bytes(const kvq_layout* layout, int batch, int max_l
 }
 
 int kvq_set_decode_path(int path) {
-    if (path < 0 || path > 2) return KVQ_ERR_INVALID_ARG;
+    if (path < 0 || path > 3) return KVQ_ERR_INVALID_ARG;
     kvq::g_decode_path = path;
     return KVQ_OK;
 }
@@ -174,7 +174,14 @@ int kvq_get_decode_path(const kvq_layout* layout) {
     if (rc) return rc;
     if (layout->k_per_channel) return 1;
     Params p = make_params(layout, nullptr);
-    return (kvq::g_decode_path != 1 && kvq::tc_supported(p)) ? 2 : 1;
+    const int path = kvq::g_decode_path;
+    if (path == 1) return 1;
+    if (path == 3) return kvq::tc_supported(p) ? 3 : 1;
+    return kvq::mma_supported(p, 1) ? 2 : 1;
+}
+
+int kvq_decode_status(unsigned int* wait_timeouts, unsigned int* bad_tickets, int clear) {
+    return cuda_status(kvq::decode_status(wait_timeouts, bad_tickets, clear != 0));
 }
 
 int kvq_quantize_append(const kvq_layout* layout, const kvq_cache* cache, const void* k_new,
@@ -203,6 +210,7 @@ int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache, const
     if ((rc = check_cache(layout, cache))) return rc;
     if (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
     if (!q || !lens || !out || max_len < 0 || !isfinite(sm_scale)) return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return KVQ_ERR_INVALID_ARG;
     if (cache->batch == 0) return KVQ_OK;
     if (cache->batch > 65535 || layout->num_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
     Params p = make_params(layout, cache);
@@ -302,6 +310,7 @@ extern "C" int kvq_decode_attention_static_scratch(const kvq_layout* layout, con
     if ((rc = check_cache(layout, cache))) return rc;
     if (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
     if (!q || !lens || !out || max_len < 0 || !isfinite(sm_scale)) return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return KVQ_ERR_INVALID_ARG;
     if (cache->batch == 0) return KVQ_OK;
     if (cache->batch > 65535 || layout->num_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
     Params p = make_params(layout, cache);

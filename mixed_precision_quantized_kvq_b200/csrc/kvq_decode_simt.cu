@@ -26,7 +26,18 @@ DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count) {
     const int npages = (maxq + kPage - 1) / kPage;
     pl.window_split = p.W > 0 ? 1 : 0;
     const int units = batch * p.hkv > 0 ? batch * p.hkv : 1;
-    pl.tc = (g_decode_path != 1 && tc_supported(p)) ? 1 : 0;
+    if ((g_decode_path == 0 || g_decode_path == 2) && mma_supported(p, batch)) {
+        // one CTA per SM at most, each with an equal share of the units; no
+        // combine launch (split pairs are merged inside the kernel)
+        const int win = p.W < max_len ? p.W : max_len;
+        // an upper bound on the units (the kernel counts them from the device lengths)
+        const long long nu = (long long)batch * p.hkv * ((maxq + 127) / 128 + (win + 15) / 16 + 1);
+        pl.mma = 1;
+        pl.ctas = (int)(nu < sm_count ? nu : sm_count);
+        if (pl.ctas < 1) pl.ctas = 1;
+        return pl;
+    }
+    pl.tc = (g_decode_path == 3 && tc_supported(p)) ? 1 : 0;
     if (pl.tc) {
         // quantized splits (slots 0 .. splits_q-1), each a whole number of
         // 128-token tiles, then the window CTAs (64 window positions each, short
@@ -74,6 +85,7 @@ DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count) {
 }
 
 size_t decode_workspace_bytes(const Params& p, int batch, const DecodePlan& pl) {
+    if (pl.mma) return mma_workspace_layout(p, batch, pl.ctas, nullptr);
     size_t rows = size_t(batch) * p.hq * pl.total_splits;
     size_t o = rows * p.d * sizeof(float);
     o = (o + 255) & ~size_t(255);
@@ -410,16 +422,61 @@ cudaError_t dispatch_kb(const Params& p, const void* q, int q_bf16, const int32_
 
 }  // namespace
 
+// decode diagnostics: [0] expired bounded waits, [1] tickets above their count
+__device__ unsigned int g_decode_status[2];
+
+namespace {
+constexpr int kMaxDev = 64;
+unsigned* g_status_addr[kMaxDev];
+unsigned* status_ptr() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+    if (!g_status_addr[dev]) {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_decode_status) != cudaSuccess) return nullptr;
+        g_status_addr[dev] = static_cast<unsigned*>(a);
+    }
+    return g_status_addr[dev];
+}
+}  // namespace
+
+cudaError_t decode_status(unsigned* wait_timeouts, unsigned* bad_tickets, bool clear) {
+    unsigned v[2] = {0u, 0u};
+    cudaError_t e = cudaMemcpyFromSymbol(v, g_decode_status, sizeof(v));
+    if (e != cudaSuccess) return e;
+    if (wait_timeouts) *wait_timeouts = v[0];
+    if (bad_tickets) *bad_tickets = v[1];
+    if (clear) {
+        const unsigned z[2] = {0u, 0u};
+        e = cudaMemcpyToSymbol(g_decode_status, z, sizeof(z));
+    }
+    return e;
+}
+
 cudaError_t launch_decode(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len,
                           float sm_scale, float* out, float* lse, void* ws, const DecodePlan& pl,
                           cudaStream_t s) {
     if (p.batch <= 0) return cudaSuccess;
+    unsigned* status = status_ptr();
+    if (!status) return cudaErrorInvalidSymbol;
     const size_t rows = size_t(p.batch) * p.hq;
     float* ws_o = reinterpret_cast<float*>(ws);
     size_t ob = (rows * pl.total_splits * p.d * sizeof(float) + 255) & ~size_t(255);
     float* ws_ml = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + ob);
     const float sl2 = sm_scale * 1.4426950408889634f;
-    cudaError_t e = pl.tc ? launch_decode_tc(p, q, q_bf16, lens, max_len, sl2, ws_o, ws_ml, pl, s)
+    if (pl.mma) {
+        size_t off_tickets = 0;
+        mma_workspace_layout(p, p.batch, pl.ctas, &off_tickets);
+        float* part = reinterpret_cast<float*>(ws);
+        uint32_t* tickets = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + off_tickets);
+        switch (p.kb) {
+            case 1: return launch_decode_mma_k1(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, pl.ctas, status, s);
+            case 2: return launch_decode_mma_k2(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, pl.ctas, status, s);
+            case 4: return launch_decode_mma_k4(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, pl.ctas, status, s);
+            default: return launch_decode_mma_k8(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, pl.ctas, status, s);
+        }
+    }
+    cudaError_t e = pl.tc ? launch_decode_tc(p, q, q_bf16, lens, max_len, sl2, ws_o, ws_ml, pl, status, s)
                   : (p.d == 128) ? dispatch_kb<128>(p, q, q_bf16, lens, max_len, sl2, ws_o, ws_ml, pl, s)
                                  : dispatch_kb<64>(p, q, q_bf16, lens, max_len, sl2, ws_o, ws_ml, pl, s);
     if (e != cudaSuccess) return e;

@@ -7,13 +7,13 @@
 namespace kvq {
 
 cudaError_t launch_decode_tc_k1(const Params&, const void*, int, const int32_t*, int, float, float*, float*,
-                                const DecodePlan&, cudaStream_t);
+                                const DecodePlan&, unsigned*, cudaStream_t);
 cudaError_t launch_decode_tc_k2(const Params&, const void*, int, const int32_t*, int, float, float*, float*,
-                                const DecodePlan&, cudaStream_t);
+                                const DecodePlan&, unsigned*, cudaStream_t);
 cudaError_t launch_decode_tc_k4(const Params&, const void*, int, const int32_t*, int, float, float*, float*,
-                                const DecodePlan&, cudaStream_t);
+                                const DecodePlan&, unsigned*, cudaStream_t);
 cudaError_t launch_decode_tc_k8(const Params&, const void*, int, const int32_t*, int, float, float*, float*,
-                                const DecodePlan&, cudaStream_t);
+                                const DecodePlan&, unsigned*, cudaStream_t);
 
 static bool bits_ok(int b) { return b == 1 || b == 2 || b == 4 || b == 8; }
 
@@ -28,12 +28,12 @@ int tc_ctas_per_sm(const Params& p) {
 }
 
 cudaError_t launch_decode_tc(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len,
-                             float scale_log2, float* ws_o, float* ws_ml, const DecodePlan& pl, cudaStream_t s) {
+                             float scale_log2, float* ws_o, float* ws_ml, const DecodePlan& pl, unsigned* status, cudaStream_t s) {
     switch (p.kb) {
-        case 1: return launch_decode_tc_k1(p, q, q_bf16, lens, max_len, scale_log2, ws_o, ws_ml, pl, s);
-        case 2: return launch_decode_tc_k2(p, q, q_bf16, lens, max_len, scale_log2, ws_o, ws_ml, pl, s);
-        case 4: return launch_decode_tc_k4(p, q, q_bf16, lens, max_len, scale_log2, ws_o, ws_ml, pl, s);
-        case 8: return launch_decode_tc_k8(p, q, q_bf16, lens, max_len, scale_log2, ws_o, ws_ml, pl, s);
+        case 1: return launch_decode_tc_k1(p, q, q_bf16, lens, max_len, scale_log2, ws_o, ws_ml, pl, status, s);
+        case 2: return launch_decode_tc_k2(p, q, q_bf16, lens, max_len, scale_log2, ws_o, ws_ml, pl, status, s);
+        case 4: return launch_decode_tc_k4(p, q, q_bf16, lens, max_len, scale_log2, ws_o, ws_ml, pl, status, s);
+        case 8: return launch_decode_tc_k8(p, q, q_bf16, lens, max_len, scale_log2, ws_o, ws_ml, pl, status, s);
         default: return cudaErrorNotSupported;
     }
 }

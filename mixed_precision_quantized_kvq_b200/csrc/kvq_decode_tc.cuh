@@ -59,8 +59,6 @@ constexpr int kWinSmem = 2 * WCH * D * 2;     // key and value rows of a chunk
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr unsigned FULL = 0xffffffffu;
 
-// number of bounded waits that expired (diagnostic; 0 in normal operation)
-static __device__ unsigned int g_tc_wait_timeouts;
 
 constexpr int ns_cols(int nhc) { return ((12 * nhc + 15) / 16) * 16; }
 // score accumulator buffers: two when they fit in 256 columns with the rest
@@ -528,7 +526,7 @@ template <int KB, int VB, int NHC>
 __global__ void __launch_bounds__(kThreads, ctas_per_sm(KB, VB, NHC))
 decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, const int32_t* __restrict__ lens,
                  const int max_len, const float scale_log2, float* __restrict__ ws_o, float* __restrict__ ws_ml,
-                 const int pps, const int nws, const int slots) {
+                 const int pps, const int nws, const int slots, unsigned int* __restrict__ status) {
     using C = Cfg<KB, VB, NHC>;
     using LY = Layout<KB, VB, NHC>;
     constexpr int R = LY::R;
@@ -945,7 +943,7 @@ decode_tc_kernel(const Params p, const void* __restrict__ q, const int q_bf16, c
                 ws_ml[row * 2 + 1] = bad ? NAN : ls;
             }
         }
-        if (bad && t == 0) atomicAdd(&g_tc_wait_timeouts, 1u);
+        if (bad && t == 0) atomicAdd(&status[0], 1u);
     }
     // ------------------------------------------------------------------ teardown
     tc_fence_before();

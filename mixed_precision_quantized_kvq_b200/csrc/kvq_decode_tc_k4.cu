@@ -4,8 +4,8 @@
 namespace kvq {
 
 cudaError_t launch_decode_tc_k4(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len,
-                                float sl2, float* ws_o, float* ws_ml, const DecodePlan& pl, cudaStream_t s) {
-    return tc::launch_kb<4>(p, q, q_bf16, lens, max_len, sl2, ws_o, ws_ml, pl, s);
+                                float sl2, float* ws_o, float* ws_ml, const DecodePlan& pl, unsigned* status, cudaStream_t s) {
+    return tc::launch_kb<4>(p, q, q_bf16, lens, max_len, sl2, ws_o, ws_ml, pl, status, s);
 }
 
 }  // namespace kvq

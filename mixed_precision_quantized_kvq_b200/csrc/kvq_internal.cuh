@@ -119,7 +119,9 @@ __device__ __forceinline__ void rotate_warp(float (&x)[D / 32], const int8_t* si
 
 // ---- launchers -----------------------------------------------------------
 struct DecodePlan {
-    int tc;             // 1: tensor-core kernel, 0: CUDA-core kernel
+    int mma;            // 1: persistent register-fragment tensor-core kernel (no combine launch)
+    int ctas;           // its grid: one CTA per SM at most
+    int tc;             // 1: two-phase tcgen05 kernel, 0: CUDA-core kernel (when mma == 0)
     int splits_q;       // splits over quantized pages
     int pages_per_split;
     int window_split;   // partial slots of the bf16 window (CUDA-core kernel: 0 or 1; tensor-core
@@ -128,13 +130,27 @@ struct DecodePlan {
     int grid_x;         // CTAs per (sequence, kv-head)
     int window_slot;    // slot index of the window partial
 };
+// persistent register-fragment tensor-core decode (kvq_decode_mma.cuh), one key bit width per file
+cudaError_t launch_decode_mma_k1(const Params&, const void*, int, const int32_t*, int, float, float*, float*, float*,
+                                 uint32_t*, int, unsigned*, cudaStream_t);
+cudaError_t launch_decode_mma_k2(const Params&, const void*, int, const int32_t*, int, float, float*, float*, float*,
+                                 uint32_t*, int, unsigned*, cudaStream_t);
+cudaError_t launch_decode_mma_k4(const Params&, const void*, int, const int32_t*, int, float, float*, float*, float*,
+                                 uint32_t*, int, unsigned*, cudaStream_t);
+cudaError_t launch_decode_mma_k8(const Params&, const void*, int, const int32_t*, int, float, float*, float*, float*,
+                                 uint32_t*, int, unsigned*, cudaStream_t);
 // decode path selection: 0 = automatic, 1 = CUDA cores, 2 = tensor cores
 extern int g_decode_path;
 DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count);
 bool tc_supported(const Params& p);
+bool mma_supported(const Params& p, int batch);
+// workspace of the persistent kernel: merge partials of `ctas` CTAs, then one
+// ticket per (sequence, kv-head); returns the bytes, and the tickets' offset
+size_t mma_workspace_layout(const Params& p, int batch, int ctas, size_t* off_tickets);
 int tc_ctas_per_sm(const Params& p);
 cudaError_t launch_decode_tc(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len,
-                             float scale_log2, float* ws_o, float* ws_ml, const DecodePlan& pl, cudaStream_t s);
+                             float scale_log2, float* ws_o, float* ws_ml, const DecodePlan& pl, unsigned* status,
+                             cudaStream_t s);
 size_t decode_workspace_bytes(const Params& p, int batch, const DecodePlan& plan);
 
 cudaError_t launch_quantize_append(const Params& p, const void* k_new, const void* v_new,
@@ -147,5 +163,9 @@ cudaError_t launch_rotate_keys(const Params& p, const void* k, int in_bf16, int 
 cudaError_t launch_decode(const Params& p, const void* q, int q_bf16, const int32_t* lens,
                           int max_len, float sm_scale, float* out, float* lse, void* ws,
                           const DecodePlan& plan, cudaStream_t s);
+// decode diagnostics (device words the decode kernels count into): [0] bounded
+// waits that expired, [1] tickets found above their count.  Read and
+// optionally cleared by decode_status (blocking).
+cudaError_t decode_status(unsigned* wait_timeouts, unsigned* bad_tickets, bool clear);
 
 }  // namespace kvq

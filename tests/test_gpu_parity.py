@@ -15,10 +15,12 @@ from gpu_harness import Pair, check_close, torch_raw
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(autouse=True, params=[kvq.DECODE_AUTO, kvq.DECODE_CUDA_CORES], ids=["auto", "cuda_cores"])
+@pytest.fixture(autouse=True, params=[kvq.DECODE_AUTO, kvq.DECODE_CUDA_CORES, kvq.DECODE_TCGEN05],
+                ids=["auto", "cuda_cores", "tcgen05"])
 def decode_path(request):
-    """Every case runs on the automatic choice (tensor cores where the layout
-    allows) and on the CUDA-core kernel."""
+    """Every case runs on the automatic choice (the persistent tensor-core
+    kernel where the layout allows), on the CUDA-core kernel and on the
+    two-phase tcgen05 kernel."""
     kvq.kvq_set_decode_path(request.param)
     yield request.param
     kvq.kvq_set_decode_path(kvq.DECODE_AUTO)
@@ -26,7 +28,8 @@ def decode_path(request):
 
 def test_tensor_core_path_selected_for_k4v2_layout(decode_path):
     lay = kvq.Layout(128, 32, 8, 4, 2, 32, 128, 64, 128)
-    want = kvq.DECODE_TENSOR_CORES if decode_path == kvq.DECODE_AUTO else kvq.DECODE_CUDA_CORES
+    want = {kvq.DECODE_AUTO: kvq.DECODE_TENSOR_CORES, kvq.DECODE_CUDA_CORES: kvq.DECODE_CUDA_CORES,
+            kvq.DECODE_TCGEN05: kvq.DECODE_TCGEN05}[decode_path]
     assert kvq.kvq_get_decode_path(lay) == want
     assert kvq.kvq_get_decode_path(kvq.Layout(64, 4, 4, 4, 2, 32, 64, 64, 0)) == kvq.DECODE_CUDA_CORES
 

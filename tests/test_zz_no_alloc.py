@@ -30,7 +30,8 @@ def test_scratch_size_matches_header():
     assert m and int(m[1]) * int(m[2]) * int(m[3]) == kvq.KVQ_STATIC_SCRATCH_BYTES
 
 
-@pytest.mark.parametrize("path", [kvq.DECODE_AUTO, kvq.DECODE_CUDA_CORES], ids=["auto", "cuda_cores"])
+@pytest.mark.parametrize("path", [kvq.DECODE_AUTO, kvq.DECODE_CUDA_CORES, kvq.DECODE_TCGEN05],
+                         ids=["auto", "cuda_cores", "tcgen05"])
 def test_two_calls_in_a_row_match_workspace_entry_point(path):
     w = wl.Workload(name="no_alloc", batch=6, num_q_heads=16, num_kv_heads=4, head_dim=128, seq_len=0,
                     k_bits=4, v_bits=2, k_group=32, v_group=128, window=40, ragged=(1, 2500),
@@ -67,10 +68,21 @@ def test_two_calls_in_a_row_match_workspace_entry_point(path):
 
 
 def test_rejects_problem_larger_than_scratch():
-    """batch 1024 x 32 query heads needs more than 16 MiB of partials: refused on
-    the host with KVQ_ERR_WORKSPACE, nothing launched, outputs untouched."""
+    """On the two-phase tcgen05 path, whose split partials grow with the batch,
+    batch 1024 x 32 query heads needs more than 16 MiB: refused on the host
+    with KVQ_ERR_WORKSPACE, nothing launched, outputs untouched.  (The
+    persistent kernel's partials are bounded by the SM count: about 1.3 MB.)"""
     lay = kvq.Layout(128, 32, 8, 4, 2, 32, 128, 64, 0)
     batch, max_len = 1024, 4096
+    assert kvq.kvq_decode_workspace_bytes(lay, batch, max_len) < 2 * 1024 * 1024
+    kvq.kvq_set_decode_path(kvq.DECODE_TCGEN05)
+    try:
+        _reject_large(lay, batch, max_len)
+    finally:
+        kvq.kvq_set_decode_path(kvq.DECODE_AUTO)
+
+
+def _reject_large(lay, batch, max_len):
     assert kvq.kvq_decode_workspace_bytes(lay, batch, max_len) > kvq.KVQ_STATIC_SCRATCH_BYTES
     pt = torch.full((batch, 1), -1, dtype=torch.int32, device="cuda")
     cache = kvq.PagedCache.allocate(lay, pt, 1)
