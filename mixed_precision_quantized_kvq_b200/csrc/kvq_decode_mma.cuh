@@ -23,19 +23,22 @@
 // The newest W positions (bf16 window) run on bf16 mma m16n8k16 with the
 // query and the weights as bf16 (high, low) pairs.
 //
-// Work: the (sequence, kv-head) pairs are cut into units (UP pages of
-// quantized tokens, or WU window positions); the units are laid end to end
-// and each CTA (one per SM) takes an equal contiguous range, each of its
-// consumer warps an equal contiguous share of that.  A producer warp streams
-// the units' pages into a ring of shared-memory slots with 1-D bulk copies
-// (window rows with 16-byte cp.async into a swizzled layout), completion
-// counted on an mbarrier per slot.  Every consumer warp keeps its own online
-// softmax state; a pair that spans several warps is merged through shared
-// memory, a pair that spans several CTAs through a partial in the workspace
-// merged by the CTA that finishes it last (an atomic ticket per pair, reset
-// by that CTA).  Every mbarrier wait is bounded.
+// Work: the (sequence, kv-head) pairs are cut into units (one page of
+// quantized tokens, or WU window positions); the units are laid end to end,
+// each CTA (one per SM) takes an equal contiguous range and each of its warps
+// an equal contiguous share of that.  Every warp streams its own units
+// through a private ring of shared-memory slots, issuing the copies (1-D bulk
+// copies for pages, 16-byte cp.async into a swizzled layout for window rows)
+// two units ahead of the one it computes, with completion counted on an
+// mbarrier per slot; page-table entries are read one unit before they are
+// needed.  Every warp keeps its own online-softmax state; a pair that spans
+// several warps is merged through shared memory, a pair that spans several
+// CTAs through a partial in the workspace merged by the CTA that finishes it
+// last (an atomic ticket per pair, reset by that CTA).  Every mbarrier wait is
+// bounded.
 #pragma once
 
+#include <cuda.h>
 #include <math.h>
 
 #include "kvq_internal.cuh"
@@ -49,16 +52,14 @@ using namespace ptx;
 
 constexpr int D = 128;
 constexpr int NKG = 4;                         // key groups of 32 channels
-constexpr int NW = 8;                          // consumer warps
-constexpr int kThreads = 32 * (NW + 1);        // + one producer warp
-constexpr int kMaxSlots = 32;
+constexpr int kMaxWarps = 8;
+constexpr int kMaxSpw = 4;                     // ring slots per warp
 constexpr int kMaxBatch = 4096;                // schedule tables live in shared memory
 constexpr int kSmemBudget = 227 * 1024;
 constexpr unsigned FULL = 0xffffffffu;
 constexpr uint64_t kWaitNs = 1000000000ull;    // bound on every wait: 1 s
 constexpr uint64_t kDrainNs = 100000000ull;
 constexpr float kLn2 = 0.69314718055994530942f;
-
 
 // window positions per window unit: about the bytes of a quantized unit
 __host__ __device__ constexpr int window_unit(int qbytes) {
@@ -67,7 +68,7 @@ __host__ __device__ constexpr int window_unit(int qbytes) {
 
 template <int KB, int VB, int NH>
 struct Cfg {
-    static constexpr int UP = 2;                         // pages per quantized unit
+    static constexpr int UP = 1;                         // pages per quantized unit
     static constexpr int TOK = UP * kPage;               // tokens per quantized unit
     static constexpr int HS = NH / 4;                    // heads per thread
     static constexpr int NT = NH == 4 ? 2 : 3;           // 8-column tiles of (head, limb)
@@ -84,35 +85,41 @@ struct Cfg {
     static constexpr int QBYTES = OFF_VM + UP * VMETA;
     static constexpr int WU = window_unit(QBYTES);
     static constexpr int WROWS = WU * D * 2;             // bytes of the key (or value) rows of a window unit
-    static constexpr int SLOT = ((QBYTES > 2 * WROWS ? QBYTES : 2 * WROWS) + 127) & ~127;
-    static constexpr int QAREA = NH * 512 + NH * 32;     // per consumer warp: limb / bf16 query staging + scalars
+    // slots start 1024-byte aligned (the window tiles use the 128-byte TMA swizzle)
+    static constexpr int SLOT = ((QBYTES > 2 * WROWS ? QBYTES : 2 * WROWS) + 1023) & ~1023;
+    // eight warps when two slots each fit beside the per-warp areas, else four
+    static constexpr int NW = 8 * 2 * SLOT <= 160 * 1024 ? 8 : 4;
+    static constexpr int QAREA = NH * 512 + NH * 32;     // per warp: limb / bf16 query staging + scalars
     static_assert(KCODES % 16 == 0 && KMETA % 16 == 0 && VCODES % 16 == 0 && VMETA % 16 == 0, "bulk sizes");
 };
 
 struct Head {
-    uint64_t full[kMaxSlots];
-    uint64_t empty[kMaxSlots];
+    uint64_t full[kMaxWarps][kMaxSpw];
+    int upg[kMaxWarps][kMaxSpw];           // page of the unit in each slot (-1: none)
+    int cnt[kMaxWarps][2];                 // warps done with a pair they share, by owner warp and kind
+    int wfirst[kMaxWarps], wlast[kMaxWarps];   // pairs of each warp's first and last unit (-1: no units)
     int abort;
     int cs, ce, cta_pair0;                 // this CTA's unit range and the pair of its first unit
-    int wpair[NW][2];                      // pairs of a warp's incomplete segments, -1 if none
 };
 
-__host__ __device__ inline int off_sched() { return (int(sizeof(Head)) + 15) & ~15; }
-__host__ __device__ inline int off_qarea(int batch) { return (off_sched() + 8 * (batch + 1) + 127) & ~127; }
 // merge partials: per head a row of D outputs, the running maximum and the
 // weight sum, padded to PST floats so that every row starts 16-byte aligned
 constexpr int PST = D + 4;
 template <int NH>
 __host__ __device__ constexpr int part_floats() { return NH * PST; }
+
+__host__ __device__ inline int off_sched() { return (int(sizeof(Head)) + 15) & ~15; }
+__host__ __device__ inline int off_qarea(int batch) { return (off_sched() + 8 * (batch + 1) + 127) & ~127; }
 // a warp's first segment, when another warp began its pair, is parked here
-// until the merge: NW partials of g heads
+// until the merge: one partial of g heads per warp
 template <int KB, int VB, int NH>
 __host__ __device__ inline int off_park(int batch) {
-    return (off_qarea(batch) + NW * Cfg<KB, VB, NH>::QAREA + 127) & ~127;
+    return (off_qarea(batch) + Cfg<KB, VB, NH>::NW * Cfg<KB, VB, NH>::QAREA + 127) & ~127;
 }
+// (the ring itself starts at the next 1024-byte aligned address from here)
 template <int KB, int VB, int NH>
 __host__ __device__ inline int off_ring(int batch, int g) {
-    return (off_park<KB, VB, NH>(batch) + NW * g * PST * 4 + 127) & ~127;
+    return (off_park<KB, VB, NH>(batch) + Cfg<KB, VB, NH>::NW * g * PST * 4 + 127) & ~127;
 }
 
 // ---------------------------------------------------------------- helpers
@@ -273,9 +280,23 @@ __device__ __forceinline__ float limb_pv(int32_t l0, int32_t l1, int32_t l2) {
     else return fmaf(fmaf((float)l0, 256.0f, (float)l1), 256.0f, (float)l2);
 }
 
-// swizzle of the 16-byte chunks of window row t: ldmatrix rows (tokens
-// 2r or 2r+1 for scores, r or 8+r for ·V) fall in distinct bank groups
-__device__ __forceinline__ int wswz(int t) { return (t & 7) ^ ((t >> 3) & 1); }
+// Window rows arrive as TMA tiles of 16 rows x 64 channels (128 bytes) with
+// the 128-byte swizzle: in tile row r the 16-byte chunk c sits at position
+// c ^ (r mod 8), so the eight rows an ldmatrix reads (tokens r .. r+7 at one
+// chunk) fall in eight distinct bank groups.  Tiles of the key (or value)
+// rows of a unit: [16-row block][channel half] of 2 KB each.
+__device__ __forceinline__ uint32_t wrow(uint32_t base, int t, int c) {
+    const int tt = t & 15;
+    return base + (t >> 4) * 4096 + (c >> 3) * 2048 + tt * 128 + (((c & 7) ^ (tt & 7)) << 4);
+}
+// 2-D tiled TMA load (no multicast) of the box at (x, y) into shared memory
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
 
 // ---------------------------------------------------------------- schedule
 struct UnitPos {
@@ -315,14 +336,52 @@ struct State {
     }
 };
 
+// The query of kv-head h of sequence b: lane l gets channels 4l .. 4l+3 of
+// each of the NH heads (zeros for heads r >= g).  All loads are issued before
+// any is used.
+template <int NH>
+__device__ __forceinline__ void load_query(const Params& p, const void* q, int q_bf16, int b, int h, int lane,
+                                           float (&x)[NH][4]) {
+    const int g = p.g;
+    const size_t row0 = (size_t(b) * p.hq + size_t(h) * g) * D + 4 * lane;
+    if (q_bf16) {
+        uint2 v[NH];
+#pragma unroll
+        for (int r = 0; r < NH; ++r)
+            v[r] = r < g ? __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(q) + row0 +
+                                                                 size_t(r) * D))
+                         : make_uint2(0u, 0u);
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            x[r][0] = bf_lo(v[r].x);
+            x[r][1] = bf_hi(v[r].x);
+            x[r][2] = bf_lo(v[r].y);
+            x[r][3] = bf_hi(v[r].y);
+        }
+    } else {
+        float4 v[NH];
+#pragma unroll
+        for (int r = 0; r < NH; ++r)
+            v[r] = r < g ? __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(q) + row0 + size_t(r) * D))
+                         : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            x[r][0] = v[r].x;
+            x[r][1] = v[r].y;
+            x[r][2] = v[r].z;
+            x[r][3] = v[r].w;
+        }
+    }
+}
+
 // ---------------------------------------------------------------- query preparation
 // Query of kv-head h of sequence b: int8 limbs of the (rotated) query in the
 // score MMA's K order, staged in the warp's area, then read into the B
 // fragments; per head the limb unit (times sm_scale*log2 e) and the sums of
 // the rotated query per key group (times the same).
 template <int KB, int NH>
-__device__ void prep_query(const Params& p, const void* q, int q_bf16, int b, int h, uint8_t* qa, float sl2,
-                           int lane, uint32_t (&qb)[NKG][Cfg<KB, 1, NH>::NT][2], float (&cq)[NH / 4],
+__device__ void prep_query(const Params& p, const float (&xq)[NH][4], uint8_t* qa, float sl2, int lane,
+                           uint32_t (&qb)[NKG][Cfg<KB, 1, NH>::NT][2], float (&cq)[NH / 4],
                            float (&cz)[NH / 4][NKG]) {
     constexpr int NT = Cfg<KB, 1, NH>::NT;
     const int g = p.g;
@@ -330,24 +389,8 @@ __device__ void prep_query(const Params& p, const void* q, int q_bf16, int b, in
     float* qs = reinterpret_cast<float*>(qa + NH * 512);         // [head][8]
 #pragma unroll 1
     for (int r = 0; r < NH; ++r) {
-        float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        if (r < g) {
-            const size_t off = (size_t(b) * p.hq + size_t(h) * g + r) * D + 4 * lane;
-            if (q_bf16) {
-                const uint2 v = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(q) + off));
-                x[0] = bf_lo(v.x);
-                x[1] = bf_hi(v.x);
-                x[2] = bf_lo(v.y);
-                x[3] = bf_hi(v.y);
-            } else {
-                const float4 v = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(q) + off));
-                x[0] = v.x;
-                x[1] = v.y;
-                x[2] = v.z;
-                x[3] = v.w;
-            }
-            if (p.rotate) rotate_warp<D>(x, p.signs, lane);
-        }
+        float x[4] = {xq[r][0], xq[r][1], xq[r][2], xq[r][3]};
+        if (r < g && p.rotate) rotate_warp<D>(x, p.signs, lane);
         float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
         amax = warp_max(amax);
         float gs = (x[0] + x[1]) + (x[2] + x[3]);
@@ -406,27 +449,12 @@ __device__ void prep_query(const Params& p, const void* q, int q_bf16, int b, in
 template <int NH>
 __device__ void prep_window_query(const Params& p, const void* q, int q_bf16, int b, int h, uint8_t* qa, int lane) {
     __nv_bfloat16* wq = reinterpret_cast<__nv_bfloat16*>(qa);
-    const int g = p.g;
+    float xq[NH][4];
+    load_query<NH>(p, q, q_bf16, b, h, lane, xq);
     __syncwarp();
-#pragma unroll 1
+#pragma unroll
     for (int r = 0; r < NH; ++r) {
-        float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        if (r < g) {
-            const size_t off = (size_t(b) * p.hq + size_t(h) * g + r) * D + 4 * lane;
-            if (q_bf16) {
-                const uint2 v = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(q) + off));
-                x[0] = bf_lo(v.x);
-                x[1] = bf_hi(v.x);
-                x[2] = bf_lo(v.y);
-                x[3] = bf_hi(v.y);
-            } else {
-                const float4 v = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(q) + off));
-                x[0] = v.x;
-                x[1] = v.y;
-                x[2] = v.z;
-                x[3] = v.w;
-            }
-        }
+        const float* x = xq[r];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const __nv_bfloat16 hi = __float2bfloat16_rn(x[c]);
@@ -440,13 +468,14 @@ __device__ void prep_window_query(const Params& p, const void* q, int q_bf16, in
 
 // ---------------------------------------------------------------- the kernel
 template <int KB, int VB, int NH>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<KB, VB, NH>::NW * 32, 1)
 decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, const int32_t* __restrict__ lens,
                   const int max_len, const float sl2, float* __restrict__ out, float* __restrict__ lse,
-                  float* __restrict__ part, uint32_t* __restrict__ tickets, const int R,
-                  unsigned int* __restrict__ status) {
+                  float* __restrict__ part, uint32_t* __restrict__ tickets, const int SPW,
+                  unsigned int* __restrict__ status, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v) {
     using C = Cfg<KB, VB, NH>;
-    constexpr int HS = C::HS, NT = C::NT, TOK = C::TOK, WU = C::WU;
+    constexpr int HS = C::HS, NT = C::NT, TOK = C::TOK, WU = C::WU, NW = C::NW, kThreads = NW * 32;
     extern __shared__ __align__(1024) uint8_t smem[];
     Head& hd = *reinterpret_cast<Head*>(smem);
     const int B = p.batch, H = p.hkv, g = p.g;
@@ -454,8 +483,11 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
     int* LB = S + (B + 1);                                    // [B] clamped lengths  (S, LB: 8(B+1) bytes)
     uint8_t* qarea = smem + off_qarea(B);
     float* park = reinterpret_cast<float*>(smem + off_park<KB, VB, NH>(B));   // [NW][g][PST]
-    uint8_t* ring = smem + off_ring<KB, VB, NH>(B, p.g);
-    const uint32_t ring_s = smem_u32(ring);
+    uint8_t* ring;                                                          // [NW][SPW][SLOT], 1024-aligned
+    {
+        const uint32_t a = smem_u32(smem) + off_ring<KB, VB, NH>(B, p.g);
+        ring = smem + (((a + 1023u) & ~1023u) - smem_u32(smem));
+    }
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int W = p.W;
 
@@ -467,10 +499,8 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
         S[b + 1] = L == 0 ? 1 : (lq + TOK - 1) / TOK + (wl + WU - 1) / WU;
     }
     if (tid == 0) {
-        for (int i = 0; i < R; ++i) {
-            mbar_init(&hd.full[i], 1);
-            mbar_init(&hd.empty[i], 1);
-        }
+        for (int w = 0; w < NW; ++w)
+            for (int i = 0; i < SPW; ++i) mbar_init(&hd.full[w][i], 1);
         mbar_fence_init();
         hd.abort = 0;
     }
@@ -505,12 +535,27 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
             hd.cta_pair0 = -1;
         }
     }
-    if (tid < NW * 2) hd.wpair[tid >> 1][tid & 1] = -1;
+    if (tid < NW * 2) hd.cnt[tid >> 1][tid & 1] = 0;
+    if (tid < NW) {
+        const int n = base_n + (tid < rem ? 1 : 0), u0 = cs + tid * base_n + min(tid, rem);
+        int pf = -1, pl = -1;
+        if (n > 0) {
+            const UnitPos a = locate(S, B, H, u0), z = locate(S, B, H, u0 + n - 1);
+            pf = a.b * H + a.h;
+            pl = z.b * H + z.h;
+        }
+        hd.wfirst[tid] = pf;
+        hd.wlast[tid] = pl;
+    }
     __syncthreads();
     if (len <= 0) return;
 
-    auto wstart = [&](int w) { return cs + w * base_n + min(w, rem); };
-    auto wsize = [&](int w) { return base_n + (w < rem ? 1 : 0); };
+    const int w = warp, g8 = lane >> 2, tig = lane & 3;
+    const int nunits = base_n + (w < rem ? 1 : 0);
+    const int wbeg = cs + w * base_n + min(w, rem);
+    uint8_t* qa = qarea + w * C::QAREA;
+    uint8_t* wring = ring + size_t(w) * SPW * C::SLOT;
+    const uint32_t wring_s = smem_u32(wring);
     auto aborted = [&]() { return *reinterpret_cast<volatile int*>(&hd.abort) != 0; };
     // warp-collective bounded wait: every lane gets the same answer
     auto wait_bar = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -519,115 +564,83 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
         if (!ok && lane == 0 && atomicExch(&hd.abort, 1) == 0) atomicAdd(&status[0], 1u);
         return ok;
     };
+    // page-table entry of unit u when it is a quantized unit, else -1; the
+    // value is checked where it is used, so that the load is not waited for here
+    auto page_raw = [&](const UnitPos& u) -> int {
+        const int L = LB[u.b], lq = L - min(W, L), nq = (lq + TOK - 1) / TOK;
+        int v = -1;
+        if (L > 0 && u.j < nq && u.j < p.max_pages) v = __ldg(p.page_table + size_t(u.b) * p.max_pages + u.j);
+        return v;
+    };
+    auto next_unit = [&](UnitPos& u) {
+        if (++u.j == u.n) {
+            u.j = 0;
+            if (++u.h == H) {
+                u.h = 0;
+                if (u.b + 1 < B) ++u.b;
+            }
+            u.n = S[u.b + 1] - S[u.b];
+        }
+    };
+    int issued = 0;                     // units whose copies this warp has issued
+    // page-table entries of this warp's units: lane l holds those of units l, l+32, l+64, l+96
+    int pgr[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) pgr[r] = lane + 32 * r < nunits ? page_raw(locate(S, B, H, wbeg + lane + 32 * r)) : -1;
+    // copies of unit u (the warp's unit k) into this warp's slot `slot`
+    auto issue = [&](int slot, const UnitPos& u, int k) {
+        int raw;
+        if (k < 128) {
+            const int v = k < 32 ? pgr[0] : (k < 64 ? pgr[1] : (k < 96 ? pgr[2] : pgr[3]));
+            raw = __shfl_sync(FULL, v, k & 31);
+        } else {
+            raw = page_raw(u);
+        }
+        ++issued;
+        const int pg = (raw >= 0 && raw < p.num_pages) ? raw : -1;
+        if (lane == 0) hd.upg[w][slot] = pg;
+        uint64_t* bar = &hd.full[w][slot];
+        uint8_t* sl = wring + size_t(slot) * C::SLOT;
+        const int L = LB[u.b], wl = min(W, L), lq = L - wl, nq = (lq + TOK - 1) / TOK;
+        // one lane issues every copy of the unit (the copy instructions take
+        // warp-uniform operands: copies from several lanes would be serialised)
+        if (L > 0 && u.j < nq) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar, pg >= 0 ? uint32_t(C::PAGE_BYTES) : 0u);
+                if (pg >= 0) {
+                    const size_t blk = size_t(pg) * H + u.h;
+                    bulk_g2s(sl, p.k_codes + blk * C::KCODES, C::KCODES, bar);
+                    bulk_g2s(sl + C::OFF_KM, p.k_meta + blk * (kPage * NKG), C::KMETA, bar);
+                    bulk_g2s(sl + C::OFF_VC, p.v_codes + blk * C::VCODES, C::VCODES, bar);
+                    bulk_g2s(sl + C::OFF_VM, p.v_meta + blk * kPage, C::VMETA, bar);
+                }
+            }
+            __syncwarp();
+        } else if (L > 0) {
+            // window unit: ring slots [(j - nq) * WU, + WU) of the pair, whose rows are
+            // contiguous (the window's positions fill ring slots [0, min(W, L)); the
+            // order of positions does not matter to attention).  Keys then values, as
+            // 16-row x 64-channel TMA tiles.
+            const int y0 = (u.b * H + u.h) * W + (u.j - nq) * WU;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar, uint32_t(2 * WU * D * 2));
+                const uint32_t s0 = smem_u32(sl);
+#pragma unroll
+                for (int rb = 0; rb < WU / 16; ++rb)
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        tma_load_2d(s0 + rb * 4096 + half * 2048, &tm_k, half * 64, y0 + rb * 16, bar);
+                        tma_load_2d(s0 + C::WROWS + rb * 4096 + half * 2048, &tm_v, half * 64, y0 + rb * 16, bar);
+                    }
+            }
+            __syncwarp();
+        } else {
+            if (lane == 0) mbar_arrive_plain(bar);
+        }
+    };
 
-    if (warp == NW) {
-        // ============================================================ producer
-        int issued = 0;
-        for (int s0 = 0; s0 < len; s0 += 32) {
-            if (__any_sync(FULL, aborted())) break;
-            // lane i prepares step s0 + i: which unit, which pages, how many bytes
-            int kind = 0, ub = 0, uh = 0, pg0 = -1, pg1 = -1, w0 = 0, cnt = 0;
-            uint32_t bytes = 0;
-            const int s = s0 + lane;
-            if (s < len) {
-                const int w = s % NW, k = s / NW;
-                const UnitPos u = locate(S, B, H, wstart(w) + k);
-                ub = u.b;
-                uh = u.h;
-                const int L = LB[u.b], wl = min(W, L), lq = L - wl, nq = (lq + TOK - 1) / TOK;
-                if (L == 0) {
-                    kind = 0;
-                } else if (u.j < nq) {
-                    kind = 1;
-                    const int lp = u.j * C::UP;
-                    pg0 = lp * kPage < lq ? phys_page(p, u.b, lp) : -1;
-                    pg1 = (lp + 1) * kPage < lq ? phys_page(p, u.b, lp + 1) : -1;
-                    bytes = (pg0 >= 0 ? C::PAGE_BYTES : 0) + (pg1 >= 0 ? C::PAGE_BYTES : 0);
-                } else {
-                    kind = 2;
-                    w0 = lq + (u.j - nq) * WU;
-                    cnt = min(WU, L - w0);
-                }
-            }
-            const int n_here = min(32, len - s0);
-            for (int i = 0; i < n_here; ++i) {
-                const int st = s0 + i;
-                const int k_ = __shfl_sync(FULL, kind, i);
-                const int b_ = __shfl_sync(FULL, ub, i), h_ = __shfl_sync(FULL, uh, i);
-                const int p0 = __shfl_sync(FULL, pg0, i), p1 = __shfl_sync(FULL, pg1, i);
-                const int w0_ = __shfl_sync(FULL, w0, i), cnt_ = __shfl_sync(FULL, cnt, i);
-                const uint32_t by = __shfl_sync(FULL, bytes, i);
-                const int slot = st % R;
-                if (st >= R && !wait_bar(&hd.empty[slot], ((st / R) - 1) & 1)) break;
-                uint8_t* sl = ring + size_t(slot) * C::SLOT;
-                if (k_ == 1) {
-                    if (lane == 0) mbar_arrive_expect_tx(&hd.full[slot], by);
-                    __syncwarp();
-                    if (lane < 4 * C::UP) {
-                        const int e = lane >> 2, part_ = lane & 3;
-                        const int pg = e ? p1 : p0;
-                        if (pg >= 0) {
-                            const size_t blk = size_t(pg) * H + h_;
-                            const void* src;
-                            uint8_t* dst;
-                            uint32_t nb;
-                            if (part_ == 0) {
-                                src = p.k_codes + blk * C::KCODES;
-                                dst = sl + e * C::KCODES;
-                                nb = C::KCODES;
-                            } else if (part_ == 1) {
-                                src = p.k_meta + blk * (kPage * NKG);
-                                dst = sl + C::OFF_KM + e * C::KMETA;
-                                nb = C::KMETA;
-                            } else if (part_ == 2) {
-                                src = p.v_codes + blk * C::VCODES;
-                                dst = sl + C::OFF_VC + e * C::VCODES;
-                                nb = C::VCODES;
-                            } else {
-                                src = p.v_meta + blk * kPage;
-                                dst = sl + C::OFF_VM + e * C::VMETA;
-                                nb = C::VMETA;
-                            }
-                            bulk_g2s(dst, src, nb, &hd.full[slot]);
-                        }
-                    }
-                } else if (k_ == 2) {
-                    // WU rows of keys then values, 16 chunks of 16 bytes each; rows past
-                    // the window's end are zero-filled (their weights are 0, and the ·V
-                    // product must not meet non-finite values)
-                    const size_t rb = (size_t(b_) * H + h_) * size_t(W);
-                    const uint32_t base = ring_s + uint32_t(slot) * C::SLOT;
-                    for (int idx = lane; idx < 2 * WU * 16; idx += 32) {
-                        const int kv = idx / (WU * 16), rem_ = idx % (WU * 16);
-                        const int row = rem_ >> 4, c = rem_ & 15;
-                        const bool have = row < cnt_;
-                        const __nv_bfloat16* src = (kv ? p.v_win : p.k_win) +
-                                                   (rb + size_t(have ? (w0_ + row) % W : 0)) * D + c * 8;
-                        cp16_zfill(base + kv * C::WROWS + row * (D * 2) + ((c ^ wswz(row)) << 4), src, have);
-                    }
-                    cp_async_arrive(&hd.full[slot]);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_plain(&hd.full[slot]);
-                } else {
-                    if (lane == 0) mbar_arrive_plain(&hd.full[slot]);
-                }
-                issued = st + 1;
-            }
-        }
-        cp_async_wait_all();
-        if (aborted()) {
-            // nothing may still be copying into shared memory when the CTA exits
-            for (int st = max(0, issued - R); st < issued; ++st)
-                mbar_wait(&hd.full[st % R], (st / R) & 1, kDrainNs);
-        }
-    } else {
-        // ============================================================ consumers
-        const int w = warp, g8 = lane >> 2, tig = lane & 3;
-        const int nunits = wsize(w);
-        uint8_t* qa = qarea + w * C::QAREA;
-        State<NH> st;
-        st.reset();
-        int first_pair = -1, last_pair = -1;
+    State<NH> st;
+    st.reset();
 
         // normalized output and lse of heads tig (+4) of kv-head h of sequence b
         auto write_final = [&](const State<NH>& x, int b, int h) {
@@ -667,123 +680,187 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
                 }
             }
         };
-        // Merge the partials of pair P held by warps w.. of this CTA; output it
-        // if the pair lies inside the CTA, else hand a partial to the CTA that
-        // finishes the pair last.  Lane l owns channels 4l .. 4l+3.
-        auto merge_pair = [&](int P, int w0) {
-            const float* src[NW];
+        // Merge the partials of pair P held by warps wlo .. whi of this CTA
+        // (parked first segments, or final segments in the warps' rings).  A pair
+        // inside the CTA is output here.  A pair split between CTAs is merged by
+        // the first CTA that holds part of it (for which it is the last pair, done
+        // at the end of its range): every later CTA (for which it is the first
+        // pair, done early) stores its partial and counts it on the pair's ticket
+        // with a release increment; the merging CTA waits (bounded) for the count,
+        // merges, outputs and resets the ticket.  Lane l owns channels 4l .. 4l+3.
+        auto merge_pair = [&](int P, int wlo, int whi) {
+            const float* src[kMaxWarps];
             int np = 0;
-            for (int ww = w0; ww < NW; ++ww) {
-                const int slp = hd.wpair[ww][0] == P ? 0 : (hd.wpair[ww][1] == P ? 1 : -1);
-                if (slp < 0) break;
-                src[np++] = (slp == 0 ? park : reinterpret_cast<const float*>(ring)) + ww * g * PST;
+            for (int ww = wlo; ww <= whi; ++ww) {
+                const bool parked = hd.wfirst[ww] == P && hd.wlast[ww] != P;
+                src[np++] = parked ? park + ww * g * PST
+                                   : reinterpret_cast<const float*>(ring + size_t(ww) * SPW * C::SLOT);
             }
             const int b = P / H, h = P % H;
             const int n = S[b + 1] - S[b];
-            const long long u0 = (long long)H * S[b] + (long long)h * n;
-            const bool inside = u0 >= cs && u0 + n <= ce;
-            float* gdst = part + (size_t(cta) * 2 + (P == hd.cta_pair0 ? 0 : 1)) * part_floats<NH>();
-            for (int r = 0; r < g; ++r) {
-                float M = -INFINITY;
-                for (int i = 0; i < np; ++i) M = fmaxf(M, src[i][r * PST + D]);
-                const float mu = M == -INFINITY ? 0.0f : M;
-                float Ls = 0.0f, O[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            const long long u0 = (long long)H * S[b] + (long long)h * n, u1 = u0 + n;
+            float M[NH], Ls[NH], O[NH][4];
+#pragma unroll
+            for (int r = 0; r < NH; ++r) {
+                M[r] = -INFINITY;
+                Ls[r] = 0.0f;
+                O[r][0] = O[r][1] = O[r][2] = O[r][3] = 0.0f;
+                if (r >= g) continue;
+                for (int i = 0; i < np; ++i) M[r] = fmaxf(M[r], src[i][r * PST + D]);
+                const float mu = M[r] == -INFINITY ? 0.0f : M[r];
                 for (int i = 0; i < np; ++i) {
                     const float* pr = src[i] + r * PST;
                     const float wgt = pr[D] == -INFINITY ? 0.0f : ex2(pr[D] - mu);
-                    Ls = fmaf(pr[D + 1], wgt, Ls);
+                    Ls[r] = fmaf(pr[D + 1], wgt, Ls[r]);
                     const float4 v = *reinterpret_cast<const float4*>(pr + 4 * lane);
-                    O[0] = fmaf(v.x, wgt, O[0]);
-                    O[1] = fmaf(v.y, wgt, O[1]);
-                    O[2] = fmaf(v.z, wgt, O[2]);
-                    O[3] = fmaf(v.w, wgt, O[3]);
-                }
-                if (inside) {
-                    const size_t row = size_t(b) * p.hq + size_t(h) * g + r;
-                    const float inv = Ls > 0.0f ? 1.0f / Ls : 0.0f;
-                    *reinterpret_cast<float4*>(out + row * D + 4 * lane) =
-                        make_float4(O[0] * inv, O[1] * inv, O[2] * inv, O[3] * inv);
-                    if (lse && lane == 0) lse[row] = Ls > 0.0f ? (M + log2f(Ls)) * kLn2 : (Ls == 0.0f ? -INFINITY : NAN);
-                } else {
-                    *reinterpret_cast<float4*>(gdst + r * PST + 4 * lane) = make_float4(O[0], O[1], O[2], O[3]);
-                    if (lane == 0) {
-                        gdst[r * PST + D] = M;
-                        gdst[r * PST + D + 1] = Ls;
-                    }
+                    O[r][0] = fmaf(v.x, wgt, O[r][0]);
+                    O[r][1] = fmaf(v.y, wgt, O[r][1]);
+                    O[r][2] = fmaf(v.z, wgt, O[r][2]);
+                    O[r][3] = fmaf(v.w, wgt, O[r][3]);
                 }
             }
-            if (inside) return;
-            // ---- hand over: the CTA that arrives last merges every CTA's partial of P
-            __threadfence();
-            __syncwarp();
-            unsigned t = 0;
-            if (lane == 0) t = atomicAdd(&tickets[P], 1u);
-            t = __shfl_sync(FULL, t, 0);
-            const int ca = cta_of(u0, U, NC), cb = cta_of(u0 + n - 1, U, NC);
-            const unsigned need = unsigned(cb - ca);
-            if (t > need) {
-                if (lane == 0) atomicAdd(&status[1], 1u);
+            auto output = [&]() {
+#pragma unroll
+                for (int r = 0; r < NH; ++r) {
+                    if (r >= g) continue;
+                    const size_t row = size_t(b) * p.hq + size_t(h) * g + r;
+                    const float inv = Ls[r] > 0.0f ? 1.0f / Ls[r] : 0.0f;
+                    *reinterpret_cast<float4*>(out + row * D + 4 * lane) =
+                        make_float4(O[r][0] * inv, O[r][1] * inv, O[r][2] * inv, O[r][3] * inv);
+                    if (lse && lane == 0)
+                        lse[row] = Ls[r] > 0.0f ? (M[r] + log2f(Ls[r])) * kLn2 : (Ls[r] == 0.0f ? -INFINITY : NAN);
+                }
+            };
+            if (u0 >= cs && u1 <= ce) {
+                output();
                 return;
             }
-            if (t != need) return;
-            __threadfence();
-            for (int r = 0; r < g; ++r) {
-                float M = -INFINITY;
-                for (int c = ca; c <= cb; ++c) {
-                    const UnitPos f = locate(S, B, H, cta_start(c, U, NC));
-                    const float* pr = part + (size_t(c) * 2 + (f.b * H + f.h == P ? 0 : 1)) * part_floats<NH>() +
-                                      r * PST;
-                    M = fmaxf(M, __ldcg(pr + D));
+            const int ca = cta_of(u0, U, NC), cb = cta_of(u1 - 1, U, NC);
+            if (cta != ca) {
+                // a later CTA of the pair (its first pair): partial slot 0, then count it
+                float* gdst = part + size_t(cta) * 2 * part_floats<NH>();
+#pragma unroll
+                for (int r = 0; r < NH; ++r) {
+                    if (r >= g) continue;
+                    *reinterpret_cast<float4*>(gdst + r * PST + 4 * lane) = make_float4(O[r][0], O[r][1], O[r][2], O[r][3]);
+                    if (lane == 0) {
+                        gdst[r * PST + D] = M[r];
+                        gdst[r * PST + D + 1] = Ls[r];
+                    }
                 }
-                const float mu = M == -INFINITY ? 0.0f : M;
-                float Ls = 0.0f, O[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                for (int c = ca; c <= cb; ++c) {
-                    const UnitPos f = locate(S, B, H, cta_start(c, U, NC));
-                    const float* pr = part + (size_t(c) * 2 + (f.b * H + f.h == P ? 0 : 1)) * part_floats<NH>() +
-                                      r * PST;
-                    const float mc = __ldcg(pr + D);
-                    const float wgt = mc == -INFINITY ? 0.0f : ex2(mc - mu);
-                    Ls = fmaf(__ldcg(pr + D + 1), wgt, Ls);
-                    const float4 v = __ldcg(reinterpret_cast<const float4*>(pr + 4 * lane));
-                    O[0] = fmaf(v.x, wgt, O[0]);
-                    O[1] = fmaf(v.y, wgt, O[1]);
-                    O[2] = fmaf(v.z, wgt, O[2]);
-                    O[3] = fmaf(v.w, wgt, O[3]);
-                }
-                const size_t row = size_t(b) * p.hq + size_t(h) * g + r;
-                const float inv = Ls > 0.0f ? 1.0f / Ls : 0.0f;
-                *reinterpret_cast<float4*>(out + row * D + 4 * lane) =
-                    make_float4(O[0] * inv, O[1] * inv, O[2] * inv, O[3] * inv);
-                if (lse && lane == 0) lse[row] = Ls > 0.0f ? (M + log2f(Ls)) * kLn2 : (Ls == 0.0f ? -INFINITY : NAN);
+                __threadfence();                  // each lane's stores, before the count
+                __syncwarp();
+                if (lane == 0) atomicAdd(tickets + P, 1u);
+                return;
             }
+            // ---- the merging CTA: wait for the cb - ca partials of the later CTAs
+            const unsigned need = unsigned(cb - ca);
+            unsigned got = 0;
+            if (lane == 0) {
+                const uint64_t t0 = globaltimer();
+                for (;;) {
+                    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(got) : "l"(tickets + P) : "memory");
+                    if (got >= need || globaltimer() - t0 > kWaitNs) break;
+                    __nanosleep(64);
+                }
+                if (got < need) atomicAdd(&status[0], 1u);
+                if (got > need) atomicAdd(&status[1], 1u);
+            }
+            got = __shfl_sync(FULL, got, 0);
+            __threadfence();
+            if (got < need) {
+#pragma unroll
+                for (int r = 0; r < NH; ++r) Ls[r] = NAN;
+            }
+            for (int c0 = ca + 1; c0 <= cb; c0 += 2) {
+                float mc[2][NH], lc[2][NH];
+                float4 oc[2][NH];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int c = c0 + u;
+                    const bool have = c <= cb;
+                    const float* pc = part + size_t(have ? c : cb) * 2 * part_floats<NH>();
+#pragma unroll
+                    for (int r = 0; r < NH; ++r) {
+                        const bool hr = have && r < g;
+                        mc[u][r] = hr ? __ldcg(pc + r * PST + D) : -INFINITY;
+                        lc[u][r] = hr ? __ldcg(pc + r * PST + D + 1) : 0.0f;
+                        oc[u][r] = hr ? __ldcg(reinterpret_cast<const float4*>(pc + r * PST + 4 * lane))
+                                      : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+#pragma unroll
+                    for (int r = 0; r < NH; ++r) {
+                        const float mn = fmaxf(M[r], mc[u][r]);
+                        const float mu = mn == -INFINITY ? 0.0f : mn;
+                        const float al = M[r] == -INFINITY ? 0.0f : ex2(M[r] - mu);
+                        const float wgt = mc[u][r] == -INFINITY ? 0.0f : ex2(mc[u][r] - mu);
+                        M[r] = mn;
+                        Ls[r] = fmaf(lc[u][r], wgt, Ls[r] * al);
+                        O[r][0] = fmaf(oc[u][r].x, wgt, O[r][0] * al);
+                        O[r][1] = fmaf(oc[u][r].y, wgt, O[r][1] * al);
+                        O[r][2] = fmaf(oc[u][r].z, wgt, O[r][2] * al);
+                        O[r][3] = fmaf(oc[u][r].w, wgt, O[r][3] * al);
+                    }
+            }
+            output();
             if (lane == 0) tickets[P] = 0u;       // ready for the next call
         };
 
-        if (nunits > 0) {
-            UnitPos pos = locate(S, B, H, wstart(w));
-            int seg_j0 = pos.j;
-            uint32_t qb[NKG][NT][2];
-            float cq[HS], cz[HS][NKG];
-            bool wq_ready = false;
-            prep_query<KB, NH>(p, q, q_bf16, pos.b, pos.h, qa, sl2, lane, qb, cq, cz);
-            for (int k = 0; k < nunits; ++k) {
-                const int s = k * NW + w, slot = s % R;
-                const int L = LB[pos.b], wl = min(W, L), lq = L - wl, nq = (lq + TOK - 1) / TOK;
-                const uint32_t sl = ring_s + uint32_t(slot) * C::SLOT;
-                const bool kind_q = L > 0 && pos.j < nq;
-                const bool kind_w = L > 0 && pos.j >= nq;
-                int pres0 = 0, pres1 = 0;
-                if (kind_q) {
-                    const int lp = pos.j * C::UP;
-                    pres0 = lp * kPage < lq && phys_page(p, pos.b, lp) >= 0;
-                    pres1 = (lp + 1) * kPage < lq && phys_page(p, pos.b, lp + 1) >= 0;
-                }
-                if (kind_w && !wq_ready) {
-                    prep_window_query<NH>(p, q, q_bf16, pos.b, pos.h, qa, lane);
-                    wq_ready = true;
-                }
-                const bool ok = wait_bar(&hd.full[slot], (s / R) & 1);
-                if (!ok) st.bad = true;
+        // warp holding unit u of this CTA's range
+        auto warp_of = [&](long long u) -> int {
+            const long long x = u - cs, big = (long long)rem * (base_n + 1);
+            return x < big ? int(x / (base_n + 1)) : rem + int((x - big) / base_n);
+        };
+        // This warp has stored its partial of shared pair P: count it, and the
+        // last of the CTA's warps that hold a part of P merges them.
+        auto finish_shared = [&](int P) {
+            const int b = P / H, h = P % H, n = S[b + 1] - S[b];
+            const long long u0 = (long long)H * S[b] + (long long)h * n, u1 = u0 + n;
+            const int wlo = warp_of(u0 > cs ? u0 : cs), whi = warp_of((u1 < ce ? u1 : ce) - 1);
+            const int kind = hd.wlast[wlo] == P ? 1 : 0;
+            __threadfence_block();
+            __syncwarp();
+            int old = 0;
+            if (lane == 0) old = atomicAdd(&hd.cnt[wlo][kind], 1);
+            old = __shfl_sync(FULL, old, 0);
+            if (old != whi - wlo) return;
+            __threadfence_block();
+            merge_pair(P, wlo, whi);
+        };
+
+    if (nunits > 0) {
+        // ---- the first pair's query (loaded before the copies so that its loads
+        // are not queued behind them), then the first SPW units: page lookups in
+        // parallel, then the copies
+        UnitPos pos = locate(S, B, H, wbeg), ip = pos;
+        float xq0[NH][4];
+        load_query<NH>(p, q, q_bf16, pos.b, pos.h, lane, xq0);
+        for (int i = 0; i < SPW && i < nunits; ++i) {
+            issue(i, ip, i);
+            next_unit(ip);
+        }
+        int seg_j0 = pos.j;
+        uint32_t qb[NKG][NT][2];
+        float cq[HS], cz[HS][NKG];
+        bool wq_ready = false;
+        prep_query<KB, NH>(p, xq0, qa, sl2, lane, qb, cq, cz);
+        for (int k = 0; k < nunits; ++k) {
+            const int slot = k % SPW;
+            const int L = LB[pos.b], wl = min(W, L), lq = L - wl, nq = (lq + TOK - 1) / TOK;
+            const uint32_t sl = wring_s + uint32_t(slot) * C::SLOT;
+            const bool kind_q = L > 0 && pos.j < nq;
+            const bool kind_w = L > 0 && pos.j >= nq;
+            const int pres1 = 0;
+            if (kind_w && !wq_ready) {
+                prep_window_query<NH>(p, q, q_bf16, pos.b, pos.h, qa, lane);
+                wq_ready = true;
+            }
+            const bool ok = wait_bar(&hd.full[w][slot], (k / SPW) & 1);
+            if (!ok) st.bad = true;
+            const int pres0 = kind_q && hd.upg[w][slot] >= 0;
                 if (ok && kind_q) {
                     // ---------------------------------------------- quantized unit
                     const int tok0 = pos.j * TOK;
@@ -807,10 +884,7 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
                                 kfrag<KB>(kc, tA, tB, grp, tig, a);
                                 int32_t d[NT][4];
 #pragma unroll
-                                for (int nt = 0; nt < NT; ++nt) {
-                                    d[nt][0] = d[nt][1] = d[nt][2] = d[nt][3] = 0;
-                                    mma_u8s8(d[nt], a, qb[grp][nt][0], qb[grp][nt][1]);
-                                }
+                                for (int nt = 0; nt < NT; ++nt) mma_u8s8_z(d[nt], a, qb[grp][nt][0], qb[grp][nt][1]);
                                 const float2 fA = half2f(mAw[grp]), fB = half2f(mBw[grp]);
 #pragma unroll
                                 for (int hs = 0; hs < HS; ++hs) {
@@ -912,13 +986,14 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
                         const int chA = 16 * mt + g8, chB = chA + 8;
                         int32_t acc[NT][4];
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0;
-#pragma unroll
                         for (int s4 = 0; s4 < 2 * C::UP; ++s4) {
                             uint32_t a[4];
                             vfrag<VB>(sl + C::OFF_VC + (s4 >> 1) * C::VCODES, chA, chB, s4 & 1, tig, a);
 #pragma unroll
-                            for (int nt = 0; nt < NT; ++nt) mma_u8u8(acc[nt], a, bq[s4][nt][0], bq[s4][nt][1]);
+                            for (int nt = 0; nt < NT; ++nt) {
+                                if (s4 == 0) mma_u8u8_z(acc[nt], a, bq[s4][nt][0], bq[s4][nt][1]);
+                                else mma_u8u8(acc[nt], a, bq[s4][nt][0], bq[s4][nt][1]);
+                            }
                         }
 #pragma unroll
                         for (int hs = 0; hs < HS; ++hs) {
@@ -932,40 +1007,48 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
                 } else if (ok && kind_w) {
                     // ---------------------------------------------- window unit
                     constexpr int NB = WU / 16;
-                    const int w0 = lq + (pos.j - nq) * WU, cnt = min(WU, L - w0);
+                    const int cnt = min(WU, wl - (pos.j - nq) * WU);    // ring slots of the unit that hold tokens
                     const __nv_bfloat16* wq = reinterpret_cast<const __nv_bfloat16*>(qa);
                     const uint32_t kbase = sl, vbase = sl + C::WROWS;
+                    if (cnt < WU) {
+                        // value rows past the window's end: zeros, so that their zero weights
+                        // meet finite values in the ·V product
+                        for (int idx = lane; idx < (WU - cnt) * 16; idx += 32)
+                            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(wrow(vbase, cnt + (idx >> 4), idx & 15)),
+                                         "r"(0)
+                                         : "memory");
+                        fence_proxy_async();    // before a later bulk copy into this slot
+                        __syncwarp();
+                    }
                     float sw[HS][NB][2];
 #pragma unroll
                     for (int bb = 0; bb < NB; ++bb) {
                         float d[HS][4];
-#pragma unroll
-                        for (int hs = 0; hs < HS; ++hs) d[hs][0] = d[hs][1] = d[hs][2] = d[hs][3] = 0.0f;
                         const int mi = lane >> 3, r = lane & 7;
-                        const int tq = 16 * bb + 2 * r + (mi & 1);
+                        const int tq = 16 * bb + r + 8 * (mi & 1);      // score rows: tokens in order
 #pragma unroll
                         for (int s8 = 0; s8 < 8; ++s8) {
                             uint32_t a[4];
-                            const int ch = 2 * s8 + (mi >> 1);
-                            ldsm_x4(a, kbase + tq * (D * 2) + ((ch ^ wswz(tq)) << 4));
+                            ldsm_x4(a, wrow(kbase, tq, 2 * s8 + (mi >> 1)));
 #pragma unroll
                             for (int hs = 0; hs < HS; ++hs) {
                                 const int head = (g8 >> 1) + 4 * hs, hl = g8 & 1;
                                 const __nv_bfloat16* qq = wq + (head * 2 + hl) * D + 16 * s8 + 2 * tig;
                                 const uint32_t b0 = *reinterpret_cast<const uint32_t*>(qq);
                                 const uint32_t b1 = *reinterpret_cast<const uint32_t*>(qq + 8);
-                                mma_bf16(d[hs], a, b0, b1);
+                                if (s8 == 0) mma_bf16_z(d[hs], a, b0, b1);
+                                else mma_bf16(d[hs], a, b0, b1);
                             }
                         }
-                        const int t0 = 16 * bb + 2 * g8;
+                        const int t0 = 16 * bb + g8;                   // rows g8 and g8 + 8
 #pragma unroll
                         for (int hs = 0; hs < HS; ++hs) {
                             sw[hs][bb][0] = t0 < cnt ? (d[hs][0] + d[hs][1]) * sl2 : -INFINITY;
-                            sw[hs][bb][1] = t0 + 1 < cnt ? (d[hs][2] + d[hs][3]) * sl2 : -INFINITY;
+                            sw[hs][bb][1] = t0 + 8 < cnt ? (d[hs][2] + d[hs][3]) * sl2 : -INFINITY;
                         }
                     }
                     float alpha[HS];
-                    uint32_t phi[HS][NB], plo[HS][NB];
+                    uint32_t px[HS][NB][2];          // per row (g8, g8 + 8): bf16 {high, low} of p
 #pragma unroll
                     for (int hs = 0; hs < HS; ++hs) {
                         float mx = -INFINITY;
@@ -982,37 +1065,42 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
                             const float p0 = sw[hs][bb][0] == -INFINITY ? 0.0f : ex2(sw[hs][bb][0] - mu);
                             const float p1 = sw[hs][bb][1] == -INFINITY ? 0.0f : ex2(sw[hs][bb][1] - mu);
                             ls += p0 + p1;
-                            phi[hs][bb] = pack_bf16(p0, p1);
-                            plo[hs][bb] = pack_bf16(p0 - bf_lo(phi[hs][bb]), p1 - bf_hi(phi[hs][bb]));
+                            const uint32_t hi = pack_bf16(p0, p1);
+                            const uint32_t lo = pack_bf16(p0 - bf_lo(hi), p1 - bf_hi(hi));
+                            px[hs][bb][0] = __byte_perm(hi, lo, 0x5410);   // row g8:     {high, low}
+                            px[hs][bb][1] = __byte_perm(hi, lo, 0x7632);   // row g8 + 8: {high, low}
                         }
                         st.l[hs] = fmaf(st.l[hs], alpha[hs], ls);
                         st.pz[hs] *= alpha[hs];
                     }
+                    // B fragment of the weights: tokens 2tig, 2tig+1 (and 8 more) of column
+                    // (head g8/2, high or low part g8%2), held by the lanes of rows 2tig, 2tig+1
                     uint32_t bv[NB][HS][2];
-                    const int srcA = 4 * tig + (g8 >> 1), odd = g8 & 1;
+                    const int se = 4 * (2 * tig) + (g8 >> 1), so = se + 4;
+                    const uint32_t sel = (g8 & 1) ? 0x7632u : 0x5410u;
 #pragma unroll
                     for (int bb = 0; bb < NB; ++bb)
 #pragma unroll
                         for (int hs = 0; hs < HS; ++hs)
 #pragma unroll
                             for (int hf = 0; hf < 2; ++hf) {
-                                const uint32_t x0 = __shfl_sync(FULL, phi[hs][bb], srcA + 16 * hf);
-                                const uint32_t x1 = __shfl_sync(FULL, plo[hs][bb], srcA + 16 * hf);
-                                bv[bb][hs][hf] = odd ? x1 : x0;
+                                const uint32_t xe = __shfl_sync(FULL, px[hs][bb][hf], se);
+                                const uint32_t xo = __shfl_sync(FULL, px[hs][bb][hf], so);
+                                bv[bb][hs][hf] = __byte_perm(xe, xo, sel);
                             }
 #pragma unroll
                     for (int mt = 0; mt < 8; ++mt) {
                         float dv[HS][4];
-#pragma unroll
-                        for (int hs = 0; hs < HS; ++hs) dv[hs][0] = dv[hs][1] = dv[hs][2] = dv[hs][3] = 0.0f;
                         const int mi = lane >> 3, r = lane & 7;
 #pragma unroll
                         for (int bb = 0; bb < NB; ++bb) {
                             uint32_t a[4];
-                            const int tv = 16 * bb + r + 8 * (mi >> 1), ch = 2 * mt + (mi & 1);
-                            ldsm_x4_t(a, vbase + tv * (D * 2) + ((ch ^ wswz(tv)) << 4));
+                            ldsm_x4_t(a, wrow(vbase, 16 * bb + r + 8 * (mi >> 1), 2 * mt + (mi & 1)));
 #pragma unroll
-                            for (int hs = 0; hs < HS; ++hs) mma_bf16(dv[hs], a, bv[bb][hs][0], bv[bb][hs][1]);
+                            for (int hs = 0; hs < HS; ++hs) {
+                                if (bb == 0) mma_bf16_z(dv[hs], a, bv[bb][hs][0], bv[bb][hs][1]);
+                                else mma_bf16(dv[hs], a, bv[bb][hs][0], bv[bb][hs][1]);
+                            }
                         }
 #pragma unroll
                         for (int hs = 0; hs < HS; ++hs) {
@@ -1022,7 +1110,11 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
                     }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive_plain(&hd.empty[slot]);
+                // ---- the slot is free: copies of unit k + SPW into it
+                if (k + SPW < nunits && !aborted()) {
+                    issue(slot, ip, k + SPW);
+                    next_unit(ip);
+                }
 
                 // ---- end of a segment: the pair is done, or the warp's range ends
                 const bool pair_end = pos.j + 1 == pos.n, last_unit = k + 1 == nunits;
@@ -1030,14 +1122,13 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
                     const int pair = pos.b * H + pos.h;
                     if (seg_j0 == 0 && pair_end) {            // the whole pair: final output
                         write_final(st, pos.b, pos.h);
-                        st.reset();
-                    } else if (!last_unit) {                  // the warp's first segment, begun by another warp
-                        store_partial(st, park + w * g * PST);
-                        first_pair = pair;
-                        st.reset();
-                    } else {                                  // the warp's last segment, taken up by another
-                        last_pair = pair;
+                    } else {
+                        // a pair shared with other warps (or CTAs): the first segment is parked,
+                        // the final one goes to this warp's ring (its copies are all consumed)
+                        store_partial(st, last_unit ? reinterpret_cast<float*>(wring) : park + w * g * PST);
+                        finish_shared(pair);
                     }
+                    st.reset();
                 }
                 // ---- next unit
                 if (!pair_end) {
@@ -1051,28 +1142,18 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
                     pos.n = S[pos.b + 1] - S[pos.b];
                     seg_j0 = 0;
                     wq_ready = false;
-                    prep_query<KB, NH>(p, q, q_bf16, pos.b, pos.h, qa, sl2, lane, qb, cq, cz);
+                    float xq[NH][4];
+                    load_query<NH>(p, q, q_bf16, pos.b, pos.h, lane, xq);
+                    prep_query<KB, NH>(p, xq, qa, sl2, lane, qb, cq, cz);
                 }
             }
-        }
 
-        // ---- merge of pairs split between warps (and CTAs); the ring is free now
-        named_barrier(1, NW * 32);
-        float* pbase = reinterpret_cast<float*>(ring);
-        if (last_pair >= 0) store_partial(st, pbase + w * g * PST);
-        if (lane == 0) {            // slot 0: the parked first segment, slot 1: the final segment
-            hd.wpair[w][0] = first_pair;
-            hd.wpair[w][1] = last_pair;
-        }
-        named_barrier(1, NW * 32);
-#pragma unroll 1
-        for (int sl = 0; sl < 2; ++sl) {
-            const int P = hd.wpair[w][sl];
-            if (P < 0) continue;
-            if (w > 0 && (hd.wpair[w - 1][0] == P || hd.wpair[w - 1][1] == P)) continue;   // not the owner
-            merge_pair(P, w);
+        if (aborted()) {
+            // nothing may still be copying into shared memory when the CTA exits
+            for (int u = max(0, issued - SPW); u < issued; ++u) mbar_wait(&hd.full[w][u % SPW], (u / SPW) & 1, kDrainNs);
         }
     }
+
 }
 
 }  // namespace mma
