@@ -27,16 +27,23 @@ def small(**kw):
 def rotated_pair(w, lens, steps=0):
     """A pair whose oracle side quantizes the library's rotated keys (the
     rotation itself agrees with the oracle's fp64 product to round-off; the
-    codes are compared from the rotated fp32 keys on)."""
+    codes are compared from the rotated fp32 keys on).  Positions that stay
+    in the bf16 window keep their unrotated keys."""
     pair = Pair(w, lens, steps=steps)
-    kr, vr, _, _, cu, _ = wl.prefill(w, lens, with_f32=False)
+    kr, vr, kf, _, cu, _ = wl.prefill(w, lens)
     rot = torch.empty(kr.shape, dtype=torch.float32, device="cuda")
     kvq.kvq_rotate_keys(pair.glay, torch_raw(kr), rot)
+    rot = rot.cpu().numpy()
+    # rotated rows where the position ends up quantized, raw rows in the window
+    rows = kf.astype(np.float32).copy()
+    for b in range(w.batch):
+        nq = max(0, int(lens[b]) - w.window)
+        rows[cu[b]:cu[b] + nq] = rot[cu[b]:cu[b] + nq]
     olay = oracle.Layout.from_workload(w.with_(rotate_keys=False))
     pair.ocache = oracle.Cache(olay, w.batch, pair.pt, pair.num_pages)
     pair.lens[:] = 0
     pair.glens.zero_()
-    pair.append(kr, vr, cu, oracle_k=np.ascontiguousarray(rot.cpu().numpy()), oracle_dtype=oracle.IN_F32)
+    pair.append(kr, vr, cu, oracle_k=np.ascontiguousarray(rows), oracle_dtype=oracle.IN_F32)
     return pair
 
 
