@@ -193,8 +193,8 @@ int kvq_get_decode_path(const kvq_layout* layout);
  *                  kernel then writes NaN for the outputs it could not
  *                  finish; 0 in normal operation)
  *   bad_tickets    merge tickets found above their count, i.e. a workspace
- *                  that was not zero-filled before its first use (those
- *                  outputs are not written)
+ *                  that was not zero-filled before its first use (the
+ *                  outputs of those (sequence, kv-head) pairs are not valid)
  * Either pointer may be NULL; clear != 0 resets both counters.  This call
  * reads device memory synchronously (it waits for the device), unlike every
  * other entry point; use it for checking, not inside a timed loop. */

@@ -99,7 +99,6 @@ struct Head {
     int cnt[kMaxWarps][2];                 // warps done with a pair they share, by owner warp and kind
     int wfirst[kMaxWarps], wlast[kMaxWarps];   // pairs of each warp's first and last unit (-1: no units)
     int abort;
-    int cs, ce, cta_pair0;                 // this CTA's unit range and the pair of its first unit
 };
 
 // merge partials: per head a row of D outputs, the running maximum and the
@@ -313,8 +312,6 @@ __device__ __forceinline__ UnitPos locate(const int* S, int B, int H, int u) {
     const int n = S[lo + 1] - S[lo], r = u - H * S[lo];
     return {lo, r / n, r % n, n};
 }
-__device__ __forceinline__ int cta_start(long long c, long long U, long long C) { return (int)((c * U) / C); }
-__device__ __forceinline__ int cta_of(long long u, long long U, long long C) { return (int)(((u + 1) * C - 1) / U); }
 
 // ---------------------------------------------------------------- per-thread state
 template <int NH>
@@ -380,7 +377,7 @@ __device__ __forceinline__ void load_query(const Params& p, const void* q, int q
 // fragments; per head the limb unit (times sm_scale*log2 e) and the sums of
 // the rotated query per key group (times the same).
 template <int KB, int NH>
-__device__ void prep_query(const Params& p, const float (&xq)[NH][4], uint8_t* qa, float sl2, int lane,
+__device__ __forceinline__ void prep_query(const Params& p, const float (&xq)[NH][4], uint8_t* qa, float sl2, int lane,
                            uint32_t (&qb)[NKG][Cfg<KB, 1, NH>::NT][2], float (&cq)[NH / 4],
                            float (&cz)[NH / 4][NKG]) {
     constexpr int NT = Cfg<KB, 1, NH>::NT;
@@ -447,7 +444,7 @@ __device__ void prep_query(const Params& p, const float (&xq)[NH][4], uint8_t* q
 // Unrotated query as bf16 (high, low) pairs for the window scores:
 // [head][high/low][channel] bf16 in the warp's area.
 template <int NH>
-__device__ void prep_window_query(const Params& p, const void* q, int q_bf16, int b, int h, uint8_t* qa, int lane) {
+__device__ __forceinline__ void prep_window_query(const Params& p, const void* q, int q_bf16, int b, int h, uint8_t* qa, int lane) {
     __nv_bfloat16* wq = reinterpret_cast<__nv_bfloat16*>(qa);
     float xq[NH][4];
     load_query<NH>(p, q, q_bf16, b, h, lane, xq);
@@ -466,10 +463,235 @@ __device__ void prep_window_query(const Params& p, const void* q, int q_bf16, in
     __syncwarp();
 }
 
+// ---------------------------------------------------------------- end of a segment
+// What the end of a segment reads besides the warp's accumulators.
+struct Split {
+    int U, NC;              // units, CTAs with units (NC <= U)
+    int q, r;               // U = q NC + r
+    float inv_nc, inv_u;    // 1 / NC, NC / U
+};
+__device__ __forceinline__ Split make_split(int U, int NC) {
+    return {U, NC, U / NC, U % NC, 1.0f / float(NC), float(NC) / float(U)};
+}
+// floor(t / NC) for 0 <= t < 2^24, from the float quotient corrected by one step
+__device__ __forceinline__ int div_nc(int t, const Split& s) {
+    int d = int(float(t) * s.inv_nc);
+    if ((d + 1) * s.NC <= t) ++d;
+    if (d * s.NC > t) --d;
+    return d;
+}
+// first unit of CTA c: floor(c U / NC) = c q + floor(c r / NC)
+__device__ __forceinline__ int cta_start(int c, const Split& s) { return c * s.q + div_nc(c * s.r, s); }
+// CTA holding unit u
+__device__ __forceinline__ int cta_of(int u, const Split& s) {
+    int c = min(s.NC - 1, int(float(u) * s.inv_u));
+    while (c + 1 < s.NC && cta_start(c + 1, s) <= u) ++c;
+    while (c > 0 && cta_start(c, s) > u) --c;
+    return c;
+}
+
+struct SegCtx {
+    Head* hd;
+    const int* S;           // units per pair, prefix over sequences
+    float* park;            // [NW][g][PST] parked first segments
+    uint8_t* ring;          // the warps' rings (a warp's final partial goes to its first slot)
+    float* out;
+    float* lse;
+    float* part;            // [CTAs][2][NH][PST] partials of pairs split between CTAs
+    uint32_t* tickets;
+    unsigned* status;
+    int hq, g, H, SPW, slot_bytes, cs, ce, base_n, rem;
+    Split sp;
+};
+
+// normalized output and lse of heads tig (+4) of kv-head h of sequence b
+template <int NH>
+__device__ __forceinline__ void write_final(const SegCtx& c, const State<NH>& x, int b, int h, int lane) {
+    const int g8 = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int hs = 0; hs < NH / 4; ++hs) {
+        const float lt = grp_sum(x.l[hs]), zt = grp_sum(x.pz[hs]);
+        const int r = tig + 4 * hs;
+        if (r >= c.g) continue;
+        const size_t row = size_t(b) * c.hq + size_t(h) * c.g + r;
+        const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            c.out[row * D + 16 * mt + g8] = x.bad ? NAN : (x.o[hs][mt][0] + zt) * inv;
+            c.out[row * D + 16 * mt + g8 + 8] = x.bad ? NAN : (x.o[hs][mt][1] + zt) * inv;
+        }
+        if (c.lse && g8 == 0)
+            c.lse[row] = x.bad ? NAN : (lt > 0.0f ? (x.m[hs] + log2f(lt)) * kLn2 : -INFINITY);
+    }
+}
+
+// unnormalized partial: per head D outputs (including the zero-point term),
+// the running maximum (log2 domain) and the weight sum
+template <int NH>
+__device__ __forceinline__ void store_partial(const SegCtx& c, const State<NH>& x, float* dst, int lane) {
+    const int g8 = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int hs = 0; hs < NH / 4; ++hs) {
+        const float lt = grp_sum(x.l[hs]), zt = grp_sum(x.pz[hs]);
+        const int r = tig + 4 * hs;
+        if (r >= c.g) continue;
+        float* d = dst + r * PST;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            d[16 * mt + g8] = x.bad ? NAN : x.o[hs][mt][0] + zt;
+            d[16 * mt + g8 + 8] = x.bad ? NAN : x.o[hs][mt][1] + zt;
+        }
+        if (g8 == 0) {
+            d[D] = x.bad ? 0.0f : x.m[hs];
+            d[D + 1] = x.bad ? NAN : lt;
+        }
+    }
+}
+
+__device__ __forceinline__ float4 ld_relaxed_v4(const float* a) {
+    float4 v;
+    asm volatile("ld.relaxed.gpu.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(a)
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ float2 ld_relaxed_v2(const float* a) {
+    float2 v;
+    asm volatile("ld.relaxed.gpu.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(a) : "memory");
+    return v;
+}
+
+// Merge the partials of pair P: first those of warps wlo .. whi of this CTA
+// (parked first segments, or final segments in the warps' rings); a pair
+// inside the CTA is then output.  For a pair split between CTAs every CTA
+// stores its merged partial and then takes a ticket of the pair; the CTA that
+// takes the last ticket merges the other CTAs' partials, outputs and resets
+// the ticket, so that no CTA waits for another.  One loop over all the
+// partials keeps the code short (it runs cold, once or twice per warp).
+// Lane l owns channels 4l .. 4l+3.
+template <int NH>
+__device__ __forceinline__ void merge_pair(const SegCtx& c, int P, int wlo, int whi, int lane) {
+    const int g = c.g, H = c.H;
+    const int b = P / H, h = P - b * H;
+    const int n = c.S[b + 1] - c.S[b];
+    const int u0 = H * c.S[b] + h * n, u1 = u0 + n;
+    const bool inside = u0 >= c.cs && u1 <= c.ce;
+    const int cta = blockIdx.x;
+    const int ca = inside ? cta : cta_of(u0, c.sp), cb = inside ? cta : cta_of(u1 - 1, c.sp);
+    const int nloc = whi - wlo + 1, nall = nloc + (cb - ca);
+    float M[NH], Ls[NH], O[NH][4];
+#pragma unroll
+    for (int r = 0; r < NH; ++r) {
+        M[r] = -INFINITY;
+        Ls[r] = 0.0f;
+        O[r][0] = O[r][1] = O[r][2] = O[r][3] = 0.0f;
+    }
+#pragma unroll 1
+    for (int it = 0; it < nall; ++it) {
+        if (it == nloc) {
+            // this CTA's partial goes to its slot (0 when P is the CTA's first pair, else 1)
+            float* gdst = c.part + (size_t(cta) * 2 + (u0 > c.cs ? 1 : 0)) * part_floats<NH>();
+#pragma unroll
+            for (int r = 0; r < NH; ++r) {
+                if (r >= g) continue;
+                *reinterpret_cast<float4*>(gdst + r * PST + 4 * lane) = make_float4(O[r][0], O[r][1], O[r][2], O[r][3]);
+                if (lane == 0) *reinterpret_cast<float2*>(gdst + r * PST + D) = make_float2(M[r], Ls[r]);
+            }
+            __syncwarp();                     // every lane's stores, then lane 0's release
+            unsigned old = 0;
+            if (lane == 0) old = atom_add_acq_rel_gpu(c.tickets + P, 1u);
+            old = __shfl_sync(FULL, old, 0);
+            const unsigned need = unsigned(cb - ca);   // tickets taken before the last one
+            if (old < need) return;
+            if (old > need) {
+                // the ticket was not zero at the start of the call: output NaN
+                if (lane == 0) atomicAdd(&c.status[1], 1u);
+#pragma unroll
+                for (int r = 0; r < NH; ++r) Ls[r] = NAN;
+            }
+            __syncwarp();                     // lane 0's acquire, then every lane's loads
+        }
+        const float* src;
+        if (it < nloc) {
+            const int ww = wlo + it;
+            const bool parked = c.hd->wfirst[ww] == P && c.hd->wlast[ww] != P;
+            src = parked ? c.park + ww * g * PST
+                         : reinterpret_cast<const float*>(c.ring + size_t(ww) * c.SPW * c.slot_bytes);
+        } else {
+            int cc = ca + (it - nloc);
+            if (cc >= cta) ++cc;              // every CTA of the pair but this one
+            src = c.part + (size_t(cc) * 2 + (u0 > cta_start(cc, c.sp) ? 1 : 0)) * part_floats<NH>();
+        }
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            if (r >= g) continue;
+            const float2 ml = ld_relaxed_v2(src + r * PST + D);
+            const float4 v = ld_relaxed_v4(src + r * PST + 4 * lane);
+            const float mn = fmaxf(M[r], ml.x);
+            const float mu = mn == -INFINITY ? 0.0f : mn;
+            const float al = M[r] == -INFINITY ? 0.0f : ex2(M[r] - mu);
+            const float wgt = ml.x == -INFINITY ? 0.0f : ex2(ml.x - mu);
+            M[r] = mn;
+            Ls[r] = fmaf(ml.y, wgt, Ls[r] * al);
+            O[r][0] = fmaf(v.x, wgt, O[r][0] * al);
+            O[r][1] = fmaf(v.y, wgt, O[r][1] * al);
+            O[r][2] = fmaf(v.z, wgt, O[r][2] * al);
+            O[r][3] = fmaf(v.w, wgt, O[r][3] * al);
+        }
+    }
+    if (!inside && lane == 0) c.tickets[P] = 0u;   // ready for the next call
+    // lane r < g: the reciprocal weight sum and the lse of head r
+    float myL = Ls[0], myM = M[0];
+#pragma unroll
+    for (int r = 1; r < NH; ++r)
+        if (lane == r) myL = Ls[r], myM = M[r];
+    const float inv = myL > 0.0f ? __fdividef(1.0f, myL) : 0.0f;   // within 2 ulp
+    const size_t row0 = size_t(b) * c.hq + size_t(h) * g;
+    if (c.lse && lane < g)
+        c.lse[row0 + lane] = myL > 0.0f ? (myM + log2f(myL)) * kLn2 : (myL == 0.0f ? -INFINITY : NAN);
+#pragma unroll
+    for (int r = 0; r < NH; ++r) {
+        const float ir = __shfl_sync(FULL, inv, r);
+        if (r < g)
+            *reinterpret_cast<float4*>(c.out + (row0 + r) * D + 4 * lane) =
+                make_float4(O[r][0] * ir, O[r][1] * ir, O[r][2] * ir, O[r][3] * ir);
+    }
+}
+
+// The segment of warp w that ends here covers part of kv-head h of sequence b,
+// shared with other warps or CTAs: the partial is stored (the warp's first
+// segment to its parking area, its final one to its ring, whose copies are all
+// consumed) and counted.  Returns the pair when this warp was the last of the
+// CTA's warps that hold a part of it (it then owes the merge of warps
+// wlo .. whi, done after its units, so that the merge code runs once per warp
+// at most twice and never between two units), else -1.
+template <int NH>
+__device__ __forceinline__ int post_segment(const SegCtx& c, const State<NH>& x, int b, int h, bool last_unit, int w,
+                                            int lane, int& wlo, int& whi) {
+    store_partial<NH>(c, x, last_unit ? reinterpret_cast<float*>(c.ring + size_t(w) * c.SPW * c.slot_bytes)
+                                      : c.park + w * c.g * PST, lane);
+    const int P = b * c.H + h, n = c.S[b + 1] - c.S[b];
+    const int u0 = c.H * c.S[b] + h * n, u1 = u0 + n;
+    // warp holding unit u of this CTA's range
+    auto warp_of = [&](int u) -> int {
+        const int x0 = u - c.cs, big = c.rem * (c.base_n + 1);
+        return x0 < big ? x0 / (c.base_n + 1) : c.rem + (x0 - big) / c.base_n;
+    };
+    wlo = warp_of(u0 > c.cs ? u0 : c.cs);
+    whi = warp_of((u1 < c.ce ? u1 : c.ce) - 1);
+    const int kind = c.hd->wlast[wlo] == P ? 1 : 0;
+    __syncwarp();                             // every lane's stores, then lane 0's release
+    int old = 0;
+    if (lane == 0) old = atom_add_acq_rel_cta(&c.hd->cnt[wlo][kind], 1);
+    old = __shfl_sync(FULL, old, 0);
+    return old == whi - wlo ? P : -1;
+}
+
 // ---------------------------------------------------------------- the kernel
 template <int KB, int VB, int NH>
 __global__ void __launch_bounds__(Cfg<KB, VB, NH>::NW * 32, 1)
-decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, const int32_t* __restrict__ lens,
+decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, const int q_bf16, const int32_t* __restrict__ lens,
                   const int max_len, const float sl2, float* __restrict__ out, float* __restrict__ lse,
                   float* __restrict__ part, uint32_t* __restrict__ tickets, const int SPW,
                   unsigned int* __restrict__ status, const __grid_constant__ CUtensorMap tm_k,
@@ -521,20 +743,11 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
     }
     __syncthreads();
     // every active CTA gets at least one unit (U >= 1: a sequence has at least one unit per kv-head)
-    const long long U = (long long)H * S[B], NC = min((long long)gridDim.x, U);
+    const int U = H * S[B], NC = min(int(gridDim.x), U);
+    const Split sp = make_split(U, NC);
     const int cta = blockIdx.x;
-    const int cs = cta < NC ? cta_start(cta, U, NC) : 0, ce = cta < NC ? cta_start(cta + 1, U, NC) : 0;
+    const int cs = cta < NC ? cta_start(cta, sp) : 0, ce = cta < NC ? cta_start(cta + 1, sp) : 0;
     const int len = ce - cs, base_n = len / NW, rem = len % NW;
-    if (tid == 0) {
-        hd.cs = cs;
-        hd.ce = ce;
-        if (len > 0) {
-            const UnitPos u0 = locate(S, B, H, cs);
-            hd.cta_pair0 = u0.b * H + u0.h;
-        } else {
-            hd.cta_pair0 = -1;
-        }
-    }
     if (tid < NW * 2) hd.cnt[tid >> 1][tid & 1] = 0;
     if (tid < NW) {
         const int n = base_n + (tid < rem ? 1 : 0), u0 = cs + tid * base_n + min(tid, rem);
@@ -602,26 +815,38 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
         uint64_t* bar = &hd.full[w][slot];
         uint8_t* sl = wring + size_t(slot) * C::SLOT;
         const int L = LB[u.b], wl = min(W, L), lq = L - wl, nq = (lq + TOK - 1) / TOK;
-        // one lane issues every copy of the unit (the copy instructions take
-        // warp-uniform operands: copies from several lanes would be serialised)
         if (L > 0 && u.j < nq) {
-            if (lane == 0) {
-                mbar_arrive_expect_tx(bar, pg >= 0 ? uint32_t(C::PAGE_BYTES) : 0u);
-                if (pg >= 0) {
-                    const size_t blk = size_t(pg) * H + u.h;
-                    bulk_g2s(sl, p.k_codes + blk * C::KCODES, C::KCODES, bar);
-                    bulk_g2s(sl + C::OFF_KM, p.k_meta + blk * (kPage * NKG), C::KMETA, bar);
-                    bulk_g2s(sl + C::OFF_VC, p.v_codes + blk * C::VCODES, C::VCODES, bar);
-                    bulk_g2s(sl + C::OFF_VM, p.v_meta + blk * kPage, C::VMETA, bar);
-                }
+            // a page: the four blocks in 16-byte pieces from every lane (a bulk copy
+            // holds the lane that issues it for about a hundred cycles, so four of
+            // them per unit cost more than these); each lane's copies arrive on the
+            // slot's barrier when they land, lane 0 adds the barrier's one arrival
+            if (pg >= 0) {
+                const size_t blk = size_t(pg) * H + u.h;
+                const uint32_t s0 = smem_u32(sl);
+                const uint8_t* kc = p.k_codes + blk * C::KCODES;
+                const uint8_t* km = reinterpret_cast<const uint8_t*>(p.k_meta + blk * (kPage * NKG));
+                const uint8_t* vc = p.v_codes + blk * C::VCODES;
+                const uint8_t* vm = reinterpret_cast<const uint8_t*>(p.v_meta + blk * kPage);
+#pragma unroll
+                for (int i = lane; i < C::KCODES / 16; i += 32) cp16(s0 + 16 * i, kc + 16 * i);
+#pragma unroll
+                for (int i = lane; i < C::KMETA / 16; i += 32) cp16(s0 + C::OFF_KM + 16 * i, km + 16 * i);
+#pragma unroll
+                for (int i = lane; i < C::VCODES / 16; i += 32) cp16(s0 + C::OFF_VC + 16 * i, vc + 16 * i);
+#pragma unroll
+                for (int i = lane; i < C::VMETA / 16; i += 32) cp16(s0 + C::OFF_VM + 16 * i, vm + 16 * i);
+                cp_async_arrive(bar);
             }
             __syncwarp();
+            if (lane == 0) mbar_arrive_plain(bar);
         } else if (L > 0) {
             // window unit: ring slots [(j - nq) * WU, + WU) of the pair, whose rows are
             // contiguous (the window's positions fill ring slots [0, min(W, L)); the
             // order of positions does not matter to attention).  Keys then values, as
             // 16-row x 64-channel TMA tiles.
             const int y0 = (u.b * H + u.h) * W + (u.j - nq) * WU;
+            fence_proxy_async();        // every lane's earlier writes to the slot (cp.async pieces) first
+            __syncwarp();
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar, uint32_t(2 * WU * D * 2));
                 const uint32_t s0 = smem_u32(sl);
@@ -642,202 +867,13 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
     State<NH> st;
     st.reset();
 
-        // normalized output and lse of heads tig (+4) of kv-head h of sequence b
-        auto write_final = [&](const State<NH>& x, int b, int h) {
-#pragma unroll
-            for (int hs = 0; hs < HS; ++hs) {
-                const float lt = grp_sum(x.l[hs]), zt = grp_sum(x.pz[hs]);
-                const int r = tig + 4 * hs;
-                if (r >= g) continue;
-                const size_t row = size_t(b) * p.hq + size_t(h) * g + r;
-                const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
-#pragma unroll
-                for (int mt = 0; mt < 8; ++mt) {
-                    out[row * D + 16 * mt + g8] = x.bad ? NAN : (x.o[hs][mt][0] + zt) * inv;
-                    out[row * D + 16 * mt + g8 + 8] = x.bad ? NAN : (x.o[hs][mt][1] + zt) * inv;
-                }
-                if (lse && g8 == 0)
-                    lse[row] = x.bad ? NAN : (lt > 0.0f ? (x.m[hs] + log2f(lt)) * kLn2 : -INFINITY);
-            }
-        };
-        // unnormalized partial: per head D outputs (including the zero-point
-        // term), the running maximum (log2 domain) and the weight sum
-        auto store_partial = [&](const State<NH>& x, float* dst) {
-#pragma unroll
-            for (int hs = 0; hs < HS; ++hs) {
-                const float lt = grp_sum(x.l[hs]), zt = grp_sum(x.pz[hs]);
-                const int r = tig + 4 * hs;
-                if (r >= g) continue;
-                float* d = dst + r * PST;
-#pragma unroll
-                for (int mt = 0; mt < 8; ++mt) {
-                    d[16 * mt + g8] = x.bad ? NAN : x.o[hs][mt][0] + zt;
-                    d[16 * mt + g8 + 8] = x.bad ? NAN : x.o[hs][mt][1] + zt;
-                }
-                if (g8 == 0) {
-                    d[D] = x.bad ? 0.0f : x.m[hs];
-                    d[D + 1] = x.bad ? NAN : lt;
-                }
-            }
-        };
-        // Merge the partials of pair P held by warps wlo .. whi of this CTA
-        // (parked first segments, or final segments in the warps' rings).  A pair
-        // inside the CTA is output here.  A pair split between CTAs is merged by
-        // the first CTA that holds part of it (for which it is the last pair, done
-        // at the end of its range): every later CTA (for which it is the first
-        // pair, done early) stores its partial and counts it on the pair's ticket
-        // with a release increment; the merging CTA waits (bounded) for the count,
-        // merges, outputs and resets the ticket.  Lane l owns channels 4l .. 4l+3.
-        auto merge_pair = [&](int P, int wlo, int whi) {
-            const float* src[kMaxWarps];
-            int np = 0;
-            for (int ww = wlo; ww <= whi; ++ww) {
-                const bool parked = hd.wfirst[ww] == P && hd.wlast[ww] != P;
-                src[np++] = parked ? park + ww * g * PST
-                                   : reinterpret_cast<const float*>(ring + size_t(ww) * SPW * C::SLOT);
-            }
-            const int b = P / H, h = P % H;
-            const int n = S[b + 1] - S[b];
-            const long long u0 = (long long)H * S[b] + (long long)h * n, u1 = u0 + n;
-            float M[NH], Ls[NH], O[NH][4];
-#pragma unroll
-            for (int r = 0; r < NH; ++r) {
-                M[r] = -INFINITY;
-                Ls[r] = 0.0f;
-                O[r][0] = O[r][1] = O[r][2] = O[r][3] = 0.0f;
-                if (r >= g) continue;
-                for (int i = 0; i < np; ++i) M[r] = fmaxf(M[r], src[i][r * PST + D]);
-                const float mu = M[r] == -INFINITY ? 0.0f : M[r];
-                for (int i = 0; i < np; ++i) {
-                    const float* pr = src[i] + r * PST;
-                    const float wgt = pr[D] == -INFINITY ? 0.0f : ex2(pr[D] - mu);
-                    Ls[r] = fmaf(pr[D + 1], wgt, Ls[r]);
-                    const float4 v = *reinterpret_cast<const float4*>(pr + 4 * lane);
-                    O[r][0] = fmaf(v.x, wgt, O[r][0]);
-                    O[r][1] = fmaf(v.y, wgt, O[r][1]);
-                    O[r][2] = fmaf(v.z, wgt, O[r][2]);
-                    O[r][3] = fmaf(v.w, wgt, O[r][3]);
-                }
-            }
-            auto output = [&]() {
-#pragma unroll
-                for (int r = 0; r < NH; ++r) {
-                    if (r >= g) continue;
-                    const size_t row = size_t(b) * p.hq + size_t(h) * g + r;
-                    const float inv = Ls[r] > 0.0f ? 1.0f / Ls[r] : 0.0f;
-                    *reinterpret_cast<float4*>(out + row * D + 4 * lane) =
-                        make_float4(O[r][0] * inv, O[r][1] * inv, O[r][2] * inv, O[r][3] * inv);
-                    if (lse && lane == 0)
-                        lse[row] = Ls[r] > 0.0f ? (M[r] + log2f(Ls[r])) * kLn2 : (Ls[r] == 0.0f ? -INFINITY : NAN);
-                }
-            };
-            if (u0 >= cs && u1 <= ce) {
-                output();
-                return;
-            }
-            const int ca = cta_of(u0, U, NC), cb = cta_of(u1 - 1, U, NC);
-            if (cta != ca) {
-                // a later CTA of the pair (its first pair): partial slot 0, then count it
-                float* gdst = part + size_t(cta) * 2 * part_floats<NH>();
-#pragma unroll
-                for (int r = 0; r < NH; ++r) {
-                    if (r >= g) continue;
-                    *reinterpret_cast<float4*>(gdst + r * PST + 4 * lane) = make_float4(O[r][0], O[r][1], O[r][2], O[r][3]);
-                    if (lane == 0) {
-                        gdst[r * PST + D] = M[r];
-                        gdst[r * PST + D + 1] = Ls[r];
-                    }
-                }
-                __threadfence();                  // each lane's stores, before the count
-                __syncwarp();
-                if (lane == 0) atomicAdd(tickets + P, 1u);
-                return;
-            }
-            // ---- the merging CTA: wait for the cb - ca partials of the later CTAs
-            const unsigned need = unsigned(cb - ca);
-            unsigned got = 0;
-            if (lane == 0) {
-                const uint64_t t0 = globaltimer();
-                for (;;) {
-                    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(got) : "l"(tickets + P) : "memory");
-                    if (got >= need || globaltimer() - t0 > kWaitNs) break;
-                    __nanosleep(64);
-                }
-                if (got < need) atomicAdd(&status[0], 1u);
-                if (got > need) atomicAdd(&status[1], 1u);
-            }
-            got = __shfl_sync(FULL, got, 0);
-            __threadfence();
-            if (got < need) {
-#pragma unroll
-                for (int r = 0; r < NH; ++r) Ls[r] = NAN;
-            }
-            for (int c0 = ca + 1; c0 <= cb; c0 += 2) {
-                float mc[2][NH], lc[2][NH];
-                float4 oc[2][NH];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int c = c0 + u;
-                    const bool have = c <= cb;
-                    const float* pc = part + size_t(have ? c : cb) * 2 * part_floats<NH>();
-#pragma unroll
-                    for (int r = 0; r < NH; ++r) {
-                        const bool hr = have && r < g;
-                        mc[u][r] = hr ? __ldcg(pc + r * PST + D) : -INFINITY;
-                        lc[u][r] = hr ? __ldcg(pc + r * PST + D + 1) : 0.0f;
-                        oc[u][r] = hr ? __ldcg(reinterpret_cast<const float4*>(pc + r * PST + 4 * lane))
-                                      : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 2; ++u)
-#pragma unroll
-                    for (int r = 0; r < NH; ++r) {
-                        const float mn = fmaxf(M[r], mc[u][r]);
-                        const float mu = mn == -INFINITY ? 0.0f : mn;
-                        const float al = M[r] == -INFINITY ? 0.0f : ex2(M[r] - mu);
-                        const float wgt = mc[u][r] == -INFINITY ? 0.0f : ex2(mc[u][r] - mu);
-                        M[r] = mn;
-                        Ls[r] = fmaf(lc[u][r], wgt, Ls[r] * al);
-                        O[r][0] = fmaf(oc[u][r].x, wgt, O[r][0] * al);
-                        O[r][1] = fmaf(oc[u][r].y, wgt, O[r][1] * al);
-                        O[r][2] = fmaf(oc[u][r].z, wgt, O[r][2] * al);
-                        O[r][3] = fmaf(oc[u][r].w, wgt, O[r][3] * al);
-                    }
-            }
-            output();
-            if (lane == 0) tickets[P] = 0u;       // ready for the next call
-        };
-
-        // warp holding unit u of this CTA's range
-        auto warp_of = [&](long long u) -> int {
-            const long long x = u - cs, big = (long long)rem * (base_n + 1);
-            return x < big ? int(x / (base_n + 1)) : rem + int((x - big) / base_n);
-        };
-        // This warp has stored its partial of shared pair P: count it, and the
-        // last of the CTA's warps that hold a part of P merges them.
-        auto finish_shared = [&](int P) {
-            const int b = P / H, h = P % H, n = S[b + 1] - S[b];
-            const long long u0 = (long long)H * S[b] + (long long)h * n, u1 = u0 + n;
-            const int wlo = warp_of(u0 > cs ? u0 : cs), whi = warp_of((u1 < ce ? u1 : ce) - 1);
-            const int kind = hd.wlast[wlo] == P ? 1 : 0;
-            __threadfence_block();
-            __syncwarp();
-            int old = 0;
-            if (lane == 0) old = atomicAdd(&hd.cnt[wlo][kind], 1);
-            old = __shfl_sync(FULL, old, 0);
-            if (old != whi - wlo) return;
-            __threadfence_block();
-            merge_pair(P, wlo, whi);
-        };
-
     if (nunits > 0) {
         // ---- the first pair's query (loaded before the copies so that its loads
         // are not queued behind them), then the first SPW units: page lookups in
         // parallel, then the copies
         UnitPos pos = locate(S, B, H, wbeg), ip = pos;
-        float xq0[NH][4];
-        load_query<NH>(p, q, q_bf16, pos.b, pos.h, lane, xq0);
+        float xq[NH][4];
+        load_query<NH>(p, q, q_bf16, pos.b, pos.h, lane, xq);
         for (int i = 0; i < SPW && i < nunits; ++i) {
             issue(i, ip, i);
             next_unit(ip);
@@ -845,9 +881,15 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
         int seg_j0 = pos.j;
         uint32_t qb[NKG][NT][2];
         float cq[HS], cz[HS][NKG];
-        bool wq_ready = false;
-        prep_query<KB, NH>(p, xq0, qa, sl2, lane, qb, cq, cz);
+        bool q_ready = false, wq_ready = false;
+        int mp0 = -1, mlo0 = 0, mhi0 = 0, mp1 = -1, mlo1 = 0, mhi1 = 0;   // merges this warp owes
         for (int k = 0; k < nunits; ++k) {
+            // the pair's query (one place for the first pair and every later one)
+            if (!q_ready) {
+                if (k > 0) load_query<NH>(p, q, q_bf16, pos.b, pos.h, lane, xq);
+                prep_query<KB, NH>(p, xq, qa, sl2, lane, qb, cq, cz);
+                q_ready = true;
+            }
             const int slot = k % SPW;
             const int L = LB[pos.b], wl = min(W, L), lq = L - wl, nq = (lq + TOK - 1) / TOK;
             const uint32_t sl = wring_s + uint32_t(slot) * C::SLOT;
@@ -1119,14 +1161,20 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
                 // ---- end of a segment: the pair is done, or the warp's range ends
                 const bool pair_end = pos.j + 1 == pos.n, last_unit = k + 1 == nunits;
                 if (pair_end || last_unit) {
-                    const int pair = pos.b * H + pos.h;
-                    if (seg_j0 == 0 && pair_end) {            // the whole pair: final output
-                        write_final(st, pos.b, pos.h);
+                    const SegCtx sc{&hd, S, park, ring, out, lse, part, tickets, status, p.hq, g, H, SPW, C::SLOT,
+                                    cs, ce, base_n, rem, sp};
+                    if (seg_j0 == 0 && pair_end) {    // the whole pair in this warp: final output
+                        write_final<NH>(sc, st, pos.b, pos.h, lane);
                     } else {
-                        // a pair shared with other warps (or CTAs): the first segment is parked,
-                        // the final one goes to this warp's ring (its copies are all consumed)
-                        store_partial(st, last_unit ? reinterpret_cast<float*>(wring) : park + w * g * PST);
-                        finish_shared(pair);
+                        int lo, hi;
+                        const int P = post_segment<NH>(sc, st, pos.b, pos.h, last_unit, w, lane, lo, hi);
+                        if (P >= 0) {
+                            if (mp0 < 0) {
+                                mp0 = P, mlo0 = lo, mhi0 = hi;
+                            } else {
+                                mp1 = P, mlo1 = lo, mhi1 = hi;
+                            }
+                        }
                     }
                     st.reset();
                 }
@@ -1141,12 +1189,21 @@ decode_mma_kernel(const Params p, const void* __restrict__ q, const int q_bf16, 
                     }
                     pos.n = S[pos.b + 1] - S[pos.b];
                     seg_j0 = 0;
-                    wq_ready = false;
-                    float xq[NH][4];
-                    load_query<NH>(p, q, q_bf16, pos.b, pos.h, lane, xq);
-                    prep_query<KB, NH>(p, xq, qa, sl2, lane, qb, cq, cz);
+                    q_ready = wq_ready = false;
                 }
             }
+
+        // ---- the merges this warp owes (the partials stay where they were stored:
+        // parking areas and the rings of warps that are done with their units)
+        if (mp0 >= 0) {
+            const SegCtx sc{&hd, S, park, ring, out, lse, part, tickets, status, p.hq, g, H, SPW, C::SLOT,
+                            cs, ce, base_n, rem, sp};
+#pragma unroll 1
+            for (int i = 0; i < 2; ++i) {
+                const int P = i ? mp1 : mp0;
+                if (P >= 0) merge_pair<NH>(sc, P, i ? mlo1 : mlo0, i ? mhi1 : mhi0, lane);
+            }
+        }
 
         if (aborted()) {
             // nothing may still be copying into shared memory when the CTA exits

@@ -71,18 +71,15 @@ cudaError_t launch_one(const Params& p, const void* q, int q_bf16, const int32_t
     CUtensorMap mk, mv;
     const cudaError_t em = window_maps(p, &mk, &mv);
     if (em != cudaSuccess) return em;
-    // cooperative launch: the CTAs that merge pairs split between CTAs wait (bounded)
-    // for the partials of later CTAs, so every CTA of the grid must be resident
+    // no CTA waits for another (pairs split between CTAs are merged by the CTA
+    // that finishes last), so a plain launch of one CTA per SM
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(ctas);
     cfg.blockDim = dim3(C::NW * 32);
     cfg.dynamicSmemBytes = bytes;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
     return cudaLaunchKernelEx(&cfg, kern, p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, spw, status, mk,
                               mv);
 }

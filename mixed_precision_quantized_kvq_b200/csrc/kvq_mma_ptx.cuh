@@ -64,6 +64,10 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t saddr) {
                  : "memory");
 }
 
+// 16-byte cp.async (L2 only)
+__device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
 // 16-byte cp.async (L2 only); src_bytes 0 writes zeros and reads nothing
 __device__ __forceinline__ void cp16_zfill(uint32_t dst, const void* src, bool have) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(have ? 16 : 0)
@@ -75,6 +79,22 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
     asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Atomic adds with acquire-release semantics (release publishes the stores
+// that precede them in this thread, and, through a preceding warp barrier,
+// those of its warp; acquire makes the releases they read from visible).
+// Unlike a sequentially consistent fence they do not wait for the memory
+// traffic of the rest of the SM.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* a, unsigned v) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(a), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ int atom_add_acq_rel_cta(int* a, int v) {
+    int old;
+    asm volatile("atom.acq_rel.cta.shared::cta.add.s32 %0, [%1], %2;" : "=r"(old) : "r"(smem_u32(a)), "r"(v) : "memory");
+    return old;
+}
 
 __device__ __forceinline__ void mbar_arrive_plain(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
