@@ -118,7 +118,7 @@ __host__ __device__ inline int off_park(int batch) {
 // (the ring itself starts at the next 1024-byte aligned address from here)
 template <int KB, int VB, int NH>
 __host__ __device__ inline int off_ring(int batch, int g) {
-    return (off_park<KB, VB, NH>(batch) + Cfg<KB, VB, NH>::NW * g * PST * 4 + 127) & ~127;
+    return (off_park<KB, VB, NH>(batch) + Cfg<KB, VB, NH>::NW * NH * PST * 4 + 127) & ~127;
 }
 
 // ---------------------------------------------------------------- helpers
@@ -493,7 +493,7 @@ __device__ __forceinline__ int cta_of(int u, const Split& s) {
 struct SegCtx {
     Head* hd;
     const int* S;           // units per pair, prefix over sequences
-    float* park;            // [NW][g][PST] parked first segments
+    float* park;            // [NW][NH][PST] parked first segments
     uint8_t* ring;          // the warps' rings (a warp's final partial goes to its first slot)
     float* out;
     float* lse;
@@ -566,9 +566,10 @@ __device__ __forceinline__ float2 ld_relaxed_v2(const float* a) {
 // (parked first segments, or final segments in the warps' rings); a pair
 // inside the CTA is then output.  For a pair split between CTAs every CTA
 // stores its merged partial and then takes a ticket of the pair; the CTA that
-// takes the last ticket merges the other CTAs' partials, outputs and resets
-// the ticket, so that no CTA waits for another.  One loop over all the
-// partials keeps the code short (it runs cold, once or twice per warp).
+// takes the last ticket merges every CTA's partial in CTA order (the result
+// does not depend on the order the CTAs finished in), outputs and resets the
+// ticket, so that no CTA waits for another.  One loop over all the partials
+// keeps the code short (it runs cold, once or twice per warp).
 // Lane l owns channels 4l .. 4l+3.
 template <int NH>
 __device__ __forceinline__ void merge_pair(const SegCtx& c, int P, int wlo, int whi, int lane) {
@@ -579,7 +580,7 @@ __device__ __forceinline__ void merge_pair(const SegCtx& c, int P, int wlo, int 
     const bool inside = u0 >= c.cs && u1 <= c.ce;
     const int cta = blockIdx.x;
     const int ca = inside ? cta : cta_of(u0, c.sp), cb = inside ? cta : cta_of(u1 - 1, c.sp);
-    const int nloc = whi - wlo + 1, nall = nloc + (cb - ca);
+    const int nloc = whi - wlo + 1, nall = nloc + (inside ? 0 : cb - ca + 1);
     float M[NH], Ls[NH], O[NH][4];
 #pragma unroll
     for (int r = 0; r < NH; ++r) {
@@ -604,11 +605,15 @@ __device__ __forceinline__ void merge_pair(const SegCtx& c, int P, int wlo, int 
             old = __shfl_sync(FULL, old, 0);
             const unsigned need = unsigned(cb - ca);   // tickets taken before the last one
             if (old < need) return;
-            if (old > need) {
-                // the ticket was not zero at the start of the call: output NaN
-                if (lane == 0) atomicAdd(&c.status[1], 1u);
+            // the last CTA folds every CTA's partial, its own too, in CTA order, so
+            // that the result does not depend on which CTA finished last
+            const bool bad = old > need;      // the ticket was not zero at the start of the call
+            if (bad && lane == 0) atomicAdd(&c.status[1], 1u);
 #pragma unroll
-                for (int r = 0; r < NH; ++r) Ls[r] = NAN;
+            for (int r = 0; r < NH; ++r) {
+                M[r] = -INFINITY;
+                Ls[r] = bad ? NAN : 0.0f;
+                O[r][0] = O[r][1] = O[r][2] = O[r][3] = 0.0f;
             }
             __syncwarp();                     // lane 0's acquire, then every lane's loads
         }
@@ -616,28 +621,34 @@ __device__ __forceinline__ void merge_pair(const SegCtx& c, int P, int wlo, int 
         if (it < nloc) {
             const int ww = wlo + it;
             const bool parked = c.hd->wfirst[ww] == P && c.hd->wlast[ww] != P;
-            src = parked ? c.park + ww * g * PST
+            src = parked ? c.park + ww * NH * PST
                          : reinterpret_cast<const float*>(c.ring + size_t(ww) * c.SPW * c.slot_bytes);
         } else {
-            int cc = ca + (it - nloc);
-            if (cc >= cta) ++cc;              // every CTA of the pair but this one
+            const int cc = ca + (it - nloc);
             src = c.part + (size_t(cc) * 2 + (u0 > cta_start(cc, c.sp) ? 1 : 0)) * part_floats<NH>();
+        }
+        // every row's loads first (all in flight together; a slot always holds NH
+        // rows, those of heads r >= g are read and ignored), then the fold
+        float2 ml[NH];
+        float4 v[NH];
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            ml[r] = ld_relaxed_v2(src + r * PST + D);
+            v[r] = ld_relaxed_v4(src + r * PST + 4 * lane);
         }
 #pragma unroll
         for (int r = 0; r < NH; ++r) {
             if (r >= g) continue;
-            const float2 ml = ld_relaxed_v2(src + r * PST + D);
-            const float4 v = ld_relaxed_v4(src + r * PST + 4 * lane);
-            const float mn = fmaxf(M[r], ml.x);
+            const float mn = fmaxf(M[r], ml[r].x);
             const float mu = mn == -INFINITY ? 0.0f : mn;
             const float al = M[r] == -INFINITY ? 0.0f : ex2(M[r] - mu);
-            const float wgt = ml.x == -INFINITY ? 0.0f : ex2(ml.x - mu);
+            const float wgt = ml[r].x == -INFINITY ? 0.0f : ex2(ml[r].x - mu);
             M[r] = mn;
-            Ls[r] = fmaf(ml.y, wgt, Ls[r] * al);
-            O[r][0] = fmaf(v.x, wgt, O[r][0] * al);
-            O[r][1] = fmaf(v.y, wgt, O[r][1] * al);
-            O[r][2] = fmaf(v.z, wgt, O[r][2] * al);
-            O[r][3] = fmaf(v.w, wgt, O[r][3] * al);
+            Ls[r] = fmaf(ml[r].y, wgt, Ls[r] * al);
+            O[r][0] = fmaf(v[r].x, wgt, O[r][0] * al);
+            O[r][1] = fmaf(v[r].y, wgt, O[r][1] * al);
+            O[r][2] = fmaf(v[r].z, wgt, O[r][2] * al);
+            O[r][3] = fmaf(v[r].w, wgt, O[r][3] * al);
         }
     }
     if (!inside && lane == 0) c.tickets[P] = 0u;   // ready for the next call
@@ -670,7 +681,7 @@ template <int NH>
 __device__ __forceinline__ int post_segment(const SegCtx& c, const State<NH>& x, int b, int h, bool last_unit, int w,
                                             int lane, int& wlo, int& whi) {
     store_partial<NH>(c, x, last_unit ? reinterpret_cast<float*>(c.ring + size_t(w) * c.SPW * c.slot_bytes)
-                                      : c.park + w * c.g * PST, lane);
+                                      : c.park + w * NH * PST, lane);
     const int P = b * c.H + h, n = c.S[b + 1] - c.S[b];
     const int u0 = c.H * c.S[b] + h * n, u1 = u0 + n;
     // warp holding unit u of this CTA's range
@@ -704,7 +715,7 @@ decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, 
     int* S = reinterpret_cast<int*>(smem + off_sched());    // [B+1] units of one pair of sequences < b
     int* LB = S + (B + 1);                                    // [B] clamped lengths  (S, LB: 8(B+1) bytes)
     uint8_t* qarea = smem + off_qarea(B);
-    float* park = reinterpret_cast<float*>(smem + off_park<KB, VB, NH>(B));   // [NW][g][PST]
+    float* park = reinterpret_cast<float*>(smem + off_park<KB, VB, NH>(B));   // [NW][NH][PST]
     uint8_t* ring;                                                          // [NW][SPW][SLOT], 1024-aligned
     {
         const uint32_t a = smem_u32(smem) + off_ring<KB, VB, NH>(B, p.g);
