@@ -99,6 +99,7 @@ struct Head {
     int cnt[kMaxWarps][2];                 // warps done with a pair they share, by owner warp and kind
     int wfirst[kMaxWarps], wlast[kMaxWarps];   // pairs of each warp's first and last unit (-1: no units)
     int abort;
+    int done;                              // warps past their units
 };
 
 // merge partials: per head a row of D outputs, the running maximum and the
@@ -300,6 +301,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 // ---------------------------------------------------------------- schedule
 struct UnitPos {
     int b, h, j, n;
+    int L, nq;      // the sequence's length and quantized units (set per pair)
 };
 // unit u -> sequence b, kv-head h, index j inside the pair, units n of the pair
 __device__ __forceinline__ UnitPos locate(const int* S, int B, int H, int u) {
@@ -310,7 +312,7 @@ __device__ __forceinline__ UnitPos locate(const int* S, int B, int H, int u) {
         else hi = mid - 1;
     }
     const int n = S[lo + 1] - S[lo], r = u - H * S[lo];
-    return {lo, r / n, r % n, n};
+    return {lo, r / n, r % n, n, 0, 0};
 }
 
 // ---------------------------------------------------------------- per-thread state
@@ -572,70 +574,41 @@ __device__ __forceinline__ float2 ld_relaxed_v2(const float* a) {
 // keeps the code short (it runs cold, once or twice per warp).
 // Lane l owns channels 4l .. 4l+3.
 template <int NH>
-__device__ __forceinline__ void merge_pair(const SegCtx& c, int P, int wlo, int whi, int lane) {
+__device__ __forceinline__ void merge_pair(const SegCtx& c, int P, int wlo, int whi, int lane, bool dry = false) {
     const int g = c.g, H = c.H;
     const int b = P / H, h = P - b * H;
     const int n = c.S[b + 1] - c.S[b];
     const int u0 = H * c.S[b] + h * n, u1 = u0 + n;
     const bool inside = u0 >= c.cs && u1 <= c.ce;
     const int cta = blockIdx.x;
-    const int ca = inside ? cta : cta_of(u0, c.sp), cb = inside ? cta : cta_of(u1 - 1, c.sp);
-    const int nloc = whi - wlo + 1, nall = nloc + (inside ? 0 : cb - ca + 1);
     float M[NH], Ls[NH], O[NH][4];
+    auto reset = [&](float l0) {
 #pragma unroll
-    for (int r = 0; r < NH; ++r) {
-        M[r] = -INFINITY;
-        Ls[r] = 0.0f;
-        O[r][0] = O[r][1] = O[r][2] = O[r][3] = 0.0f;
-    }
-#pragma unroll 1
-    for (int it = 0; it < nall; ++it) {
-        if (it == nloc) {
-            // this CTA's partial goes to its slot (0 when P is the CTA's first pair, else 1)
-            float* gdst = c.part + (size_t(cta) * 2 + (u0 > c.cs ? 1 : 0)) * part_floats<NH>();
-#pragma unroll
-            for (int r = 0; r < NH; ++r) {
-                if (r >= g) continue;
-                *reinterpret_cast<float4*>(gdst + r * PST + 4 * lane) = make_float4(O[r][0], O[r][1], O[r][2], O[r][3]);
-                if (lane == 0) *reinterpret_cast<float2*>(gdst + r * PST + D) = make_float2(M[r], Ls[r]);
-            }
-            __syncwarp();                     // every lane's stores, then lane 0's release
-            unsigned old = 0;
-            if (lane == 0) old = atom_add_acq_rel_gpu(c.tickets + P, 1u);
-            old = __shfl_sync(FULL, old, 0);
-            const unsigned need = unsigned(cb - ca);   // tickets taken before the last one
-            if (old < need) return;
-            // the last CTA folds every CTA's partial, its own too, in CTA order, so
-            // that the result does not depend on which CTA finished last
-            const bool bad = old > need;      // the ticket was not zero at the start of the call
-            if (bad && lane == 0) atomicAdd(&c.status[1], 1u);
-#pragma unroll
-            for (int r = 0; r < NH; ++r) {
-                M[r] = -INFINITY;
-                Ls[r] = bad ? NAN : 0.0f;
-                O[r][0] = O[r][1] = O[r][2] = O[r][3] = 0.0f;
-            }
-            __syncwarp();                     // lane 0's acquire, then every lane's loads
+        for (int r = 0; r < NH; ++r) {
+            M[r] = -INFINITY;
+            Ls[r] = l0;
+            O[r][0] = O[r][1] = O[r][2] = O[r][3] = 0.0f;
         }
-        const float* src;
-        if (it < nloc) {
-            const int ww = wlo + it;
-            const bool parked = c.hd->wfirst[ww] == P && c.hd->wlast[ww] != P;
-            src = parked ? c.park + ww * NH * PST
-                         : reinterpret_cast<const float*>(c.ring + size_t(ww) * c.SPW * c.slot_bytes);
-        } else {
-            const int cc = ca + (it - nloc);
-            src = c.part + (size_t(cc) * 2 + (u0 > cta_start(cc, c.sp) ? 1 : 0)) * part_floats<NH>();
+    };
+    // every row of a partial is loaded before any is folded (a slot always holds
+    // NH rows; those of heads r >= g are read and ignored): parts of this CTA
+    // from shared memory with plain loads (the counter's acquire orders them),
+    // other CTAs' partials with relaxed loads at GPU scope (past the L1)
+    auto load_local = [&](const float* src, float2 (&ml)[NH], float4 (&v)[NH]) {
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            ml[r] = *reinterpret_cast<const float2*>(src + r * PST + D);
+            v[r] = *reinterpret_cast<const float4*>(src + r * PST + 4 * lane);
         }
-        // every row's loads first (all in flight together; a slot always holds NH
-        // rows, those of heads r >= g are read and ignored), then the fold
-        float2 ml[NH];
-        float4 v[NH];
+    };
+    auto load = [&](const float* src, float2 (&ml)[NH], float4 (&v)[NH]) {
 #pragma unroll
         for (int r = 0; r < NH; ++r) {
             ml[r] = ld_relaxed_v2(src + r * PST + D);
             v[r] = ld_relaxed_v4(src + r * PST + 4 * lane);
         }
+    };
+    auto fold = [&](const float2 (&ml)[NH], const float4 (&v)[NH]) {
 #pragma unroll
         for (int r = 0; r < NH; ++r) {
             if (r >= g) continue;
@@ -650,8 +623,58 @@ __device__ __forceinline__ void merge_pair(const SegCtx& c, int P, int wlo, int 
             O[r][2] = fmaf(v[r].z, wgt, O[r][2] * al);
             O[r][3] = fmaf(v[r].w, wgt, O[r][3] * al);
         }
+    };
+    reset(0.0f);
+    // the parts of this CTA's warps
+#pragma unroll 1
+    for (int ww = wlo; ww <= whi; ++ww) {
+        const bool parked = c.hd->wfirst[ww] == P && c.hd->wlast[ww] != P;
+        float2 ml[NH];
+        float4 v[NH];
+        load_local(parked ? c.park + ww * NH * PST
+                          : reinterpret_cast<const float*>(c.ring + size_t(ww) * c.SPW * c.slot_bytes),
+                   ml, v);
+        fold(ml, v);
     }
-    if (!inside && lane == 0) c.tickets[P] = 0u;   // ready for the next call
+    if (!inside) {
+        const int ca = cta_of(u0, c.sp), cb = cta_of(u1 - 1, c.sp);
+        // this CTA's partial goes to its slot (0 when P is the CTA's first pair, else 1)
+        float* gdst = c.part + (size_t(cta) * 2 + (u0 > c.cs ? 1 : 0)) * part_floats<NH>();
+        if (!dry) {
+#pragma unroll
+            for (int r = 0; r < NH; ++r) {
+                if (r >= g) continue;
+                *reinterpret_cast<float4*>(gdst + r * PST + 4 * lane) = make_float4(O[r][0], O[r][1], O[r][2], O[r][3]);
+                if (lane == 0) *reinterpret_cast<float2*>(gdst + r * PST + D) = make_float2(M[r], Ls[r]);
+            }
+        }
+        __syncwarp();                         // every lane's stores, then lane 0's release
+        const unsigned need = unsigned(cb - ca);   // tickets taken before the last one
+        unsigned old = need;
+        if (lane == 0 && !dry) old = atom_add_acq_rel_gpu(c.tickets + P, 1u);
+        old = __shfl_sync(FULL, old, 0);
+        if (old < need) return;
+        // the last CTA folds every CTA's partial, its own too, in CTA order, so that
+        // the result does not depend on which CTA finished last; two at a time
+        const bool bad = old > need;          // the ticket was not zero at the start of the call
+        if (bad && lane == 0) atomicAdd(&c.status[1], 1u);
+        reset(bad ? NAN : 0.0f);
+        __syncwarp();                         // lane 0's acquire, then every lane's loads
+#pragma unroll 1
+        for (int cc = ca; cc <= cb; cc += 2) {
+            const bool two = cc + 1 <= cb;
+            const float* s0 = c.part + (size_t(cc) * 2 + (u0 > cta_start(cc, c.sp) ? 1 : 0)) * part_floats<NH>();
+            const float* s1 = two ? c.part + (size_t(cc + 1) * 2 + (u0 > cta_start(cc + 1, c.sp) ? 1 : 0)) * part_floats<NH>()
+                                  : s0;
+            float2 ml0[NH], ml1[NH];
+            float4 v0[NH], v1[NH];
+            load(s0, ml0, v0);
+            load(s1, ml1, v1);
+            fold(ml0, v0);
+            if (two) fold(ml1, v1);
+        }
+        if (lane == 0 && !dry) c.tickets[P] = 0u;   // ready for the next call
+    }
     // lane r < g: the reciprocal weight sum and the lse of head r
     float myL = Ls[0], myM = M[0];
 #pragma unroll
@@ -659,12 +682,12 @@ __device__ __forceinline__ void merge_pair(const SegCtx& c, int P, int wlo, int 
         if (lane == r) myL = Ls[r], myM = M[r];
     const float inv = myL > 0.0f ? __fdividef(1.0f, myL) : 0.0f;   // within 2 ulp
     const size_t row0 = size_t(b) * c.hq + size_t(h) * g;
-    if (c.lse && lane < g)
-        c.lse[row0 + lane] = myL > 0.0f ? (myM + log2f(myL)) * kLn2 : (myL == 0.0f ? -INFINITY : NAN);
+    const float lv = myL > 0.0f ? (myM + log2f(myL)) * kLn2 : (myL == 0.0f ? -INFINITY : NAN);
+    if (c.lse && lane < g && !dry) c.lse[row0 + lane] = lv;
 #pragma unroll
     for (int r = 0; r < NH; ++r) {
         const float ir = __shfl_sync(FULL, inv, r);
-        if (r < g)
+        if (r < g && !dry)
             *reinterpret_cast<float4*>(c.out + (row0 + r) * D + 4 * lane) =
                 make_float4(O[r][0] * ir, O[r][1] * ir, O[r][2] * ir, O[r][3] * ir);
     }
@@ -736,6 +759,7 @@ decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, 
             for (int i = 0; i < SPW; ++i) mbar_init(&hd.full[w][i], 1);
         mbar_fence_init();
         hd.abort = 0;
+        hd.done = 0;
     }
     __syncthreads();
     if (warp == 0) {
@@ -796,6 +820,11 @@ decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, 
         if (L > 0 && u.j < nq && u.j < p.max_pages) v = __ldg(p.page_table + size_t(u.b) * p.max_pages + u.j);
         return v;
     };
+    // length and quantized units of the unit's sequence (kept per pair)
+    auto fill = [&](UnitPos& u) {
+        u.L = LB[u.b];
+        u.nq = (u.L - min(W, u.L) + TOK - 1) / TOK;
+    };
     auto next_unit = [&](UnitPos& u) {
         if (++u.j == u.n) {
             u.j = 0;
@@ -804,6 +833,7 @@ decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, 
                 if (u.b + 1 < B) ++u.b;
             }
             u.n = S[u.b + 1] - S[u.b];
+            fill(u);
         }
     };
     int issued = 0;                     // units whose copies this warp has issued
@@ -825,7 +855,7 @@ decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, 
         if (lane == 0) hd.upg[w][slot] = pg;
         uint64_t* bar = &hd.full[w][slot];
         uint8_t* sl = wring + size_t(slot) * C::SLOT;
-        const int L = LB[u.b], wl = min(W, L), lq = L - wl, nq = (lq + TOK - 1) / TOK;
+        const int L = u.L, nq = u.nq;
         if (L > 0 && u.j < nq) {
             // a page: the four blocks in 16-byte pieces from every lane (a bulk copy
             // holds the lane that issues it for about a hundred cycles, so four of
@@ -882,7 +912,9 @@ decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, 
         // ---- the first pair's query (loaded before the copies so that its loads
         // are not queued behind them), then the first SPW units: page lookups in
         // parallel, then the copies
-        UnitPos pos = locate(S, B, H, wbeg), ip = pos;
+        UnitPos pos = locate(S, B, H, wbeg);
+        fill(pos);
+        UnitPos ip = pos;
         float xq[NH][4];
         load_query<NH>(p, q, q_bf16, pos.b, pos.h, lane, xq);
         for (int i = 0; i < SPW && i < nunits; ++i) {
@@ -894,6 +926,8 @@ decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, 
         float cq[HS], cz[HS][NKG];
         bool q_ready = false, wq_ready = false;
         int mp0 = -1, mlo0 = 0, mhi0 = 0, mp1 = -1, mlo1 = 0, mhi1 = 0;   // merges this warp owes
+        int slot = 0;
+        uint32_t phase = 0;             // parity of the slot's barrier for this unit
         for (int k = 0; k < nunits; ++k) {
             // the pair's query (one place for the first pair and every later one)
             if (!q_ready) {
@@ -901,8 +935,7 @@ decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, 
                 prep_query<KB, NH>(p, xq, qa, sl2, lane, qb, cq, cz);
                 q_ready = true;
             }
-            const int slot = k % SPW;
-            const int L = LB[pos.b], wl = min(W, L), lq = L - wl, nq = (lq + TOK - 1) / TOK;
+            const int L = pos.L, wl = min(W, L), lq = L - wl, nq = pos.nq;
             const uint32_t sl = wring_s + uint32_t(slot) * C::SLOT;
             const bool kind_q = L > 0 && pos.j < nq;
             const bool kind_w = L > 0 && pos.j >= nq;
@@ -911,7 +944,7 @@ decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, 
                 prep_window_query<NH>(p, q, q_bf16, pos.b, pos.h, qa, lane);
                 wq_ready = true;
             }
-            const bool ok = wait_bar(&hd.full[w][slot], (k / SPW) & 1);
+            const bool ok = wait_bar(&hd.full[w][slot], phase);
             if (!ok) st.bad = true;
             const int pres0 = kind_q && hd.upg[w][slot] >= 0;
                 if (ok && kind_q) {
@@ -1164,7 +1197,7 @@ decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, 
                 }
                 __syncwarp();
                 // ---- the slot is free: copies of unit k + SPW into it
-                if (k + SPW < nunits && !aborted()) {
+                if (k + SPW < nunits && ok) {
                     issue(slot, ip, k + SPW);
                     next_unit(ip);
                 }
@@ -1190,6 +1223,10 @@ decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, 
                     st.reset();
                 }
                 // ---- next unit
+                if (++slot == SPW) {
+                    slot = 0;
+                    phase ^= 1u;
+                }
                 if (!pair_end) {
                     ++pos.j;
                 } else if (!last_unit) {
@@ -1199,13 +1236,27 @@ decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, 
                         ++pos.b;
                     }
                     pos.n = S[pos.b + 1] - S[pos.b];
+                    fill(pos);
                     seg_j0 = 0;
                     q_ready = wq_ready = false;
                 }
             }
 
         // ---- the merges this warp owes (the partials stay where they were stored:
-        // parking areas and the rings of warps that are done with their units)
+        // parking areas and the rings of warps that are done with their units).
+        // A warp that owes none and is among the first half of the CTA's warps to
+        // be done runs the merge code once without effects (no stores, no
+        // tickets; loads from the CTA's first pair's parts), so that the merging
+        // warps of this SM find that code in the instruction cache.
+        int rank_done = 0;
+        if (lane == 0) rank_done = atomicAdd(&hd.done, 1);
+        rank_done = __shfl_sync(FULL, rank_done, 0);
+        if (mp0 < 0 && rank_done < NW / 2) {
+            const SegCtx sc{&hd, S, park, ring, out, lse, part, tickets, status, p.hq, g, H, SPW, C::SLOT,
+                            cs, ce, base_n, rem, sp};
+            const UnitPos f = locate(S, B, H, cs);
+            merge_pair<NH>(sc, f.b * H + f.h, 0, 0, lane, true);
+        }
         if (mp0 >= 0) {
             const SegCtx sc{&hd, S, park, ring, out, lse, part, tickets, status, p.hq, g, H, SPW, C::SLOT,
                             cs, ce, base_n, rem, sp};
