@@ -244,6 +244,28 @@ int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache,
                          float sm_scale, float* out, float* lse,
                          void* workspace, size_t workspace_bytes, kvq_stream_t stream);
 
+/* One decode step: kvq_quantize_append(k_new, v_new, in_dtype, cu_new,
+ * lens_old, max_new) followed by kvq_decode_attention(q, q_dtype, lens,
+ * max_len, sm_scale, out, lse, workspace) on the same stream, with the same
+ * arguments, results and error codes as those two calls (lens_old is the
+ * append's `lens`: tokens before the step; lens the decode's: tokens after
+ * it, typically lens_old + 1; both stay unmodified).  Not in the pages: it
+ * exists so that the decode's start-up overlaps the append.  When the append
+ * is one launch (at most 8 new tokens per sequence, and not more than the
+ * window) and the persistent tensor-core decode applies, the decode is
+ * launched as the append's programmatic dependent: it reads lens, the page
+ * table and q while the append runs, and the cache only after the append's
+ * results are visible; otherwise the two calls run one after the other.
+ * Every argument of both calls is checked before anything is enqueued.
+ * q, lens, lens_old, cu_new and the page table must not overlap what the
+ * append writes (the cache's codes, metadata and window). */
+int kvq_append_decode(const kvq_layout* layout, const kvq_cache* cache,
+                      const void* k_new, const void* v_new, int in_dtype,
+                      const int32_t* cu_new, const int32_t* lens_old, int max_new,
+                      const void* q, int q_dtype, const int32_t* lens, int max_len,
+                      float sm_scale, float* out, float* lse,
+                      void* workspace, size_t workspace_bytes, kvq_stream_t stream);
+
 /* Bytes of the library's static decode scratch (per device). */
 #define KVQ_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
 

@@ -71,6 +71,7 @@ def lib() -> C.CDLL:
         L.kvq_quantize_append.argtypes = [LP, CP, P, P, I, P, P, I, P]
         L.kvq_decode_attention.argtypes = [LP, CP, P, I, P, I, C.c_float, P, P, P, S, P]
         L.kvq_decode_attention_static_scratch.argtypes = [LP, CP, P, I, P, I, C.c_float, P, P, P]
+        L.kvq_append_decode.argtypes = [LP, CP, P, P, I, P, P, I, P, I, P, I, C.c_float, P, P, P, S, P]
         L.kvq_dequantize.argtypes = [LP, CP, P, I, P, P, P]
         L.kvq_prefill_attention.argtypes = [LP, CP, P, I, P, P, I, C.c_float, P, P, P]
         L.kvq_rotate_keys.argtypes = [LP, P, I, I, P, P]
@@ -81,7 +82,8 @@ def lib() -> C.CDLL:
         L.kvq_decode_status.argtypes = [C.POINTER(C.c_uint), C.POINTER(C.c_uint), I]
         L.kvq_decode_status.restype = I
         for n in ("kvq_page_bytes", "kvq_window_bytes", "kvq_quantize_append",
-                  "kvq_decode_attention", "kvq_decode_attention_static_scratch", "kvq_dequantize",
+                  "kvq_decode_attention", "kvq_decode_attention_static_scratch", "kvq_append_decode",
+                  "kvq_dequantize",
                   "kvq_rotate_keys"):
             getattr(L, n).restype = I
         _lib_handle = L
@@ -260,6 +262,30 @@ def kvq_decode_attention(layout: Layout, cache: PagedCache, q: torch.Tensor, len
            at_least=True)
     _call("kvq_decode_attention", C.byref(layout.c()), C.byref(cache.c()), _ptr(q), _dtype_code(q),
           _ptr(lens), int(max_len), C.c_float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+          C.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
+
+
+def kvq_append_decode(layout: Layout, cache: PagedCache, k_new: torch.Tensor, v_new: torch.Tensor,
+                      cu_new: torch.Tensor, lens_old: torch.Tensor, max_new: int, q: torch.Tensor,
+                      lens: torch.Tensor, max_len: int, sm_scale: float, out: torch.Tensor,
+                      lse: Optional[torch.Tensor], workspace: torch.Tensor, stream=None) -> None:
+    """kvq.h kvq_append_decode: kvq_quantize_append then kvq_decode_attention,
+    the decode's start-up overlapping the append."""
+    if k_new.dtype != v_new.dtype:
+        raise ValueError("k_new and v_new must share a dtype")
+    B, row = cache.batch, layout.num_kv_heads * layout.head_dim
+    _check(k_new, "k_new", _FLOAT_IN)
+    if k_new.numel() % row:
+        raise ValueError(f"k_new must hold whole rows of {row} elements ([total_new][Hkv][d])")
+    _check(v_new, "v_new", _FLOAT_IN, k_new.numel())
+    _check(cu_new, "cu_new", _I32, B + 1)
+    _check(lens_old, "lens_old", _I32, B)
+    _check_decode_args(layout, cache, q, lens, out, lse)
+    _check(workspace, "workspace", (torch.uint8,), kvq_decode_workspace_bytes(layout, cache.batch, max_len),
+           at_least=True)
+    _call("kvq_append_decode", C.byref(layout.c()), C.byref(cache.c()), _ptr(k_new), _ptr(v_new),
+          _dtype_code(k_new), _ptr(cu_new), _ptr(lens_old), int(max_new), _ptr(q), _dtype_code(q), _ptr(lens),
+          int(max_len), C.c_float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace),
           C.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
 
 

@@ -226,6 +226,44 @@ int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache, const
                                           workspace, pl, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int kvq_append_decode(const kvq_layout* layout, const kvq_cache* cache, const void* k_new, const void* v_new,
+                      int in_dtype, const int32_t* cu_new, const int32_t* lens_old, int max_new, const void* q,
+                      int q_dtype, const int32_t* lens, int max_len, float sm_scale, float* out, float* lse,
+                      void* workspace, size_t workspace_bytes, kvq_stream_t stream) {
+    // the checks of both calls, before anything is enqueued
+    int rc = check_layout(layout);
+    if (rc) return rc;
+    if ((rc = check_cache(layout, cache))) return rc;
+    if (in_dtype != KVQ_F32 && in_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+    if (max_new < 0 || !cu_new || !lens_old) return KVQ_ERR_INVALID_ARG;
+    if (max_new > 0 && (!k_new || !v_new)) return KVQ_ERR_INVALID_ARG;
+    if (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+    if (!q || !lens || !out || max_len < 0 || !isfinite(sm_scale)) return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return KVQ_ERR_INVALID_ARG;
+    if (cache->batch == 0) return KVQ_OK;
+    if (cache->batch > 65535 || layout->num_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
+    Params p = make_params(layout, cache);
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (layout->k_per_channel) {
+        if ((rc = kvq_quantize_append(layout, cache, k_new, v_new, in_dtype, cu_new, lens_old, max_new, stream)))
+            return rc;
+        return kvq_decode_attention(layout, cache, q, q_dtype, lens, max_len, sm_scale, out, lse, workspace,
+                                    workspace_bytes, stream);
+    }
+    kvq::DecodePlan pl = kvq::plan_decode(p, cache->batch, max_len, device_sm_count());
+    const size_t need = kvq::decode_workspace_bytes(p, cache->batch, pl);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return KVQ_ERR_WORKSPACE;
+    if (max_new > 0) {
+        if ((rc = cuda_status(kvq::launch_quantize_append(p, k_new, v_new, in_dtype == KVQ_BF16, cu_new, lens_old,
+                                                          max_new, s))))
+            return rc;
+        pl.after_append = pl.mma && kvq::append_is_one_launch(p, max_new) ? 1 : 0;
+    }
+    return cuda_status(kvq::launch_decode(p, q, q_dtype == KVQ_BF16, lens, max_len, sm_scale, out, lse, workspace, pl,
+                                          s));
+}
+
 int kvq_prefill_attention(const kvq_layout* layout, const kvq_cache* cache, const void* q, int q_dtype,
                           const int32_t* cu_q, const int32_t* lens, int max_q, float sm_scale, float* out,
                           float* lse, kvq_stream_t stream) {

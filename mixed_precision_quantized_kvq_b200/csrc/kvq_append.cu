@@ -199,6 +199,9 @@ __global__ void __launch_bounds__(128) append_small_kernel(Params p, const void*
                                                            const int32_t* __restrict__ cu_new,
                                                            const int32_t* __restrict__ lens) {
     constexpr int CPL = D / 32;
+    // a decode launched next as this launch's programmatic dependent may start
+    // now: it reads nothing this kernel writes before it waits for its results
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int h = blockIdx.x, b = blockIdx.y;
     const int L = lens[b];
     const int c0 = cu_new[b], n = cu_new[b + 1] - c0;
@@ -342,11 +345,15 @@ __global__ void __launch_bounds__(128) dequantize_kernel(Params p, const int32_t
 
 }  // namespace
 
+bool append_is_one_launch(const Params& p, int max_new) {
+    return max_new >= 1 && p.batch > 0 && max_new <= kSmallAppend && (p.W == 0 || max_new <= p.W);
+}
+
 cudaError_t launch_quantize_append(const Params& p, const void* k_new, const void* v_new, int in_bf16,
                                    const int32_t* cu_new, const int32_t* lens, int max_new,
                                    cudaStream_t s) {
     if (max_new <= 0 || p.batch <= 0) return cudaSuccess;
-    if (max_new <= kSmallAppend && (p.W == 0 || max_new <= p.W)) {
+    if (append_is_one_launch(p, max_new)) {
         const dim3 sgrid(p.hkv, p.batch);
         if (p.d == 128) append_small_kernel<128><<<sgrid, 128, 0, s>>>(p, k_new, v_new, in_bf16, cu_new, lens);
         else append_small_kernel<64><<<sgrid, 128, 0, s>>>(p, k_new, v_new, in_bf16, cu_new, lens);

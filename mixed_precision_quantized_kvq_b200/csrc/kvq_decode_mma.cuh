@@ -727,7 +727,7 @@ template <int KB, int VB, int NH>
 __global__ void __launch_bounds__(Cfg<KB, VB, NH>::NW * 32, 1)
 decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, const int q_bf16, const int32_t* __restrict__ lens,
                   const int max_len, const float sl2, float* __restrict__ out, float* __restrict__ lse,
-                  float* __restrict__ part, uint32_t* __restrict__ tickets, const int SPW,
+                  float* __restrict__ part, uint32_t* __restrict__ tickets, const int SPW, const int after_append,
                   unsigned int* __restrict__ status, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v) {
     using C = Cfg<KB, VB, NH>;
@@ -917,14 +917,23 @@ decode_mma_kernel(const __grid_constant__ Params p, const void* __restrict__ q, 
         UnitPos ip = pos;
         float xq[NH][4];
         load_query<NH>(p, q, q_bf16, pos.b, pos.h, lane, xq);
-        for (int i = 0; i < SPW && i < nunits; ++i) {
-            issue(i, ip, i);
-            next_unit(ip);
-        }
         int seg_j0 = pos.j;
         uint32_t qb[NKG][NT][2];
         float cq[HS], cz[HS][NKG];
         bool q_ready = false, wq_ready = false;
+        if (after_append) {
+            // launched as the programmatic dependent of an append on the same stream:
+            // everything so far read only what the append does not write (lengths,
+            // page table, query), so the query is prepared too before the wait for
+            // the append's results; the cache is read only after it
+            prep_query<KB, NH>(p, xq, qa, sl2, lane, qb, cq, cz);
+            q_ready = true;
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+        }
+        for (int i = 0; i < SPW && i < nunits; ++i) {
+            issue(i, ip, i);
+            next_unit(ip);
+        }
         int mp0 = -1, mlo0 = 0, mhi0 = 0, mp1 = -1, mlo1 = 0, mhi1 = 0;   // merges this warp owes
         int slot = 0;
         uint32_t phase = 0;             // parity of the slot's barrier for this unit

@@ -4,9 +4,9 @@
 namespace kvq {
 
 cudaError_t launch_decode_mma_k1(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len,
-                                 float sl2, float* out, float* lse, float* part, uint32_t* tickets, int ctas,
+                                 float sl2, float* out, float* lse, float* part, uint32_t* tickets, int ctas, int after_append,
                                  unsigned* status, cudaStream_t s) {
-    return mma::launch_kb<1>(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, ctas, status, s);
+    return mma::launch_kb<1>(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, ctas, after_append, status, s);
 }
 
 }  // namespace kvq

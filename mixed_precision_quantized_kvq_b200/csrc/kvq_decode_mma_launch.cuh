@@ -54,7 +54,7 @@ int ring_slots(int batch, int g) {
 
 template <int KB, int VB, int NH>
 cudaError_t launch_one(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len, float sl2,
-                       float* out, float* lse, float* part, uint32_t* tickets, int ctas, unsigned* status, cudaStream_t s) {
+                       float* out, float* lse, float* part, uint32_t* tickets, int ctas, int after_append, unsigned* status, cudaStream_t s) {
     auto kern = decode_mma_kernel<KB, VB, NH>;
     static bool configured[64];
     int dev = 0;
@@ -72,33 +72,38 @@ cudaError_t launch_one(const Params& p, const void* q, int q_bf16, const int32_t
     const cudaError_t em = window_maps(p, &mk, &mv);
     if (em != cudaSuccess) return em;
     // no CTA waits for another (pairs split between CTAs are merged by the CTA
-    // that finishes last), so a plain launch of one CTA per SM
+    // that finishes last), so a plain launch of one CTA per SM; right after an
+    // append, as its programmatic dependent (the kernel waits for the append's
+    // results before it reads the cache)
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(ctas);
     cfg.blockDim = dim3(C::NW * 32);
     cfg.dynamicSmemBytes = bytes;
     cfg.stream = s;
-    cfg.attrs = nullptr;
-    cfg.numAttrs = 0;
-    return cudaLaunchKernelEx(&cfg, kern, p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, spw, status, mk,
-                              mv);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = after_append ? attr : nullptr;
+    cfg.numAttrs = after_append ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, spw,
+                              after_append, status, mk, mv);
 }
 
 template <int KB, int VB>
 cudaError_t launch_nh(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len, float sl2,
-                      float* out, float* lse, float* part, uint32_t* tickets, int ctas, unsigned* status, cudaStream_t s) {
-    if (p.g <= 4) return launch_one<KB, VB, 4>(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, ctas, status, s);
-    return launch_one<KB, VB, 8>(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, ctas, status, s);
+                      float* out, float* lse, float* part, uint32_t* tickets, int ctas, int after_append, unsigned* status, cudaStream_t s) {
+    if (p.g <= 4) return launch_one<KB, VB, 4>(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, ctas, after_append, status, s);
+    return launch_one<KB, VB, 8>(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, ctas, after_append, status, s);
 }
 
 template <int KB>
 cudaError_t launch_kb(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len, float sl2,
-                      float* out, float* lse, float* part, uint32_t* tickets, int ctas, unsigned* status, cudaStream_t s) {
+                      float* out, float* lse, float* part, uint32_t* tickets, int ctas, int after_append, unsigned* status, cudaStream_t s) {
     switch (p.vb) {
-        case 1: return launch_nh<KB, 1>(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, ctas, status, s);
-        case 2: return launch_nh<KB, 2>(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, ctas, status, s);
-        case 4: return launch_nh<KB, 4>(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, ctas, status, s);
-        case 8: return launch_nh<KB, 8>(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, ctas, status, s);
+        case 1: return launch_nh<KB, 1>(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, ctas, after_append, status, s);
+        case 2: return launch_nh<KB, 2>(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, ctas, after_append, status, s);
+        case 4: return launch_nh<KB, 4>(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, ctas, after_append, status, s);
+        case 8: return launch_nh<KB, 8>(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, ctas, after_append, status, s);
         default: return cudaErrorNotSupported;
     }
 }

@@ -470,10 +470,10 @@ cudaError_t launch_decode(const Params& p, const void* q, int q_bf16, const int3
         float* part = reinterpret_cast<float*>(ws);
         uint32_t* tickets = reinterpret_cast<uint32_t*>(reinterpret_cast<char*>(ws) + off_tickets);
         switch (p.kb) {
-            case 1: return launch_decode_mma_k1(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, pl.ctas, status, s);
-            case 2: return launch_decode_mma_k2(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, pl.ctas, status, s);
-            case 4: return launch_decode_mma_k4(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, pl.ctas, status, s);
-            default: return launch_decode_mma_k8(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, pl.ctas, status, s);
+            case 1: return launch_decode_mma_k1(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, pl.ctas, pl.after_append, status, s);
+            case 2: return launch_decode_mma_k2(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, pl.ctas, pl.after_append, status, s);
+            case 4: return launch_decode_mma_k4(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, pl.ctas, pl.after_append, status, s);
+            default: return launch_decode_mma_k8(p, q, q_bf16, lens, max_len, sl2, out, lse, part, tickets, pl.ctas, pl.after_append, status, s);
         }
     }
     cudaError_t e = pl.tc ? launch_decode_tc(p, q, q_bf16, lens, max_len, sl2, ws_o, ws_ml, pl, status, s)

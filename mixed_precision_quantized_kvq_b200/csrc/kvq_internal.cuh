@@ -121,6 +121,8 @@ __device__ __forceinline__ void rotate_warp(float (&x)[D / 32], const int8_t* si
 struct DecodePlan {
     int mma;            // 1: persistent register-fragment tensor-core kernel (no combine launch)
     int ctas;           // its grid: one CTA per SM at most
+    int after_append;   // 1: launched right after a one-launch append on the same stream, as its
+                        //    programmatic dependent (start-up overlaps the append)
     int tc;             // 1: two-phase tcgen05 kernel, 0: CUDA-core kernel (when mma == 0)
     int splits_q;       // splits over quantized pages
     int pages_per_split;
@@ -132,13 +134,13 @@ struct DecodePlan {
 };
 // persistent register-fragment tensor-core decode (kvq_decode_mma.cuh), one key bit width per file
 cudaError_t launch_decode_mma_k1(const Params&, const void*, int, const int32_t*, int, float, float*, float*, float*,
-                                 uint32_t*, int, unsigned*, cudaStream_t);
+                                 uint32_t*, int, int, unsigned*, cudaStream_t);
 cudaError_t launch_decode_mma_k2(const Params&, const void*, int, const int32_t*, int, float, float*, float*, float*,
-                                 uint32_t*, int, unsigned*, cudaStream_t);
+                                 uint32_t*, int, int, unsigned*, cudaStream_t);
 cudaError_t launch_decode_mma_k4(const Params&, const void*, int, const int32_t*, int, float, float*, float*, float*,
-                                 uint32_t*, int, unsigned*, cudaStream_t);
+                                 uint32_t*, int, int, unsigned*, cudaStream_t);
 cudaError_t launch_decode_mma_k8(const Params&, const void*, int, const int32_t*, int, float, float*, float*, float*,
-                                 uint32_t*, int, unsigned*, cudaStream_t);
+                                 uint32_t*, int, int, unsigned*, cudaStream_t);
 // decode path selection: 0 = automatic, 1 = CUDA cores, 2 = tensor cores
 extern int g_decode_path;
 DecodePlan plan_decode(const Params& p, int batch, int max_len, int sm_count);
@@ -153,6 +155,9 @@ cudaError_t launch_decode_tc(const Params& p, const void* q, int q_bf16, const i
                              cudaStream_t s);
 size_t decode_workspace_bytes(const Params& p, int batch, const DecodePlan& plan);
 
+// the append of max_new tokens per sequence is one launch of the small-append
+// kernel (which lets a programmatic dependent start early)
+bool append_is_one_launch(const Params& p, int max_new);
 cudaError_t launch_quantize_append(const Params& p, const void* k_new, const void* v_new,
                                    int in_bf16, const int32_t* cu_new, const int32_t* lens,
                                    int max_new, cudaStream_t s);

@@ -34,6 +34,23 @@ def test_host_tensors_are_rejected():
         kvq.kvq_dequantize(lay, c, torch.zeros(B, dtype=torch.int32), 4, torch.zeros(1), torch.zeros(1))
 
 
+def test_append_decode_checks_both_calls_arguments():
+    """kvq_append_decode checks the append's and the decode's buffers."""
+    lay, c = _cache()
+    B = c.batch
+    kv = torch.zeros((B, 8, 128))
+    args = dict(cu_new=torch.zeros(B + 1, dtype=torch.int32), lens_old=torch.zeros(B, dtype=torch.int32),
+                max_new=1, q=torch.zeros((B, 32, 128), dtype=torch.bfloat16),
+                lens=torch.ones(B, dtype=torch.int32), max_len=1, sm_scale=0.1, out=torch.zeros((B, 32, 128)),
+                lse=None, workspace=torch.zeros(256, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        kvq.kvq_append_decode(lay, c, kv, kv, **args)
+    with pytest.raises(ValueError, match="share a dtype"):
+        kvq.kvq_append_decode(lay, c, kv, kv.to(torch.bfloat16), **args)
+    with pytest.raises(ValueError):
+        kvq.kvq_append_decode(lay, c, kv, kv, **dict(args, lens_old=torch.zeros(B + 1, dtype=torch.int32)))
+
+
 def test_mismatched_key_value_dtypes_are_rejected():
     lay, c = _cache()
     with pytest.raises(ValueError, match="share a dtype"):
