@@ -48,6 +48,7 @@ WORKLOADS = {"llama8b": wl.LLAMA8B, "ragged": wl.RAGGED,
                                                      k_group=64, v_group=64, k_per_channel=True)}
 # the long-context bit-allocation sweep: one workload per (key bits, value bits)
 WORKLOADS.update({f"sweep_k{v.k_bits}v{v.v_bits}": v for v in wl.sweep_variants()})
+FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 # chunked-prefill attention: (cache shape, queries per sequence in the chunk)
 PREFILL_WORKLOADS = {"prefill_llama8b": (wl.LLAMA8B, 512)}
@@ -88,6 +89,27 @@ def measured_hbm_peak():
         except (OSError, ValueError):
             pass
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_bf16_peak():
+    """Dense bf16 tensor peak (TFLOP/s) for a kernel timed alone: the measured
+    burst figure of MEASURED_PEAKS.json, else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            v = json.load(f).get("bf16_tflops")
+        if v:
+            return float(v), "measured"
+    except (OSError, ValueError):
+        pass
+    return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def prefill_on_tensor_cores(w) -> bool:
+    """The layouts the library's tensor-core prefill kernel takes (head_dim 128,
+    key groups of 32 channels of a token, unrotated keys, value groups dividing
+    128); the others run on CUDA cores."""
+    return (w.head_dim == 128 and not w.k_per_channel and not w.rotate_keys and w.k_group == 32
+            and 128 % w.v_group == 0)
 
 
 def dist_env():
@@ -723,8 +745,21 @@ def run_prefill(args):
     props = torch.cuda.get_device_properties(dev)
     clocks = sampler.summary(wall0, wall1)
     sm_max = float((clocks or {}).get("sm_max_mhz") or 1965.0)
-    peak = props.multi_processor_count * 128 * 2 * sm_max * 1e6 / 1e12   # fp32 FMA lanes x 2 flops x clock
     achieved = flops / (us * 1e-6) / 1e12
+    if prefill_on_tensor_cores(w):
+        # bf16 mma.sync with each operand split into (hi, lo): three bf16 products per
+        # algorithmic product; reported against the dense bf16 tensor peak
+        peak, kind = measured_bf16_peak()
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": None, "kernel": "kvq_prefill_attention (bf16 tensor cores, operands as bf16 hi/lo "
+                                           "pairs: 3 tensor products per algorithmic product)",
+                "peak_source": f"{kind} dense bf16 TFLOP/s" + (" (MEASURED_PEAKS.json)" if kind == "measured" else ""),
+                "tensor_flops_executed_per_step": 3 * flops}
+    else:
+        peak = props.multi_processor_count * 128 * 2 * sm_max * 1e6 / 1e12   # fp32 FMA lanes x 2 flops x clock
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": None, "kernel": "kvq_prefill_attention (CUDA cores)",
+                "peak_source": f"{props.multi_processor_count} SMs x 128 fp32 lanes x 2 flops x {sm_max:.0f} MHz"}
     line = {
         "metric": PREFILL_METRIC, "value": us_max, "unit": "us/step", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": us_max / 1e3, "higher_is_better": False, "scaling": "weak",
@@ -733,9 +768,7 @@ def run_prefill(args):
                                f"{w.num_q_heads}/{w.num_kv_heads} heads, d{w.head_dim}, K{w.k_bits}V{w.v_bits}, "
                                f"window {w.window}", "l2": "flushed (256 MB write) before every call"},
         "tflops": achieved, "flops_per_step": flops,
-        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None, "kernel": "kvq_prefill_attention (CUDA cores)",
-                     "peak_source": f"{props.multi_processor_count} SMs x 128 fp32 lanes x 2 flops x {sm_max:.0f} MHz"},
+        "roofline": roof,
         "e2e": {"value": e2e_us, "unit": "us/step", "h2d_bytes_per_step": q.numel() * q.element_size(),
                 "d2h_bytes_per_step": out.numel() * out.element_size(),
                 "api": "python binding -> C ABI, eager calls, pinned host buffers"},

@@ -105,6 +105,7 @@ cudaError_t launch_prefill_attention(const Params& p, int k_per_channel, int one
     v.scale_log2 = sm_scale * 1.4426950408889634f;
     v.out = out;
     v.lse = lse;
+    if (prefill_mma_supported(v)) return launch_prefill_mma(v, s);
     return p.d == 128 ? launch_d<128>(v, s) : launch_d<64>(v, s);
 }
 

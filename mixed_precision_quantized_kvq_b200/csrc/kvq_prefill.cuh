@@ -14,4 +14,12 @@ cudaError_t launch_prefill_attention(const Params& p, int k_per_channel, int one
                                      int q_bf16, const int32_t* cu_q, const int32_t* lens, int len_cap,
                                      int max_q, float sm_scale, float* out, float* lse, cudaStream_t s);
 
+namespace prefill {
+struct View;
+}
+// tensor-core chunked prefill (kvq_prefill_mma.cu): head_dim 128, key groups
+// of 32 channels of a token, unrotated keys, value groups dividing 128
+bool prefill_mma_supported(const prefill::View& v);
+cudaError_t launch_prefill_mma(const prefill::View& v, cudaStream_t s);
+
 }  // namespace kvq
