@@ -251,13 +251,15 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
         if (skip) continue;
 
         // ---- scores of the warp's 16 rows x 64 positions
+        // (k-step outer: eight independent accumulators between dependent MMAs)
         float s[8][4];
         const int mi = lane >> 3, rr = lane & 7;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0f;
+        for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0f;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
                 uint32_t f[4];      // Kh k0-7, Kh k8-15, Kl k0-7, Kl k8-15 of positions 8j .. 8j+7
                 ldsm_x4(f, (mi < 2 ? sKh : sKl) + swz(8 * j + rr, 2 * kk + (mi & 1), 16));
                 mma_bf16(s[j], qh[kk], f[0], f[1]);
