@@ -425,12 +425,19 @@ def run_ours(args):
     step_bytes = algorithmic_bytes(w, lens1)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     n_copies = max(2, math.ceil(2 * l2 / max(1, step_bytes)) + 1) if args.copies <= 0 else args.copies
+    def clone_cache(src):
+        return kvq.PagedCache(*[t.clone() if isinstance(t, torch.Tensor) else t
+                                for t in (src.k_codes, src.v_codes, src.k_meta, src.v_meta, src.k_win, src.v_win)],
+                              src.page_table, npages)
+
+    # The timed steps repeat the append at the same lengths on every copy, which
+    # moves the same bytes as a real step; with a window it is not idempotent (the
+    # slot that position L-W leaves is the slot token L takes), so the output check
+    # below runs one step on an untouched copy of the prefilled cache.
+    pristine = clone_cache(base) if not args.no_cpu_baseline else None
     caches = [base]
     for _ in range(n_copies - 1):
-        caches.append(kvq.PagedCache(*[t.clone() if isinstance(t, torch.Tensor) and t is not base.page_table
-                                       else t for t in (base.k_codes, base.v_codes, base.k_meta,
-                                                        base.v_meta, base.k_win, base.v_win)],
-                                     base.page_table, npages))
+        caches.append(clone_cache(base))
     qs, knew, vnew = [], [], []
     for i in range(n_copies):
         qr, _ = wl.query(w, i)
@@ -604,9 +611,10 @@ def run_ours(args):
         "clocks": clocks,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        # the oracle's first step has the inputs of cache copy 0: compare outputs
+        # the oracle's first step has the inputs of step 0 on the prefilled cache: compare outputs
         with torch.cuda.stream(stream):
-            step(0)
+            kvq.kvq_append_decode(lay, pristine, knew[0], vnew[0], cu1, glens0, 1, qs[0], glens1, max_len, scale, out,
+                                  lse, wsp)
         stream.synchronize()
         got = out.cpu().numpy()
         us_cpu, cores, sample, ref = oracle_step_timer(w, args.cpu_budget)
