@@ -184,6 +184,18 @@ int kvq_decode_status(unsigned int* wait_timeouts, unsigned int* bad_tickets, in
     return cuda_status(kvq::decode_status(wait_timeouts, bad_tickets, clear != 0));
 }
 
+// decode for key groups along positions: the per-channel decode kernel, or the
+// chunked-prefill kernel with one query per sequence for the shapes it does not take
+static int decode_per_channel(const Params& p, const void* q, int q_dtype, const int32_t* lens, int max_len,
+                              float sm_scale, float* out, float* lse, kvq_stream_t stream) {
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (kvq::decode_pc_supported(p, max_len))
+        return cuda_status(kvq::launch_decode_per_channel(p, q, q_dtype == KVQ_BF16, lens, max_len, sm_scale, out, lse,
+                                                          s));
+    return cuda_status(kvq::launch_prefill_attention(p, 1, 1, q, q_dtype == KVQ_BF16, nullptr, lens, max_len, 1,
+                                                     sm_scale, out, lse, s));
+}
+
 int kvq_quantize_append(const kvq_layout* layout, const kvq_cache* cache, const void* k_new,
                         const void* v_new, int in_dtype, const int32_t* cu_new, const int32_t* lens,
                         int max_new, kvq_stream_t stream) {
@@ -214,10 +226,8 @@ int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache, const
     if (cache->batch == 0) return KVQ_OK;
     if (cache->batch > 65535 || layout->num_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
     Params p = make_params(layout, cache);
-    if (layout->k_per_channel)   // one query per sequence through the chunked-prefill kernel
-        return cuda_status(kvq::launch_prefill_attention(p, 1, 1, q, q_dtype == KVQ_BF16, nullptr, lens, max_len,
-                                                         1, sm_scale, out, lse,
-                                                         reinterpret_cast<cudaStream_t>(stream)));
+    if (layout->k_per_channel)   // needs no workspace
+        return decode_per_channel(p, q, q_dtype, lens, max_len, sm_scale, out, lse, stream);
     kvq::DecodePlan pl = kvq::plan_decode(p, cache->batch, max_len, device_sm_count());
     const size_t need = kvq::decode_workspace_bytes(p, cache->batch, pl);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -353,9 +363,7 @@ extern "C" int kvq_decode_attention_static_scratch(const kvq_layout* layout, con
     if (cache->batch > 65535 || layout->num_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
     Params p = make_params(layout, cache);
     if (layout->k_per_channel)   // needs no scratch
-        return cuda_status(kvq::launch_prefill_attention(p, 1, 1, q, q_dtype == KVQ_BF16, nullptr, lens, max_len,
-                                                         1, sm_scale, out, lse,
-                                                         reinterpret_cast<cudaStream_t>(stream)));
+        return decode_per_channel(p, q, q_dtype, lens, max_len, sm_scale, out, lse, stream);
     kvq::DecodePlan pl = kvq::plan_decode(p, cache->batch, max_len, device_sm_count());
     if (kvq::decode_workspace_bytes(p, cache->batch, pl) > KVQ_STATIC_SCRATCH_BYTES) return KVQ_ERR_WORKSPACE;
     void* scratch = nullptr;

@@ -155,6 +155,11 @@ cudaError_t launch_decode_tc(const Params& p, const void* q, int q_bf16, const i
                              cudaStream_t s);
 size_t decode_workspace_bytes(const Params& p, int batch, const DecodePlan& plan);
 
+// decode for key groups along positions (kvq_decode_pc.cu): head_dim 128, up
+// to 8 query heads per kv-head, key groups of 16/32/64 positions, unrotated
+bool decode_pc_supported(const Params& p, int max_len);
+cudaError_t launch_decode_per_channel(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len,
+                                      float sm_scale, float* out, float* lse, cudaStream_t s);
 // the append of max_new tokens per sequence is one launch of the small-append
 // kernel (which lets a programmatic dependent start early)
 bool append_is_one_launch(const Params& p, int max_new);
