@@ -55,6 +55,9 @@ CASES = {
     "k2v2_g16_w8": dict(k_bits=2, k_group=16, window=8),
     "k1v1_g16_w8_d64": dict(head_dim=64, k_bits=1, v_bits=1, k_group=16, v_group=64, window=8),
     "k8v4_g32_w128_f32": dict(k_bits=8, v_bits=4, k_group=32, window=128, in_dtype=wl.DT_F32),
+    # five and eight query heads per kv-head (the decode kernel's 8-head build), smaller value groups
+    "k4v2_g64_w64_gqa5_vg64": dict(num_q_heads=20, v_group=64, window=64),
+    "k4v4_g16_w0_gqa8_vg32": dict(num_q_heads=32, v_bits=4, k_group=16, v_group=32, window=0),
 }
 
 
