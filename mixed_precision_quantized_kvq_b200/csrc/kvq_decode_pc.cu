@@ -13,14 +13,26 @@
 // plus a constant b.  Values keep per-token groups: o = sum_t (p_t vscale_t)
 // c_t + sum_t p_t vzero_t per value group.
 //
-// One CTA of 512 threads per (sequence, kv-head), all g query heads of the
-// kv-group together.  Per 64-position page: the page's raw blocks (key codes,
-// key metadata, value codes, value metadata) are copied into shared memory
-// one page ahead with cp.async; q' and b are formed per key group; scores
-// by (position, 16-channel part) threads reduced with shuffles; online
-// softmax per head (log2 domain); the weighted value codes by (channel,
-// position quarter) threads.  Ring positions are read as bf16 rows.  CUDA
-// cores only: the work per byte is a few multiply-adds.
+// One CTA per (sequence, kv-head), all g query heads of the kv-group
+// together; its warps take the pair's 64-position tiles in turn (warp w:
+// tiles w, w + NW, ...), each warp on its own: the raw page blocks (key
+// codes, key metadata, value codes, value metadata) of its next tile are
+// copied into the warp's second slot with cp.async while it works on the
+// current one, and the warp keeps its own online-softmax state.  The warps'
+// states are merged once, in shared memory, after the last tile: no
+// workspace, no CTA-wide barrier per tile.
+//
+// Per tile, lane l owns positions 2l and 2l+1 for the scores (the codes of a
+// channel run hold them in one byte, or two for 8-bit codes): per channel j
+// the key is dequantized, k = scale*c + zero, and multiplied into every
+// head's score.  For the weighted values lane l owns channels 4l .. 4l+3 and
+// walks the positions with the weights times value scale from a per-warp
+// table.  CUDA cores: a few multiply-adds per byte; codes become floats by
+// placing them in the mantissa of 1.0f (f = 1 + c 2^-bits, exact), which
+// keeps the integer-to-float unit out of the inner loops:
+//     scale*c + zero = (scale 2^bits) f + (zero - scale 2^bits).
+// Ring positions (at or above Q) are read as bf16 rows from global memory,
+// prefetched into L2 when the tile's copies are issued.
 #include <cuda_fp16.h>
 
 #include "kvq_internal.cuh"
@@ -30,32 +42,43 @@ namespace kvq {
 namespace {
 
 constexpr int PD = 128;
-constexpr int PT = 64;              // positions per page
-constexpr int PTH = 512;            // threads per CTA
+constexpr int PT = 64;              // positions per page (one tile)
 constexpr int GMAX = 8;             // query heads per kv-head (kernels for up to 4 and up to 8)
+constexpr int NWMAX = 8;            // warps per CTA at most
+constexpr int SMEM_MAX = 227 * 1024;
 constexpr unsigned FULLM = 0xffffffffu;
 
-// one stage of raw page data: key codes [d][kchan], key metadata [64/kg][d],
-// value codes [d][vchan], value metadata [64][nvg] (byte sizes for 8-bit codes,
-// 16-position key groups, 16-channel value groups at most)
-constexpr int ST_KC = PD * 64;
-constexpr int ST_KM = (PT / 16) * PD * 4;
-constexpr int ST_VC = PD * 64;
-constexpr int ST_VM = PT * 8 * 4;
-constexpr int ST_BYTES = ST_KC + ST_KM + ST_VC + ST_VM;
-
-template <int NH>
-struct PcSmem {
-    float q[PD][NH];                // the query (sm_scale * log2 e folded in), heads innermost
-    float qp[4][PD][NH];            // q * key scale, per key group of the page
-    float qb[4][NH];                // sum_j q_j * key zero, per key group
-    float s[PT][NH];                // scores, then weights
-    float pv[8][PT][NH];            // weight * value scale, per value group
-    float pz[8][NH];                // sum_t weight * value zero, per value group
-    float m[NH], l[NH], alpha[NH];
-    __align__(16) uint8_t raw[2][ST_BYTES];
-    int pages[1];                   // page ids of the sequence's pages (grows into the dynamic tail)
+// shared-memory geometry of one launch (bytes)
+struct PcGeom {
+    int KC, KM, VC, VM;     // the four raw blocks of a (page, kv-head)
+    int SLOT;               // KC + KM + VC + VM
+    int MT;                 // key (scale', zero') table: [PT/kg][PD] float2
+    int PW;                 // weight table: [PT][nvg][NH] float
+    int WAREA;              // per warp: two slots, the tables
+    int OFF_PAGES, OFF_AREAS;
+    int NW, bytes;
 };
+
+__host__ __device__ inline int round_up(int x, int a) { return (x + a - 1) / a * a; }
+
+PcGeom pc_geometry(const Params& p, int max_len, int nh) {
+    PcGeom g{};
+    const int nkg = p.kg > 0 ? PT / p.kg : 1;
+    g.KC = PD * PT * p.kb / 8;
+    g.KM = nkg * PD * 4;
+    g.VC = PD * PT * p.vb / 8;
+    g.VM = PT * p.nvg * 4;
+    g.SLOT = g.KC + g.KM + g.VC + g.VM;
+    g.MT = nkg * PD * 8;
+    g.PW = PT * p.nvg * nh * 4;
+    g.WAREA = round_up(2 * g.SLOT + g.MT + g.PW, 128);
+    g.OFF_PAGES = PD * nh * 4;
+    g.OFF_AREAS = round_up(g.OFF_PAGES + 4 * (max_len / PT + 1), 128);
+    const int nw = (SMEM_MAX - g.OFF_AREAS) / g.WAREA;
+    g.NW = nw < NWMAX ? nw : NWMAX;
+    g.bytes = g.OFF_AREAS + (g.NW > 0 ? g.NW : 0) * g.WAREA;
+    return g;
+}
 
 __device__ __forceinline__ float hbits(uint32_t b) {
     __half_raw r;
@@ -70,17 +93,30 @@ __device__ __forceinline__ void cpa16(uint32_t dst, const void* src) {
 __device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cpa_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 __device__ __forceinline__ void cpa_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-// code of position slot t (0..63) in a channel run of BITS*8 bytes stored
-// chunk-major above 16 bytes: [chunk][d][min(16, run)] (run of channel j)
-template <int BITS>
-__device__ __forceinline__ uint32_t run_code(const uint8_t* base, int j, int t) {
-    constexpr int chan = PT * BITS / 8, cw = chan < 16 ? chan : 16;
-    const int bit = t * BITS, byte = bit >> 3;
-    const uint8_t c8 = base[(byte / cw) * (PD * cw) + j * cw + (byte % cw)];
-    return (uint32_t(c8) >> (bit & 7)) & ((1u << BITS) - 1u);
+__device__ __forceinline__ void prefetch_l2(const void* a) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
 }
-// the codes of positions 16 qt .. 16 qt + 15 of channel j's run, as 16*BITS bits
+
+// code c (BITS wide) found at bit `sh` of x, as the float 1 + c 2^-BITS: the
+// code is moved to the top of the mantissa of 1.0f (shift, then one and-or)
+template <int BITS>
+__device__ __forceinline__ float code_f(uint32_t x, int sh) {
+    constexpr int top = 23 - BITS;
+    constexpr uint32_t mask = ((1u << BITS) - 1u) << top;
+    const uint32_t y = sh <= top ? (x << (top - sh)) : (x >> (sh - top));
+    return __uint_as_float((y & mask) | 0x3F800000u);
+}
+// the same for a shift known at run time only, sh <= 23 - BITS
+template <int BITS>
+__device__ __forceinline__ float code_f_low(uint32_t x, int sh) {
+    constexpr int top = 23 - BITS;
+    constexpr uint32_t mask = ((1u << BITS) - 1u) << top;
+    return __uint_as_float(((x << (top - sh)) & mask) | 0x3F800000u);
+}
+
+// the codes of positions 16 qt .. 16 qt + 15 of channel j's run (runs of
+// BITS*8 bytes, chunk-major above 16 bytes: [chunk][d][min(16, run)]), as
+// 16*BITS bits
 template <int BITS>
 __device__ __forceinline__ void run_quarter(const uint8_t* base, int j, int qt, uint32_t (&w)[4]) {
     constexpr int chan = PT * BITS / 8, cw = chan < 16 ? chan : 16;
@@ -108,308 +144,327 @@ __device__ __forceinline__ void ld_heads(const float* a, float (&x)[NH]) {
     }
 }
 
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULLM, v, o);
+    return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(FULLM, v, o));
+    return v;
+}
+__device__ __forceinline__ float ex2(float x) { return exp2f(x); }
+
 template <int KB, int VB, int NH>
-__global__ void __launch_bounds__(PTH, 1) decode_pc_kernel(const Params p, const void* __restrict__ qv, int q_bf16,
-                                                           const int32_t* __restrict__ lens, int max_len,
-                                                           float sl2, float* __restrict__ out,
-                                                           float* __restrict__ lse) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    PcSmem<NH>& sm = *reinterpret_cast<PcSmem<NH>*>(smem_raw);
+__global__ void __launch_bounds__(NWMAX * 32, 1) decode_pc_kernel(const Params p, const void* __restrict__ qv,
+                                                                  int q_bf16, const int32_t* __restrict__ lens,
+                                                                  int max_len, float sl2, float* __restrict__ out,
+                                                                  float* __restrict__ lse, const PcGeom geo) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
     const int h = blockIdx.x, b = blockIdx.y;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g = p.g, kg = p.kg, nkg_page = PT / kg, vg = p.vg, nvg = p.nvg;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, NW = blockDim.x >> 5;
+    const int g = p.g, kg = p.kg, nvg = p.nvg;
     const int L = max(0, min(lens[b], max_len));
     const size_t orow0 = size_t(b) * p.hq + size_t(h) * g;
     if (L == 0) {                                   // an empty sequence: o = 0, lse = -inf
-        for (int e = tid; e < g * PD; e += PTH) {
+        for (int e = tid; e < g * PD; e += blockDim.x) {
             out[(orow0 + e / PD) * PD + e % PD] = 0.0f;
             if (lse && e % PD == 0) lse[orow0 + e / PD] = -INFINITY;
         }
         return;
     }
+    float* qf = reinterpret_cast<float*>(smem_raw);                          // [PD][NH], times sm_scale log2 e
+    int* pages = reinterpret_cast<int*>(smem_raw + geo.OFF_PAGES);           // page ids of the quantized tiles
+    uint8_t* areas = smem_raw + geo.OFF_AREAS;
     const int R = p.W + kg - 1;                     // ring slots
     const int Q = L - p.W > 0 ? ((L - p.W) / kg) * kg : 0;   // positions below Q live in pages
-    constexpr int kchan = PT * KB / 8, vchan = PT * VB / 8;
-    const int KC = PD * kchan, KM = nkg_page * PD * 4, VC = PD * vchan, VM = PT * nvg * 4;
-    const int ntiles = (L + PT - 1) / PT;
-    const size_t blk = size_t(h);
+    const int ntiles = (L + PT - 1) / PT, npq = (Q + PT - 1) / PT;
+    const size_t prow = size_t(b) * p.hkv + h;      // (sequence, kv-head) row of the ring
 
-    // ---- the query of the g heads (zeros for heads r >= g)
-    for (int e = tid; e < NH * PD; e += PTH) {
+    for (int e = tid; e < NH * PD; e += blockDim.x) {
         const int r = e / PD, j = e % PD;
         float x = 0.0f;
         if (r < g) {
             const size_t idx = (orow0 + r) * PD + j;
             x = q_bf16 ? bfbits(static_cast<const uint16_t*>(qv)[idx]) : static_cast<const float*>(qv)[idx];
         }
-        sm.q[j][r] = x * sl2;
+        qf[j * NH + r] = x * sl2;
     }
-    if (tid < NH) {
-        sm.m[tid] = -INFINITY;
-        sm.l[tid] = 0.0f;
-    }
-    // page ids of the quantized tiles, read once (not one global load per tile)
-    const int npq = (Q + PT - 1) / PT;
-    for (int i = tid; i < npq; i += PTH) {
+    for (int i = tid; i < npq; i += blockDim.x) {
         const int pg = i < p.max_pages ? p.page_table[size_t(b) * p.max_pages + i] : -1;
-        sm.pages[i] = pg >= p.num_pages ? -1 : pg;
+        pages[i] = pg >= p.num_pages ? -1 : pg;
     }
     __syncthreads();
 
-    // raw page blocks of tile i into stage i % 2 (zeros for an unmapped page)
-    auto stage = [&](int i) {
-        if (i >= ntiles || i * PT >= Q) return;
-        uint8_t* dst = sm.raw[i & 1];
-        const int pg = sm.pages[i];
-        const int n16 = (KC + KM + VC + VM) / 16;
-        for (int c = tid; c < n16; c += PTH) {
-            const int off = 16 * c;
-            uint8_t* d = dst + off;
+    uint8_t* area = areas + size_t(w) * geo.WAREA;
+    float2* mt = reinterpret_cast<float2*>(area + 2 * geo.SLOT);
+    float* pw = reinterpret_cast<float*>(area + 2 * geo.SLOT + geo.MT);
+    const uint16_t* kwin = reinterpret_cast<const uint16_t*>(p.k_win) + prow * size_t(R) * PD;
+    const uint16_t* vwin = reinterpret_cast<const uint16_t*>(p.v_win) + prow * size_t(R) * PD;
+
+    // copies of tile i into slot s: the page's four blocks in 16-byte pieces
+    // (zeros for an unmapped page); ring rows of the tile are prefetched to L2
+    auto issue = [&](int i, int s) {
+        if (i >= ntiles) return;
+        const int t0 = i * PT;
+        if (t0 < Q) {
+            uint8_t* dst = area + s * geo.SLOT;
+            const int pg = pages[i];
             if (pg < 0) {
-                *reinterpret_cast<uint4*>(d) = make_uint4(0u, 0u, 0u, 0u);
-                continue;
+                for (int c = lane; c < geo.SLOT / 16; c += 32)
+                    *reinterpret_cast<uint4*>(dst + 16 * c) = make_uint4(0u, 0u, 0u, 0u);
+            } else {
+                const size_t blk = size_t(pg) * p.hkv + h;
+                const uint32_t d0 = ptx::smem_u32(dst);
+                const uint8_t* kc = p.k_codes + blk * geo.KC;
+                const uint8_t* km = reinterpret_cast<const uint8_t*>(p.k_meta) + blk * geo.KM;
+                const uint8_t* vc = p.v_codes + blk * geo.VC;
+                const uint8_t* vm = reinterpret_cast<const uint8_t*>(p.v_meta) + blk * geo.VM;
+                for (int c = lane; c < geo.KC / 16; c += 32) cpa16(d0 + 16 * c, kc + 16 * c);
+                for (int c = lane; c < geo.KM / 16; c += 32) cpa16(d0 + geo.KC + 16 * c, km + 16 * c);
+                for (int c = lane; c < geo.VC / 16; c += 32) cpa16(d0 + geo.KC + geo.KM + 16 * c, vc + 16 * c);
+                for (int c = lane; c < geo.VM / 16; c += 32)
+                    cpa16(d0 + geo.KC + geo.KM + geo.VC + 16 * c, vm + 16 * c);
             }
-            const uint8_t* src;
-            if (off < KC) src = p.k_codes + (size_t(pg) * p.hkv + blk) * KC + off;
-            else if (off < KC + KM)
-                src = reinterpret_cast<const uint8_t*>(p.k_meta) + (size_t(pg) * p.hkv + blk) * KM + (off - KC);
-            else if (off < KC + KM + VC) src = p.v_codes + (size_t(pg) * p.hkv + blk) * VC + (off - KC - KM);
-            else
-                src = reinterpret_cast<const uint8_t*>(p.v_meta) + (size_t(pg) * p.hkv + blk) * VM +
-                      (off - KC - KM - VC);
-            cpa16(ptx::smem_u32(d), src);
+        }
+        // ring positions of the tile: 256-byte key and value rows, two lines each
+        const int w0 = max(t0, Q), w1 = min(t0 + PT, L);
+        for (int e = lane; e < 4 * (w1 - w0); e += 32) {
+            const int t = w0 + (e >> 2), part = e & 3;
+            const uint16_t* row = ((part & 2) ? vwin : kwin) + size_t(t % R) * PD + (part & 1) * 64;
+            prefetch_l2(row);
         }
     };
-    stage(0);
-    cpa_commit();
 
-    float o_acc[NH];                                 // lanes with quarter 0: channel vj, every head
+    float m_run[NH], l_run[NH], o[NH][4];
 #pragma unroll
-    for (int r = 0; r < NH; ++r) o_acc[r] = 0.0f;
-    // (channel, quarter) of the value threads
-    const int vj = warp * 8 + (lane >> 2), vq = lane & 3;
-    // (position, part) of the score threads; a part is channels sp, sp + 8, ..., sp + 120
-    const int st = warp * 4 + (lane >> 3), sp = lane & 7;
+    for (int r = 0; r < NH; ++r) {
+        m_run[r] = -INFINITY;
+        l_run[r] = 0.0f;
+        o[r][0] = o[r][1] = o[r][2] = o[r][3] = 0.0f;
+    }
+    const int tA = 2 * lane, tB = tA + 1;           // score positions of this lane (in the tile)
+    const int j0 = 4 * lane;                        // value channels of this lane
+    const int gv = j0 / p.vg;                       // their value group
 
-    for (int i = 0; i < ntiles; ++i) {
-        stage(i + 1);
+    // where the codes of positions tA, tB of a channel run sit: byte offset
+    // (plus channel * cw) and bit of the first code
+    constexpr int kchan = PT * KB / 8, kcw = kchan < 16 ? kchan : 16;
+    const int kbit = tA * KB, kbyte = kbit >> 3;
+    const int koff = (kbyte / kcw) * (PD * kcw) + (kbyte % kcw), ksh = kbit & 7;
+
+    int slot = 0;
+    issue(w, 0);
+    cpa_commit();
+    for (int i = w; i < ntiles; i += NW) {
+        issue(i + NW, slot ^ 1);
         cpa_commit();
         cpa_wait_1();
-        __syncthreads();                             // stage i landed for every thread
+        __syncwarp();                               // every lane's pieces of tile i have landed
         const int t0 = i * PT;
-        const uint8_t* raw = sm.raw[i & 1];
+        const int nq = min(PT, max(0, Q - t0));     // quantized positions of the tile (a multiple of kg)
+        const int nv = min(PT, L - t0);             // valid positions of the tile
+        const uint8_t* raw = area + slot * geo.SLOT;
         const uint8_t* kc = raw;
-        const uint32_t* km = reinterpret_cast<const uint32_t*>(raw + KC);
-        const uint8_t* vc = raw + KC + KM;
-        const uint32_t* vm = reinterpret_cast<const uint32_t*>(raw + KC + KM + VC);
-        const bool paged_any = t0 < Q;
+        const uint32_t* km = reinterpret_cast<const uint32_t*>(raw + geo.KC);
+        const uint8_t* vc = raw + geo.KC + geo.KM;
+        const uint32_t* vm = reinterpret_cast<const uint32_t*>(raw + geo.KC + geo.KM + geo.VC);
 
-        // ---- q' = q * key scale and b = q . key zero, per key group of the page
-        if (paged_any) {
-            for (int e = tid; e < nkg_page * PD; e += PTH) {
-                const int gi = e / PD, j = e % PD;
-                const float sc = hbits(km[gi * PD + j] & 0xffffu);
-#pragma unroll
-                for (int r = 0; r < NH; ++r) sm.qp[gi][j][r] = sm.q[j][r] * sc;
+        // ---- key groups of the tile: (scale 2^KB, zero - scale 2^KB) per channel
+        if (nq > 0) {
+            for (int e = lane; e < (nq / kg) * PD; e += 32) {
+                const uint32_t m = km[e];
+                const float s = hbits(m & 0xffffu) * float(1 << KB);
+                mt[e] = make_float2(s, hbits(m >> 16) - s);
             }
-            // one warp per key group: 4 channels per lane, then a warp sum per head
-            for (int gi = warp; gi < nkg_page; gi += PTH / 32) {
-                float acc[NH];
+        }
+        __syncwarp();
+
+        // ---- scores of positions tA, tB for every head (log2 domain)
+        float sA[NH], sB[NH];
 #pragma unroll
-                for (int r = 0; r < NH; ++r) acc[r] = 0.0f;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int j = 4 * lane + c;
-                    const float z = hbits(km[gi * PD + j] >> 16);
-#pragma unroll
-                    for (int r = 0; r < NH; ++r) acc[r] = fmaf(sm.q[j][r], z, acc[r]);
-                }
+        for (int r = 0; r < NH; ++r) sA[r] = sB[r] = 0.0f;
+        if (tA < nq) {
+            const float2* mg = mt + (tA / kg) * PD;
+            const uint8_t* kp = kc + koff;
+#pragma unroll 4
+            for (int j = 0; j < PD; ++j) {
+                uint32_t x;
+                if constexpr (KB == 8) x = *reinterpret_cast<const uint16_t*>(kp + j * kcw);
+                else x = kp[j * kcw];
+                const float fA = code_f_low<KB>(x, ksh), fB = code_f_low<KB>(x, ksh + KB);
+                const float2 sz = mg[j];
+                const float kA = fmaf(sz.x, fA, sz.y), kB = fmaf(sz.x, fB, sz.y);
+                float qq[NH];
+                ld_heads<NH>(qf + j * NH, qq);
 #pragma unroll
                 for (int r = 0; r < NH; ++r) {
-#pragma unroll
-                    for (int o = 16; o; o >>= 1) acc[r] += __shfl_xor_sync(FULLM, acc[r], o);
-                    if (lane == 0) sm.qb[gi][r] = acc[r];
+                    sA[r] = fmaf(qq[r], kA, sA[r]);
+                    sB[r] = fmaf(qq[r], kB, sB[r]);
                 }
             }
-        }
-        __syncthreads();
-
-        // ---- scores: thread (position st, channels sp + 8c), every head
-        {
-            const int pos = t0 + st;
-            float acc[NH];
+        } else if (tA < nv) {
+            const bool hasB = tB < nv;
+            const uint16_t* ra = kwin + size_t((t0 + tA) % R) * PD;
+            const uint16_t* rb = hasB ? kwin + size_t((t0 + tB) % R) * PD : ra;
+#pragma unroll 2
+            for (int j8 = 0; j8 < PD; j8 += 8) {
+                const uint4 a = *reinterpret_cast<const uint4*>(ra + j8);
+                const uint4 c = *reinterpret_cast<const uint4*>(rb + j8);
+                const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-            for (int r = 0; r < NH; ++r) acc[r] = 0.0f;
-            if (pos < L) {
-                if (pos < Q) {
-                    const int gi = st / kg;
-#pragma unroll 4
-                    for (int c = 0; c < 16; ++c) {
-                        const int j = sp + 8 * c;
-                        const float x = float(run_code<KB>(kc, j, st));
-                        float qq[NH];
-                        ld_heads<NH>(&sm.qp[gi][j][0], qq);
+                for (int e = 0; e < 8; ++e) {
+                    const float kA = bfbits((aw[e >> 1] >> (16 * (e & 1))) & 0xffffu);
+                    const float kB = bfbits((cw[e >> 1] >> (16 * (e & 1))) & 0xffffu);
+                    float qq[NH];
+                    ld_heads<NH>(qf + (j8 + e) * NH, qq);
 #pragma unroll
-                        for (int r = 0; r < NH; ++r) acc[r] = fmaf(qq[r], x, acc[r]);
-                    }
-                } else {
-                    const uint16_t* kw = reinterpret_cast<const uint16_t*>(p.k_win) +
-                                         ((size_t(b) * p.hkv + blk) * R + size_t(pos % R)) * PD;
-#pragma unroll 4
-                    for (int c = 0; c < 16; ++c) {
-                        const int j = sp + 8 * c;
-                        const float x = bfbits(kw[j]);
-                        float qq[NH];
-                        ld_heads<NH>(&sm.q[j][0], qq);
-#pragma unroll
-                        for (int r = 0; r < NH; ++r) acc[r] = fmaf(qq[r], x, acc[r]);
+                    for (int r = 0; r < NH; ++r) {
+                        sA[r] = fmaf(qq[r], kA, sA[r]);
+                        sB[r] = fmaf(qq[r], kB, sB[r]);
                     }
                 }
             }
-#pragma unroll
-            for (int r = 0; r < NH; ++r) {
-                float v = acc[r];
-                v += __shfl_xor_sync(FULLM, v, 1);
-                v += __shfl_xor_sync(FULLM, v, 2);
-                v += __shfl_xor_sync(FULLM, v, 4);
-                acc[r] = v;
-            }
-            if (sp == 0) {
-#pragma unroll
-                for (int r = 0; r < NH; ++r)
-                    sm.s[st][r] = pos >= L ? -INFINITY : (pos < Q ? acc[r] + sm.qb[st / kg][r] : acc[r]);
-            }
         }
-        __syncthreads();
+        const bool vA = tA < nv, vB = tB < nv;
 
-        // ---- online softmax: warp r for head r
-        if (warp < g) {
-            const int r = warp;
-            const float x0 = sm.s[lane][r], x1 = sm.s[lane + 32][r];
-            float mx = fmaxf(x0, x1);
-#pragma unroll
-            for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULLM, mx, o));
-            const float m_old = sm.m[r];
-            const float mn = fmaxf(m_old, mx);       // finite: position t0 < L is in every tile
-            const float p0 = exp2f(x0 - mn), p1 = exp2f(x1 - mn);
-            float sum = p0 + p1;
-#pragma unroll
-            for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(FULLM, sum, o);
-            const float al = exp2f(m_old - mn);      // 0 on the first tile
-            sm.s[lane][r] = p0;
-            sm.s[lane + 32][r] = p1;
-            if (lane == 0) {
-                sm.m[r] = mn;
-                sm.l[r] = fmaf(sm.l[r], al, sum);
-                sm.alpha[r] = al;
-            }
-        } else if (warp < NH && lane < PT / 2) {
-            // heads r >= g: zero weights (their rows are never output)
-            sm.s[lane][warp] = 0.0f;
-            sm.s[lane + 32][warp] = 0.0f;
-            if (lane == 0) sm.alpha[warp] = 0.0f;
-        }
-        __syncthreads();
-
-        // ---- weights times value scale, and the zero-point sums, per value group
-        if (paged_any) {
-            for (int e = tid; e < nvg * PT; e += PTH) {
-                const int gv = e / PT, t = e % PT;
-                const float sc = t0 + t < Q ? hbits(vm[t * nvg + gv] & 0xffffu) : 0.0f;
-#pragma unroll
-                for (int r = 0; r < NH; ++r) sm.pv[gv][t][r] = sm.s[t][r] * sc;
-            }
-            for (int gv = warp; gv < nvg; gv += PTH / 32) {
-                float acc[NH];
-#pragma unroll
-                for (int r = 0; r < NH; ++r) acc[r] = 0.0f;
-                for (int t = lane; t < PT; t += 32) {
-                    const float z = t0 + t < Q ? hbits(vm[t * nvg + gv] >> 16) : 0.0f;
-#pragma unroll
-                    for (int r = 0; r < NH; ++r) acc[r] = fmaf(sm.s[t][r], z, acc[r]);
-                }
-#pragma unroll
-                for (int r = 0; r < NH; ++r) {
-#pragma unroll
-                    for (int o = 16; o; o >>= 1) acc[r] += __shfl_xor_sync(FULLM, acc[r], o);
-                    if (lane == 0) sm.pz[gv][r] = acc[r];
-                }
-            }
-        }
-        __syncthreads();
-
-        // ---- o = o * alpha + sum_t w_t v_t: thread (channel vj, positions 16 vq .. 16 vq + 15)
-        {
-            float acc[NH];
-#pragma unroll
-            for (int r = 0; r < NH; ++r) acc[r] = 0.0f;
-            const int gv = vj / vg;
-            const int tq0 = t0 + 16 * vq;
-            if (tq0 + 15 < Q) {
-                // every position of the quarter in the page: codes from one load
-                uint32_t w[4];
-                run_quarter<VB>(vc, vj, vq, w);
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const int bit = c * VB;
-                    const float x = float((w[bit >> 5] >> (bit & 31)) & ((1u << VB) - 1u));
-                    float pw[NH];
-                    ld_heads<NH>(&sm.pv[gv][16 * vq + c][0], pw);
-#pragma unroll
-                    for (int r = 0; r < NH; ++r) acc[r] = fmaf(pw[r], x, acc[r]);
-                }
-            } else {
-                for (int c = 0; c < 16; ++c) {
-                    const int t = 16 * vq + c, pos = t0 + t;
-                    if (pos >= L) break;
-                    float x;
-                    float pw[NH];
-                    if (pos < Q) {
-                        x = float(run_code<VB>(vc, vj, t));
-                        ld_heads<NH>(&sm.pv[gv][t][0], pw);
-                    } else {
-                        x = bfbits(reinterpret_cast<const uint16_t*>(
-                            p.v_win)[((size_t(b) * p.hkv + blk) * R + size_t(pos % R)) * PD + vj]);
-                        ld_heads<NH>(&sm.s[t][0], pw);
-                    }
-#pragma unroll
-                    for (int r = 0; r < NH; ++r) acc[r] = fmaf(pw[r], x, acc[r]);
-                }
-            }
-#pragma unroll
-            for (int r = 0; r < NH; ++r) {
-                float v = acc[r];
-                v += __shfl_xor_sync(FULLM, v, 1);
-                v += __shfl_xor_sync(FULLM, v, 2);
-                if (vq == 0) o_acc[r] = fmaf(o_acc[r], sm.alpha[r], v + (paged_any ? sm.pz[gv][r] : 0.0f));
-            }
-        }
-        __syncthreads();                             // stage i is free for tile i + 2
-    }
-    cpa_wait_0();
-
-    // ---- o / l, lse = (m + log2 l) ln 2
-    if (vq == 0) {
+        // ---- online softmax over the tile, per head
+        float pA[NH], pB[NH], alpha[NH];
 #pragma unroll
         for (int r = 0; r < NH; ++r) {
-            if (r >= g) break;
-            const float l = sm.l[r];
-            out[(orow0 + r) * PD + vj] = o_acc[r] / l;
-            if (lse && vj == 0) lse[orow0 + r] = (sm.m[r] + log2f(l)) * 0.693147180559945309f;
+            const float mx = warp_max(fmaxf(vA ? sA[r] : -INFINITY, vB ? sB[r] : -INFINITY));
+            const float mn = fmaxf(m_run[r], mx);    // finite: position t0 < L is in the tile
+            alpha[r] = ex2(m_run[r] - mn);           // 0 on the warp's first tile
+            m_run[r] = mn;
+            pA[r] = vA ? ex2(sA[r] - mn) : 0.0f;
+            pB[r] = vB ? ex2(sB[r] - mn) : 0.0f;
+            l_run[r] = fmaf(l_run[r], alpha[r], warp_sum(pA[r] + pB[r]));
+#pragma unroll
+            for (int c = 0; c < 4; ++c) o[r][c] *= alpha[r];
         }
+
+        // ---- weight table [t][value group][head]: quantized positions p*scale*2^VB,
+        // ring positions p; per value group the zero points and the mantissa offsets
+        // of the quantized positions: sum_t p (zero - scale 2^VB)
+        float corr[NH];
+#pragma unroll
+        for (int r = 0; r < NH; ++r) corr[r] = 0.0f;
+        for (int gg = 0; gg < nvg; ++gg) {
+            float z[NH];
+#pragma unroll
+            for (int r = 0; r < NH; ++r) z[r] = 0.0f;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int t = tA + half;
+                const float* pp = half ? pB : pA;
+                if (t >= nv) continue;
+                float wt[NH];
+                if (t < nq) {
+                    const uint32_t m = vm[t * nvg + gg];
+                    const float s = hbits(m & 0xffffu) * float(1 << VB), zz = hbits(m >> 16) - s;
+#pragma unroll
+                    for (int r = 0; r < NH; ++r) {
+                        wt[r] = pp[r] * s;
+                        z[r] = fmaf(pp[r], zz, z[r]);
+                    }
+                } else {
+#pragma unroll
+                    for (int r = 0; r < NH; ++r) wt[r] = pp[r];
+                }
+#pragma unroll
+                for (int r = 0; r < NH; r += 4)
+                    *reinterpret_cast<float4*>(pw + (t * nvg + gg) * NH + r) =
+                        make_float4(wt[r], wt[r + 1], wt[r + 2], wt[r + 3]);
+            }
+            if (nq > 0) {
+#pragma unroll
+                for (int r = 0; r < NH; ++r) {
+                    const float zs = warp_sum(z[r]);
+                    if (gg == gv) corr[r] = zs;
+                }
+            }
+        }
+        __syncwarp();                               // the weight table is complete
+
+        // ---- o += sum_t w_t v_t over the tile: channels j0 .. j0+3
+        for (int qt = 0; qt < nq / 16; ++qt) {
+            uint32_t cw4[4][4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) run_quarter<VB>(vc, j0 + c, qt, cw4[c]);
+#pragma unroll
+            for (int tt = 0; tt < 16; ++tt) {
+                float pq[NH];
+                ld_heads<NH>(pw + ((16 * qt + tt) * nvg + gv) * NH, pq);
+                const int bit = tt * VB;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float f = code_f<VB>(cw4[c][bit >> 5], bit & 31);
+#pragma unroll
+                    for (int r = 0; r < NH; ++r) o[r][c] = fmaf(pq[r], f, o[r][c]);
+                }
+            }
+        }
+#pragma unroll 4
+        for (int t = nq; t < nv; ++t) {
+            const uint2 v = *reinterpret_cast<const uint2*>(vwin + size_t((t0 + t) % R) * PD + j0);
+            const float x[4] = {bfbits(v.x & 0xffffu), bfbits(v.x >> 16), bfbits(v.y & 0xffffu), bfbits(v.y >> 16)};
+            float pq[NH];
+            ld_heads<NH>(pw + (t * nvg + gv) * NH, pq);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int r = 0; r < NH; ++r) o[r][c] = fmaf(pq[r], x[c], o[r][c]);
+        }
+#pragma unroll
+        for (int r = 0; r < NH; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) o[r][c] += corr[r];
+        __syncwarp();                               // slot, tables free for the next tiles
+        slot ^= 1;
+    }
+    cpa_wait_0();
+    __syncthreads();                                // every warp is done with its area
+
+    // ---- merge the warps' states: [warp][head][PD + 2] over the warp areas
+    constexpr int PS = PD + 4;
+    float* part = reinterpret_cast<float*>(areas);
+#pragma unroll
+    for (int r = 0; r < NH; ++r) {
+        if (r >= g) break;
+        *reinterpret_cast<float4*>(part + (w * NH + r) * PS + j0) = make_float4(o[r][0], o[r][1], o[r][2], o[r][3]);
+        if (lane == 0) {
+            part[(w * NH + r) * PS + PD] = m_run[r];
+            part[(w * NH + r) * PS + PD + 1] = l_run[r];
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < g * PD; e += blockDim.x) {
+        const int r = e / PD, j = e % PD;
+        float M = -INFINITY;
+        for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, part[(ww * NH + r) * PS + PD]);
+        float num = 0.0f, den = 0.0f;
+        for (int ww = 0; ww < NW; ++ww) {
+            const float mw = part[(ww * NH + r) * PS + PD];
+            if (mw == -INFINITY) continue;          // a warp without tiles
+            const float f = ex2(mw - M);
+            num = fmaf(part[(ww * NH + r) * PS + j], f, num);
+            den = fmaf(part[(ww * NH + r) * PS + PD + 1], f, den);
+        }
+        out[(orow0 + r) * PD + j] = num / den;
+        if (lse && j == 0) lse[orow0 + r] = (M + log2f(den)) * 0.693147180559945309f;
     }
 }
 
 template <int KB, int NH>
 cudaError_t launch_nh_pc(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len, float sl2,
                          float* out, float* lse, cudaStream_t s) {
+    const PcGeom geo = pc_geometry(p, max_len, NH);
     const dim3 grid(p.hkv, p.batch);
-    // the page-id table grows past the struct: one int per quantized page
-    const int bytes = int(sizeof(PcSmem<NH>)) + 4 * (max_len / PT + 1);
     auto go = [&](auto kern) -> cudaError_t {
-        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, geo.bytes);
         if (e != cudaSuccess) return e;
-        kern<<<grid, PTH, bytes, s>>>(p, q, q_bf16, lens, max_len, sl2, out, lse);
+        kern<<<grid, geo.NW * 32, geo.bytes, s>>>(p, q, q_bf16, lens, max_len, sl2, out, lse, geo);
         return cudaGetLastError();
     };
     switch (p.vb) {
@@ -430,10 +485,11 @@ cudaError_t launch_kb_pc(const Params& p, const void* q, int q_bf16, const int32
 }  // namespace
 
 bool decode_pc_supported(const Params& p, int max_len) {
-    // shared memory: the struct plus one page id per quantized page
-    const size_t bytes = sizeof(PcSmem<8>) + 4 * size_t(max_len / PT + 1);
-    return p.d == PD && p.g >= 1 && p.g <= GMAX && (p.kg == 16 || p.kg == 32 || p.kg == 64) && p.vg >= 16 &&
-           PD % p.vg == 0 && !p.rotate && bytes <= 227 * 1024;
+    if (!(p.d == PD && p.g >= 1 && p.g <= GMAX && (p.kg == 16 || p.kg == 32 || p.kg == 64) && p.vg >= 16 &&
+          PD % p.vg == 0 && !p.rotate && max_len >= 0))
+        return false;
+    // two warps at least, each with two page slots and its tables
+    return pc_geometry(p, max_len, p.g <= 4 ? 4 : 8).NW >= 2;
 }
 
 cudaError_t launch_decode_per_channel(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len,
