@@ -3,7 +3,7 @@
 //
 // Append = two launches on the caller's stream: the group kernel
 // (grid: groups completed by the longest append x kv-heads x sequences,
-// 128 threads, kg*d*9 bytes of shared memory) reads ring slots of the
+// 512 threads, about kg*d*10 bytes of shared memory) reads ring slots of the
 // positions it quantizes; the ring kernel (grid: kv-heads x sequences)
 // then writes the new positions that stay in the window.
 #include "kvq_channel.cuh"
@@ -15,6 +15,7 @@ namespace {
 struct ChanCtx {
     float* s;
     __device__ int tid() const { return threadIdx.x; }
+    __device__ int nthreads() const { return blockDim.x; }
     __device__ int bx() const { return blockIdx.x; }
     __device__ int by() const { return blockIdx.y; }
     __device__ int bz() const { return blockIdx.z; }
@@ -31,7 +32,7 @@ struct ChanCtx {
     __device__ void atomic_or(uint32_t* p, uint32_t v) const { atomicOr(p, v); }
 };
 
-__global__ void __launch_bounds__(chan::kThreads) append_groups_kernel(chan::View v) {
+__global__ void __launch_bounds__(chan::kGroupThreads) append_groups_kernel(chan::View v) {
     extern __shared__ __align__(16) float smem[];
     ChanCtx cx{smem};
     chan::append_groups_body(cx, v);
@@ -92,13 +93,13 @@ cudaError_t launch_append_per_channel(const Params& p, const void* k_new, const 
     cudaError_t e;
     if (!configured[dev]) {
         e = cudaFuncSetAttribute(append_groups_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(chan::append_smem_bytes(128, 64)));
+                                 int(chan::append_smem_bytes(128, 64, 8)));
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
-    const size_t sm = chan::append_smem_bytes(p.d, p.kg);
+    const size_t sm = chan::append_smem_bytes(p.d, p.kg, p.nvg);
     const int groups = (max_new + p.kg - 1) / p.kg;
-    append_groups_kernel<<<dim3(groups, p.hkv, p.batch), chan::kThreads, sm, s>>>(v);
+    append_groups_kernel<<<dim3(groups, p.hkv, p.batch), chan::kGroupThreads, sm, s>>>(v);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ring_write_kernel<<<dim3(p.hkv, p.batch), chan::kThreads, 0, s>>>(v);
     return cudaGetLastError();

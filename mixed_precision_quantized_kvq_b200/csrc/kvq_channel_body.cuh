@@ -114,30 +114,38 @@ KVQ_HD size_t ring_off(const View& v, int b, int h, int pos) {
     return ((size_t(b) * v.hkv + h) * v.R + size_t(pos % v.R)) * v.d;
 }
 
-// One group of n values x[0], x[stride], ...: codes into c[0..n), returns
-// the metadata word {fp16 scale | fp16 zero << 16}.
-template <class Ctx>
-KVQ_HD uint32_t quantize_span(const Ctx& cx, const float* x, int stride, int n, int bits, uint8_t* c) {
-    float mn = x[0], mx = x[0];
+// The quantizer of one group, in three parts so that several threads can
+// share a group: the extremes of a part of the group, the metadata word
+// {fp16 scale | fp16 zero << 16} of the group from its extremes (with the
+// fp32 zero and scale the codes are formed with), and the codes of a part.
+KVQ_HD void span_extremes(const float* x, int stride, int n, float& mn, float& mx) {
+    mn = x[0], mx = x[0];
     for (int i = 1; i < n; ++i) {
         mn = fminf(mn, x[size_t(i) * stride]);
         mx = fmaxf(mx, x[size_t(i) * stride]);
     }
+}
+template <class Ctx>
+KVQ_HD uint32_t span_meta(const Ctx& cx, float mn, float mx, int bits, float& zf, float& sf) {
     if (mn == 0.0f) mn = 0.0f;       // canonical +0
     if (mx == 0.0f) mx = 0.0f;
     const float qmax = float((1 << bits) - 1);
     const uint16_t zh = cx.f2h_rd(mn);
-    const float zf = half_f32(zh);
+    zf = half_f32(zh);
     const float s32 = cx.div_ru(cx.sub_ru(mx, zf), qmax);
     uint16_t sh = cx.f2h_ru(s32);
-    const float sf = half_f32(sh);
+    sf = half_f32(sh);
     if (sf == 0.0f) sh = 0;
+    return uint32_t(sh) | (uint32_t(zh) << 16);
+}
+template <class Ctx>
+KVQ_HD void span_codes(const Ctx& cx, const float* x, int stride, int n, float zf, float sf, int bits, uint8_t* c) {
+    const float qmax = float((1 << bits) - 1);
     for (int i = 0; i < n; ++i) {
         float code = 0.0f;
         if (sf != 0.0f) code = fminf(fmaxf(rintf(cx.div_rn(cx.sub_rn(x[size_t(i) * stride], zf), sf)), 0.0f), qmax);
         c[i] = uint8_t(code);
     }
-    return uint32_t(sh) | (uint32_t(zh) << 16);
 }
 
 // Write codes c[0], c[cs], ... of slots slot0 .. slot0+n-1 into channel j's
@@ -168,19 +176,38 @@ KVQ_HD void put_run(const Ctx& cx, uint8_t* blk, int d, int ch, int j, int slot0
     }
 }
 
-// shared memory of one append CTA (bytes)
-KVQ_HD size_t append_smem_bytes(int d, int kg) { return size_t(kg) * d * (4 + 4 + 1); }
+// Threads of one append CTA on the GPU (the body works with any count).
+constexpr int kGroupThreads = 512;
+// Parts a group's values are split into between threads.
+constexpr int kParts = 4;
+
+// shared memory of one append CTA (bytes): keys and values as fp32 rows of
+// d + 1 floats (the padding puts rows that different threads walk in
+// different banks), the parts' extremes, key codes [d][kg], value codes as
+// rows of d + 4 bytes
+KVQ_HD size_t append_smem_bytes(int d, int kg, int nvg) {
+    return size_t(kg) * size_t(d + 1) * 8 + size_t(d + kg * nvg) * kParts * 8 + size_t(d) * kg +
+           size_t(kg) * size_t(d + 4);
+}
+
+struct alignas(16) Words4 {
+    uint32_t w[4];
+};
 
 // Append, part 1.  CTA (gi, h, b): key group gi of the groups that this
 // append completes for sequence b, kv-head h: its kg positions' keys and
 // values (from the ring when older than L, else from the new rows) are
 // quantized into their page.  Must run before part 2 rewrites ring slots.
+// The CTA's groups (d key groups along positions, kg * nvg value groups
+// along channels) are split into kParts parts each: the parts' extremes,
+// then each part's codes from its group's metadata, then the codes packed
+// into the channel runs.
 #ifdef __CUDACC__
 #pragma nv_exec_check_disable
 #endif
 template <class Ctx>
 KVQ_HD void append_groups_body(Ctx& cx, const View& v) {
-    const int gi = cx.bx(), h = cx.by(), b = cx.bz(), tid = cx.tid();
+    const int gi = cx.bx(), h = cx.by(), b = cx.bz(), tid = cx.tid(), NT = cx.nthreads();
     const int d = v.d, G = v.kg;
     const int L = v.lens[b], n = v.cu_new[b + 1] - v.cu_new[b];
     if (n <= 0 || L < 0) return;
@@ -190,45 +217,103 @@ KVQ_HD void append_groups_body(Ctx& cx, const View& v) {
     const int pg = phys_page(v, b, g0 / kPage);
     if (pg < 0) return;
     const int slot0 = g0 % kPage;
+    const int dp = d + 1, cp = d + 4;                         // padded row strides
+    const int T = d + G * v.nvg;                              // groups: keys, then values
     float* sK = cx.smem();
-    float* sV = sK + G * d;
-    uint8_t* sC = reinterpret_cast<uint8_t*>(sV + G * d);   // value codes [G][d]
+    float* sV = sK + G * dp;
+    float* sX = sV + G * dp;                                  // [T][kParts] {min, max}
+    uint8_t* sKC = reinterpret_cast<uint8_t*>(sX + 2 * T * kParts);   // key codes [d][G]
+    uint8_t* sC = sKC + d * G;                                // value codes [G][d + 4]
 
-    for (int e = tid; e < G * d; e += kThreads) {
-        const int t = e / d, j = e % d, pos = g0 + t;
-        float kx, vx;
-        if (pos < L) {
-            const size_t w = ring_off(v, b, h, pos) + j;
-            kx = bf16_f32(v.k_win[w]);
-            vx = bf16_f32(v.v_win[w]);
-        } else {
-            const size_t row = (size_t(v.cu_new[b] + pos - L) * v.hkv + h) * d + j;
-            if (v.in_bf16) {
-                kx = bf16_f32(static_cast<const uint16_t*>(v.k_new)[row]);
-                vx = bf16_f32(static_cast<const uint16_t*>(v.v_new)[row]);
-            } else {
-                kx = static_cast<const float*>(v.k_new)[row];
-                vx = static_cast<const float*>(v.v_new)[row];
+    // positions still in the ring: 16-byte loads of 8 channels, every load of a
+    // thread's batch issued before its stores (one memory latency per batch)
+    const int nring = imax(0, imin(G, L - g0));
+    const int d8 = d / 8, nvec = nring * d8;
+    for (int base = 0; base < nvec; base += 8 * NT) {
+        Words4 kk[8] = {}, vv[8] = {};
+        for (int u = 0; u < 8; ++u) {
+            const int e = base + u * NT + tid;
+            if (e < nvec) {
+                const size_t w = ring_off(v, b, h, g0 + e / d8) + 8 * size_t(e % d8);
+                kk[u] = *reinterpret_cast<const Words4*>(v.k_win + w);
+                vv[u] = *reinterpret_cast<const Words4*>(v.v_win + w);
             }
         }
-        sK[t * d + j] = kx;
-        sV[t * d + j] = vx;
+        for (int u = 0; u < 8; ++u) {
+            const int e = base + u * NT + tid;
+            if (e >= nvec) continue;
+            const int t = e / d8, j = 8 * (e % d8);
+            for (int c = 0; c < 8; ++c) {
+                sK[t * dp + j + c] = bf16_f32(uint16_t(kk[u].w[c >> 1] >> (16 * (c & 1))));
+                sV[t * dp + j + c] = bf16_f32(uint16_t(vv[u].w[c >> 1] >> (16 * (c & 1))));
+            }
+        }
+    }
+    // positions among the new rows
+    for (int e = nring * d + tid; e < G * d; e += NT) {
+        const int t = e / d, j = e % d, pos = g0 + t;
+        const size_t row = (size_t(v.cu_new[b] + pos - L) * v.hkv + h) * d + j;
+        float kx, vx;
+        if (v.in_bf16) {
+            kx = bf16_f32(static_cast<const uint16_t*>(v.k_new)[row]);
+            vx = bf16_f32(static_cast<const uint16_t*>(v.v_new)[row]);
+        } else {
+            kx = static_cast<const float*>(v.k_new)[row];
+            vx = static_cast<const float*>(v.v_new)[row];
+        }
+        sK[t * dp + j] = kx;
+        sV[t * dp + j] = vx;
     }
     cx.sync();
-    // keys: one group per channel, one thread per channel
-    for (int j = tid; j < d; j += kThreads) {
-        uint8_t c[64];
-        *k_meta_at(v, pg, h, slot0, j) = quantize_span(cx, sK + j, d, G, v.kb, c);
-        put_run(cx, k_block(v, pg, h), d, v.kch, j, slot0, G, v.kb, c, 1);
-    }
-    // values: per token, groups of vg channels
-    for (int e = tid; e < G * v.nvg; e += kThreads) {
-        const int t = e / v.nvg, grp = e % v.nvg;
-        *v_meta_at(v, pg, h, slot0 + t, grp) =
-            quantize_span(cx, sV + t * d + grp * v.vg, 1, v.vg, v.vb, sC + t * d + grp * v.vg);
+    // part e % kParts of group e / kParts: its values (x, stride, count)
+    auto part = [&](int e, const float*& x, int& stride, int& m) {
+        const int grp = e / kParts, k = e % kParts;
+        if (grp < d) {                                        // key group: channel grp
+            m = G / kParts;
+            x = sK + size_t(k * m) * dp + grp;
+            stride = dp;
+        } else {                                              // value group: (position, channel group)
+            const int t = (grp - d) / v.nvg, cg = (grp - d) % v.nvg;
+            m = v.vg / kParts;
+            x = sV + size_t(t) * dp + cg * v.vg + k * m;
+            stride = 1;
+        }
+    };
+    for (int e = tid; e < T * kParts; e += NT) {
+        const float* x;
+        int stride, m;
+        part(e, x, stride, m);
+        span_extremes(x, stride, m, sX[2 * e], sX[2 * e + 1]);
     }
     cx.sync();
-    for (int j = tid; j < d; j += kThreads) put_run(cx, v_block(v, pg, h), d, v.vch, j, slot0, G, v.vb, sC + j, d);
+    for (int e = tid; e < T * kParts; e += NT) {
+        const int grp = e / kParts, k = e % kParts;
+        const float* ex = sX + 2 * grp * kParts;
+        float mn = ex[0], mx = ex[1];
+        for (int i = 1; i < kParts; ++i) {
+            mn = fminf(mn, ex[2 * i]);
+            mx = fmaxf(mx, ex[2 * i + 1]);
+        }
+        float zf, sf;
+        const bool key = grp < d;
+        const uint32_t meta = span_meta(cx, mn, mx, key ? v.kb : v.vb, zf, sf);
+        const float* x;
+        int stride, m;
+        part(e, x, stride, m);
+        if (key) {
+            if (k == 0) *k_meta_at(v, pg, h, slot0, grp) = meta;
+            span_codes(cx, x, stride, m, zf, sf, v.kb, sKC + grp * G + k * m);
+        } else {
+            const int t = (grp - d) / v.nvg, cg = (grp - d) % v.nvg;
+            if (k == 0) *v_meta_at(v, pg, h, slot0 + t, cg) = meta;
+            span_codes(cx, x, stride, m, zf, sf, v.vb, sC + t * cp + cg * v.vg + k * m);
+        }
+    }
+    cx.sync();
+    for (int e = tid; e < 2 * d; e += NT) {
+        if (e < d) put_run(cx, k_block(v, pg, h), d, v.kch, e, slot0, G, v.kb, sKC + e * G, 1);
+        else put_run(cx, v_block(v, pg, h), d, v.vch, e - d, slot0, G, v.vb, sC + (e - d), cp);
+    }
 }
 
 // Append, part 2.  CTA (h, b): the new positions that stay in the window
@@ -244,7 +329,7 @@ KVQ_HD void ring_write_body(Ctx& cx, const View& v) {
     if (n <= 0 || L < 0) return;
     const int w0 = imax(paged_len(L + n, v.W, v.kg), L);
     const int cnt = L + n - w0;
-    for (int e = tid; e < cnt * d; e += kThreads) {
+    for (int e = tid; e < cnt * d; e += cx.nthreads()) {
         const int pos = w0 + e / d, j = e % d;
         const size_t row = (size_t(v.cu_new[b] + pos - L) * v.hkv + h) * d + j;
         const size_t dst = ring_off(v, b, h, pos) + j;
@@ -268,7 +353,7 @@ KVQ_HD void dequant_body(Ctx& cx, const View& v) {
     const int L = v.lens[b];
     const int Lc = imin(L, v.max_len);
     const int Q = paged_len(L, v.W, v.kg);
-    for (int e = tid; e < kPage * d; e += kThreads) {
+    for (int e = tid; e < kPage * d; e += cx.nthreads()) {
         const int t = e / d, j = e % d, pos = tile * kPage + t;
         if (pos >= Lc) continue;
         const size_t o = ((size_t(b) * v.hkv + h) * v.max_len + pos) * d + j;

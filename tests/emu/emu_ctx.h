@@ -51,6 +51,7 @@ struct Ctx {
     Block* blk;
     int t;
     int tid() const { return t; }
+    int nthreads() const { return blk->nt; }
     int bx() const { return blk->bx; }
     int by() const { return blk->by; }
     int bz() const { return blk->bz; }

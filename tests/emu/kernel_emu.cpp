@@ -115,7 +115,7 @@ int append_pc(emu::Arrays& A, std::map<std::string, double>& P) {
     v.cu_new = A.get<int32_t>("cu_new");
     const int max_new = int(P.at("max_new"));
     emu::run_grid((max_new + v.kg - 1) / v.kg, v.hkv, v.batch, kvq::chan::kThreads,
-                  kvq::chan::append_smem_bytes(v.d, v.kg),
+                  kvq::chan::append_smem_bytes(v.d, v.kg, v.nvg),
                   [&v](emu::Ctx& cx) { kvq::chan::append_groups_body(cx, v); });
     emu::run_grid(v.hkv, v.batch, 1, kvq::chan::kThreads, 0,
                   [&v](emu::Ctx& cx) { kvq::chan::ring_write_body(cx, v); });
