@@ -14,7 +14,7 @@
 // c_t + sum_t p_t vzero_t per value group.
 //
 // One CTA per (sequence, kv-head), all g query heads of the kv-group
-// together; its warps take the pair's 64-position tiles in turn (warp w:
+// together; its warps (up to 12) take the pair's 64-position tiles in turn (warp w:
 // tiles w, w + NW, ...), each warp on its own: the raw page blocks (key
 // codes, key metadata, value codes, value metadata) of its next tile are
 // copied into the warp's second slot with cp.async while it works on the
@@ -22,17 +22,24 @@
 // states are merged once, in shared memory, after the last tile: no
 // workspace, no CTA-wide barrier per tile.
 //
-// Per tile, lane l owns positions 2l and 2l+1 for the scores (the codes of a
-// channel run hold them in one byte, or two for 8-bit codes): per channel j
-// the key is dequantized, k = scale*c + zero, and multiplied into every
-// head's score.  For the weighted values lane l owns channels 4l .. 4l+3 and
-// walks the positions with the weights times value scale from a per-warp
-// table.  CUDA cores: a few multiply-adds per byte; codes become floats by
-// placing them in the mantissa of 1.0f (f = 1 + c 2^-bits, exact), which
-// keeps the integer-to-float unit out of the inner loops:
+// Per tile, the scores of the positions in pages are one tensor-core
+// contraction per key group: with the key scale and zero constant over the
+// group's kg positions of a channel,
+//     q . k_t = sum_j (q_j scale_j) c_{t,j} + sum_j q_j zero_j,
+// so q'_j = q_j scale_j (fp16 high and low parts, the query normalized per
+// head by a power of two) forms the A rows (head, part) of m16n8k16 fp16
+// products, the codes (exact in fp16) the B columns, channels the k
+// dimension; the even and odd positions of a 16-position block are two
+// n8 tiles, so that one byte of a channel run feeds both.  The second sum
+// is a warp reduction per group.  Scores go to a per-warp table.  For the
+// weighted values lane l owns channels 4l .. 4l+3 and walks the positions
+// with the weights times value scale from a per-warp table, on CUDA cores:
+// codes become floats by placing them in the mantissa of 1.0f
+// (f = 1 + c 2^-bits, exact):
 //     scale*c + zero = (scale 2^bits) f + (zero - scale 2^bits).
 // Ring positions (at or above Q) are read as bf16 rows from global memory,
-// prefetched into L2 when the tile's copies are issued.
+// prefetched into L2 when the tile's copies are issued; their scores are
+// formed on CUDA cores by the lanes that own them (positions 2l, 2l+1).
 #include <cuda_fp16.h>
 
 #include "kvq_internal.cuh"
@@ -44,7 +51,9 @@ namespace {
 constexpr int PD = 128;
 constexpr int PT = 64;              // positions per page (one tile)
 constexpr int GMAX = 8;             // query heads per kv-head (kernels for up to 4 and up to 8)
-constexpr int NWMAX = 8;            // warps per CTA at most
+// warps per CTA at most: as many as the registers of the build allow
+// (about 160 per thread for four heads, 200 for eight)
+__host__ __device__ constexpr int nw_max(int nh) { return nh == 4 ? 12 : 8; }
 constexpr int SMEM_MAX = 227 * 1024;
 constexpr unsigned FULLM = 0xffffffffu;
 
@@ -52,8 +61,9 @@ constexpr unsigned FULLM = 0xffffffffu;
 struct PcGeom {
     int KC, KM, VC, VM;     // the four raw blocks of a (page, kv-head)
     int SLOT;               // KC + KM + VC + VM
-    int MT;                 // key (scale', zero') table: [PT/kg][PD] float2
+    int MT;                 // key (scale, zero) table: [PT/kg][PD] float2
     int PW;                 // weight table: [PT][nvg][NH] float
+    int SS;                 // score table: [PT][NH] float
     int WAREA;              // per warp: two slots, the tables
     int OFF_PAGES, OFF_AREAS;
     int NW, bytes;
@@ -71,11 +81,12 @@ PcGeom pc_geometry(const Params& p, int max_len, int nh) {
     g.SLOT = g.KC + g.KM + g.VC + g.VM;
     g.MT = nkg * PD * 8;
     g.PW = PT * p.nvg * nh * 4;
-    g.WAREA = round_up(2 * g.SLOT + g.MT + g.PW, 128);
-    g.OFF_PAGES = PD * nh * 4;
+    g.SS = PT * nh * 4;
+    g.WAREA = round_up(2 * g.SLOT + g.MT + g.PW + g.SS, 128);
+    g.OFF_PAGES = PD * nh * 4 + 2 * nh * 4;
     g.OFF_AREAS = round_up(g.OFF_PAGES + 4 * (max_len / PT + 1), 128);
     const int nw = (SMEM_MAX - g.OFF_AREAS) / g.WAREA;
-    g.NW = nw < NWMAX ? nw : NWMAX;
+    g.NW = nw < nw_max(nh) ? nw : nw_max(nh);
     g.bytes = g.OFF_AREAS + (g.NW > 0 ? g.NW : 0) * g.WAREA;
     return g;
 }
@@ -106,14 +117,6 @@ __device__ __forceinline__ float code_f(uint32_t x, int sh) {
     const uint32_t y = sh <= top ? (x << (top - sh)) : (x >> (sh - top));
     return __uint_as_float((y & mask) | 0x3F800000u);
 }
-// the same for a shift known at run time only, sh <= 23 - BITS
-template <int BITS>
-__device__ __forceinline__ float code_f_low(uint32_t x, int sh) {
-    constexpr int top = 23 - BITS;
-    constexpr uint32_t mask = ((1u << BITS) - 1u) << top;
-    return __uint_as_float(((x << (top - sh)) & mask) | 0x3F800000u);
-}
-
 // the codes of positions 16 qt .. 16 qt + 15 of channel j's run (runs of
 // BITS*8 bytes, chunk-major above 16 bytes: [chunk][d][min(16, run)]), as
 // 16*BITS bits
@@ -133,6 +136,29 @@ __device__ __forceinline__ void run_quarter(const uint8_t* base, int j, int qt, 
         const uint4 u = *reinterpret_cast<const uint4*>(a);
         w[0] = u.x, w[1] = u.y, w[2] = u.z, w[3] = u.w;
     }
+}
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t h2bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+// part `limb` (0: the fp16 rounding, 1: the fp16 rounding of the rest) of the pair (x, y)
+__device__ __forceinline__ uint32_t f16_part(float x, float y, int limb) {
+    const __half2 hi = __floats2half2_rn(x, y);
+    const float2 f = __half22float2(hi);
+    const __half2 lo = __floats2half2_rn(x - f.x, y - f.y);
+    return limb ? h2bits(lo) : h2bits(hi);
+}
+// two codes (one per 16-bit half of y, BITS wide at bit 0) as an fp16 pair
+template <int BITS>
+__device__ __forceinline__ uint32_t codes_f16(uint32_t y) {
+    constexpr uint32_t m = ((1u << BITS) - 1u) * 0x00010001u;
+    const uint32_t biased = (y & m) | 0x64006400u;              // 1024 + c, exact
+    const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&biased), __floats2half2_rn(1024.0f, 1024.0f));
+    return h2bits(r);
 }
 
 template <int NH>
@@ -157,7 +183,7 @@ __device__ __forceinline__ float warp_max(float v) {
 __device__ __forceinline__ float ex2(float x) { return exp2f(x); }
 
 template <int KB, int VB, int NH>
-__global__ void __launch_bounds__(NWMAX * 32, 1) decode_pc_kernel(const Params p, const void* __restrict__ qv,
+__global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Params p, const void* __restrict__ qv,
                                                                   int q_bf16, const int32_t* __restrict__ lens,
                                                                   int max_len, float sl2, float* __restrict__ out,
                                                                   float* __restrict__ lse, const PcGeom geo) {
@@ -196,10 +222,29 @@ __global__ void __launch_bounds__(NWMAX * 32, 1) decode_pc_kernel(const Params p
         pages[i] = pg >= p.num_pages ? -1 : pg;
     }
     __syncthreads();
+    // per head a power of two that brings max_j |q_j| into [1/2, 1) (fp16 range
+    // for q_j times a key scale), and its inverse
+    float* hnorm = reinterpret_cast<float*>(smem_raw + PD * NH * 4);   // [NH] factor, [NH] inverse
+    if (w == 0) {
+#pragma unroll
+        for (int r = 0; r < NH; ++r) {
+            float a = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) a = fmaxf(a, fabsf(qf[(4 * lane + c) * NH + r]));
+            a = warp_max(a);
+            const int eb = min(252, max(1, int(__float_as_uint(a) >> 23)));
+            if (lane == 0) {
+                hnorm[r] = a > 0.0f ? __uint_as_float(uint32_t(253 - eb) << 23) : 1.0f;      // 2^(126 - eb)
+                hnorm[NH + r] = a > 0.0f ? __uint_as_float(uint32_t(eb + 1) << 23) : 1.0f;   // 2^(eb - 126)
+            }
+        }
+    }
+    __syncthreads();
 
     uint8_t* area = areas + size_t(w) * geo.WAREA;
     float2* mt = reinterpret_cast<float2*>(area + 2 * geo.SLOT);
     float* pw = reinterpret_cast<float*>(area + 2 * geo.SLOT + geo.MT);
+    float* ss = reinterpret_cast<float*>(area + 2 * geo.SLOT + geo.MT + geo.PW);   // [PT][NH] scores
     const uint16_t* kwin = reinterpret_cast<const uint16_t*>(p.k_win) + prow * size_t(R) * PD;
     const uint16_t* vwin = reinterpret_cast<const uint16_t*>(p.v_win) + prow * size_t(R) * PD;
 
@@ -248,11 +293,15 @@ __global__ void __launch_bounds__(NWMAX * 32, 1) decode_pc_kernel(const Params p
     const int j0 = 4 * lane;                        // value channels of this lane
     const int gv = j0 / p.vg;                       // their value group
 
-    // where the codes of positions tA, tB of a channel run sit: byte offset
-    // (plus channel * cw) and bit of the first code
-    constexpr int kchan = PT * KB / 8, kcw = kchan < 16 ? kchan : 16;
-    const int kbit = tA * KB, kbyte = kbit >> 3;
-    const int koff = (kbyte / kcw) * (PD * kcw) + (kbyte % kcw), ksh = kbit & 7;
+    constexpr int kchan = PT * KB / 8, kcw = kchan < 16 ? kchan : 16;   // key run, chunk bytes
+    const int g8 = lane >> 2, tig = lane & 3;       // fragment row group, thread in group
+    const int r0 = g8 >> 1, limb = g8 & 1;          // A row g8: head r0, part limb (row g8 + 8: head r0 + 4)
+    float f0 = 1.0f, f1 = 1.0f, i0 = 1.0f, i1 = 1.0f;   // normalization of heads r0 (and r0 + 4)
+#pragma unroll
+    for (int r = 0; r < NH; ++r) {
+        if (r == r0) f0 = hnorm[r], i0 = hnorm[NH + r];
+        if (NH == 8 && r == r0 + 4) f1 = hnorm[r], i1 = hnorm[NH + r];
+    }
 
     int slot = 0;
     issue(w, 0);
@@ -271,12 +320,88 @@ __global__ void __launch_bounds__(NWMAX * 32, 1) decode_pc_kernel(const Params p
         const uint8_t* vc = raw + geo.KC + geo.KM;
         const uint32_t* vm = reinterpret_cast<const uint32_t*>(raw + geo.KC + geo.KM + geo.VC);
 
-        // ---- key groups of the tile: (scale 2^KB, zero - scale 2^KB) per channel
+        // ---- key groups of the tile: (scale, zero) per channel
         if (nq > 0) {
             for (int e = lane; e < (nq / kg) * PD; e += 32) {
                 const uint32_t m = km[e];
-                const float s = hbits(m & 0xffffu) * float(1 << KB);
-                mt[e] = make_float2(s, hbits(m >> 16) - s);
+                mt[e] = make_float2(hbits(m & 0xffffu), hbits(m >> 16));
+            }
+        }
+        __syncwarp();
+
+        // ---- scores of the positions in the page, per key group (tensor cores)
+        for (int gi = 0; gi < nq / kg; ++gi) {
+            const float2* mg = mt + gi * PD;
+            // the zero-point sum of every head: channels 4l .. 4l+3, then the warp
+            float bz[NH];
+#pragma unroll
+            for (int r = 0; r < NH; ++r) bz[r] = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float z = mg[4 * lane + c].y;
+                float qq[NH];
+                ld_heads<NH>(qf + (4 * lane + c) * NH, qq);
+#pragma unroll
+                for (int r = 0; r < NH; ++r) bz[r] = fmaf(qq[r], z, bz[r]);
+            }
+            float b0 = 0.0f, b1 = 0.0f;
+#pragma unroll
+            for (int r = 0; r < NH; ++r) {
+                const float t = warp_sum(bz[r]);
+                if (r == r0) b0 = t;
+                if (NH == 8 && r == r0 + 4) b1 = t;
+            }
+            // A fragments: rows (head, part) of q_j 2^-e scale_j, channels 16 ks + {2tig, +1, +8, +9}
+            uint32_t af[8][4];
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int c = 16 * ks + 2 * tig + 8 * hf;
+                    const float s0 = mg[c].x, s1 = mg[c + 1].x;
+                    af[ks][2 * hf] = f16_part(qf[c * NH + r0] * f0 * s0, qf[(c + 1) * NH + r0] * f0 * s1, limb);
+                    af[ks][2 * hf + 1] =
+                        NH == 8 ? f16_part(qf[c * NH + r0 + 4] * f1 * s0, qf[(c + 1) * NH + r0 + 4] * f1 * s1, limb)
+                                : 0u;
+                }
+            }
+            // 16-position blocks of the group: even and odd positions as two n8 tiles
+            for (int blk = gi * (kg / 16); blk < (gi + 1) * (kg / 16); ++blk) {
+                const int bit = (16 * blk + 2 * g8) * KB, byte = bit >> 3, sh = bit & 7;
+                const uint8_t* kb0 = kc + (byte / kcw) * (PD * kcw) + (byte % kcw);
+                float de[4] = {0.0f, 0.0f, 0.0f, 0.0f}, dd[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const int c0 = 16 * ks + 2 * tig;
+                    uint32_t x[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int c = c0 + (u & 1) + 8 * (u >> 1);
+                        if constexpr (KB == 8) x[u] = *reinterpret_cast<const uint16_t*>(kb0 + c * kcw);
+                        else x[u] = kb0[c * kcw];
+                    }
+                    const uint32_t y01 = __byte_perm(x[0], x[1], 0x5410) >> sh;
+                    const uint32_t y23 = __byte_perm(x[2], x[3], 0x5410) >> sh;
+                    const uint32_t a4[4] = {af[ks][0], af[ks][1], af[ks][2], af[ks][3]};
+                    mma_f16(de, a4, codes_f16<KB>(y01), codes_f16<KB>(y23));
+                    mma_f16(dd, a4, codes_f16<KB>(y01 >> KB), codes_f16<KB>(y23 >> KB));
+                }
+                // rows g8 and g8 ^ 1 are the two parts of one head: lanes 4 apart
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    de[i] += __shfl_xor_sync(FULLM, de[i], 4);
+                    dd[i] += __shfl_xor_sync(FULLM, dd[i], 4);
+                }
+                // lane (g8, tig) holds positions 16 blk + 4 tig + {0 (de), 1 (dd), 2 (de), 3 (dd)};
+                // the lanes of part 0 store the even ones, those of part 1 the odd ones
+                const float* d = limb ? dd : de;
+                const int t0p = 16 * blk + 4 * tig + limb;
+                ss[t0p * NH + r0] = fmaf(d[0], i0, b0);
+                ss[(t0p + 2) * NH + r0] = fmaf(d[1], i0, b0);
+                if (NH == 8) {
+                    ss[t0p * NH + r0 + 4] = fmaf(d[2], i1, b1);
+                    ss[(t0p + 2) * NH + r0 + 4] = fmaf(d[3], i1, b1);
+                }
             }
         }
         __syncwarp();
@@ -286,24 +411,8 @@ __global__ void __launch_bounds__(NWMAX * 32, 1) decode_pc_kernel(const Params p
 #pragma unroll
         for (int r = 0; r < NH; ++r) sA[r] = sB[r] = 0.0f;
         if (tA < nq) {
-            const float2* mg = mt + (tA / kg) * PD;
-            const uint8_t* kp = kc + koff;
-#pragma unroll 4
-            for (int j = 0; j < PD; ++j) {
-                uint32_t x;
-                if constexpr (KB == 8) x = *reinterpret_cast<const uint16_t*>(kp + j * kcw);
-                else x = kp[j * kcw];
-                const float fA = code_f_low<KB>(x, ksh), fB = code_f_low<KB>(x, ksh + KB);
-                const float2 sz = mg[j];
-                const float kA = fmaf(sz.x, fA, sz.y), kB = fmaf(sz.x, fB, sz.y);
-                float qq[NH];
-                ld_heads<NH>(qf + j * NH, qq);
-#pragma unroll
-                for (int r = 0; r < NH; ++r) {
-                    sA[r] = fmaf(qq[r], kA, sA[r]);
-                    sB[r] = fmaf(qq[r], kB, sB[r]);
-                }
-            }
+            ld_heads<NH>(ss + tA * NH, sA);
+            ld_heads<NH>(ss + tB * NH, sB);
         } else if (tA < nv) {
             const bool hasB = tB < nv;
             const uint16_t* ra = kwin + size_t((t0 + tA) % R) * PD;
