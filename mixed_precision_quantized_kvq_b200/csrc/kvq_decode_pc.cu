@@ -14,7 +14,7 @@
 // c_t + sum_t p_t vzero_t per value group.
 //
 // One CTA per (sequence, kv-head), all g query heads of the kv-group
-// together; its warps (up to 12) take the pair's 64-position tiles in turn (warp w:
+// together; its warps (up to 8) take the pair's 64-position tiles in turn (warp w:
 // tiles w, w + NW, ...), each warp on its own: the raw page blocks (key
 // codes, key metadata, value codes, value metadata) of its next tile are
 // copied into the warp's second slot with cp.async while it works on the
@@ -51,9 +51,9 @@ namespace {
 constexpr int PD = 128;
 constexpr int PT = 64;              // positions per page (one tile)
 constexpr int GMAX = 8;             // query heads per kv-head (kernels for up to 4 and up to 8)
-// warps per CTA at most: as many as the registers of the build allow
-// (about 160 per thread for four heads, 200 for eight)
-__host__ __device__ constexpr int nw_max(int nh) { return nh == 4 ? 12 : 8; }
+// warps per CTA at most (about 200 registers per thread)
+__host__ __device__ constexpr int nw_max(int nh) { return 8; }
+constexpr int PHROW = 36;           // words per row of the fp16 weight table (32 used; the rest spreads banks)
 constexpr int SMEM_MAX = 227 * 1024;
 constexpr unsigned FULLM = 0xffffffffu;
 
@@ -64,6 +64,7 @@ struct PcGeom {
     int MT;                 // key (scale, zero) table: [PT/kg][PD] float2
     int PW;                 // weight table: [PT][nvg][NH] float
     int SS;                 // score table: [PT][NH] float
+    int PH;                 // four heads: weight parts [nvg][8][36] fp16 pairs, zero sums [nvg][4]
     int WAREA;              // per warp: two slots, the tables
     int OFF_PAGES, OFF_AREAS;
     int NW, bytes;
@@ -82,7 +83,8 @@ PcGeom pc_geometry(const Params& p, int max_len, int nh) {
     g.MT = nkg * PD * 8;
     g.PW = PT * p.nvg * nh * 4;
     g.SS = PT * nh * 4;
-    g.WAREA = round_up(2 * g.SLOT + g.MT + g.PW + g.SS, 128);
+    g.PH = nh == 4 ? p.nvg * (8 * PHROW + 4) * 4 : 0;
+    g.WAREA = round_up(2 * g.SLOT + g.MT + g.PW + g.SS + g.PH, 128);
     g.OFF_PAGES = PD * nh * 4 + 2 * nh * 4;
     g.OFF_AREAS = round_up(g.OFF_PAGES + 4 * (max_len / PT + 1), 128);
     const int nw = (SMEM_MAX - g.OFF_AREAS) / g.WAREA;
@@ -159,6 +161,37 @@ __device__ __forceinline__ uint32_t codes_f16(uint32_t y) {
     const uint32_t biased = (y & m) | 0x64006400u;              // 1024 + c, exact
     const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&biased), __floats2half2_rn(1024.0f, 1024.0f));
     return h2bits(r);
+}
+
+// the codes of positions 2 tig + 8 hf and the next one (a pair never
+// straddles a word) of a k-step's words, as an fp16 pair, the first in the
+// low half; the word is chosen without indexing the array at run time
+template <int BITS, int HF>
+__device__ __forceinline__ uint32_t vpair_f16(const uint32_t (&w)[4], int tig) {
+    const int pos = (2 * tig + 8 * HF) * BITS;
+    uint32_t x;
+    if constexpr (BITS == 8) x = (tig >> 1) ? w[2 * HF + 1] : w[2 * HF];
+    else x = w[(8 * HF * BITS) >> 5];
+    x >>= pos & 31;
+    return codes_f16<BITS>((x & ((1u << BITS) - 1u)) | ((x << (16 - BITS)) & (((1u << BITS) - 1u) << 16)));
+}
+// the codes of positions 16 ks .. 16 ks + 15 of channel j's value run (2*BITS bytes)
+template <int BITS>
+__device__ __forceinline__ void vrun_kstep(const uint8_t* base, int j, int ks, uint32_t (&w)[4]) {
+    constexpr int chan = PT * BITS / 8, cw = chan < 16 ? chan : 16;
+    const int byte = 2 * BITS * ks;
+    const uint8_t* a = base + (byte / cw) * (PD * cw) + j * cw + (byte % cw);
+    if constexpr (BITS == 1) {
+        w[0] = *reinterpret_cast<const uint16_t*>(a);
+    } else if constexpr (BITS == 2) {
+        w[0] = *reinterpret_cast<const uint32_t*>(a);
+    } else if constexpr (BITS == 4) {
+        const uint2 u = *reinterpret_cast<const uint2*>(a);
+        w[0] = u.x, w[1] = u.y;
+    } else {
+        const uint4 u = *reinterpret_cast<const uint4*>(a);
+        w[0] = u.x, w[1] = u.y, w[2] = u.z, w[3] = u.w;
+    }
 }
 
 template <int NH>
@@ -245,6 +278,12 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
     float2* mt = reinterpret_cast<float2*>(area + 2 * geo.SLOT);
     float* pw = reinterpret_cast<float*>(area + 2 * geo.SLOT + geo.MT);
     float* ss = reinterpret_cast<float*>(area + 2 * geo.SLOT + geo.MT + geo.PW);   // [PT][NH] scores
+    uint32_t* ph = reinterpret_cast<uint32_t*>(area + 2 * geo.SLOT + geo.MT + geo.PW + geo.SS);
+    float* crr = reinterpret_cast<float*>(ph + nvg * 8 * PHROW);                    // [nvg][4]
+    // four heads: the weighted values of the positions in pages on tensor cores
+    // (rows: channels, k: positions, columns: (head, part) of the weights)
+    constexpr bool VMMA = NH == 4;
+    const int lvg = __ffs(p.vg) - 1;                // value groups of 16 .. 128 channels
     const uint16_t* kwin = reinterpret_cast<const uint16_t*>(p.k_win) + prow * size_t(R) * PD;
     const uint16_t* vwin = reinterpret_cast<const uint16_t*>(p.v_win) + prow * size_t(R) * PD;
 
@@ -289,6 +328,10 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
         l_run[r] = 0.0f;
         o[r][0] = o[r][1] = o[r][2] = o[r][3] = 0.0f;
     }
+    // four heads: channels 16 mt + g8 (+ 8) of head tig, high and low weight parts
+    float ov[VMMA ? 8 : 1][4];
+#pragma unroll
+    for (int mt = 0; mt < (VMMA ? 8 : 1); ++mt) ov[mt][0] = ov[mt][1] = ov[mt][2] = ov[mt][3] = 0.0f;
     const int tA = 2 * lane, tB = tA + 1;           // score positions of this lane (in the tile)
     const int j0 = 4 * lane;                        // value channels of this lane
     const int gv = j0 / p.vg;                       // their value group
@@ -452,10 +495,22 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
 #pragma unroll
             for (int c = 0; c < 4; ++c) o[r][c] *= alpha[r];
         }
+        if constexpr (VMMA) {
+            float at = alpha[0];
+#pragma unroll
+            for (int r = 1; r < NH; ++r) at = tig == r ? alpha[r] : at;
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) ov[mt][i] *= at;
+        }
 
-        // ---- weight table [t][value group][head]: quantized positions p*scale*2^VB,
-        // ring positions p; per value group the zero points and the mantissa offsets
-        // of the quantized positions: sum_t p (zero - scale 2^VB)
+        // ---- weight tables.  Eight heads: [t][value group][head] on CUDA cores,
+        // positions in pages p*scale*2^VB, ring positions p; per value group the
+        // zero points and the mantissa offsets: sum_t p (zero - scale 2^VB).
+        // Four heads: positions in pages as fp16 parts of p*scale, [group][(head,
+        // part)][t/2] (lane l writes word l: positions 2l, 2l+1), and the zero
+        // sums sum_t p zero per group; ring positions p in the float table.
         float corr[NH];
 #pragma unroll
         for (int r = 0; r < NH; ++r) corr[r] = 0.0f;
@@ -463,11 +518,22 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
             float z[NH];
 #pragma unroll
             for (int r = 0; r < NH; ++r) z[r] = 0.0f;
+            if (VMMA && tA < nq) {
+                const uint32_t mA = vm[tA * nvg + gg], mB = vm[tB * nvg + gg];
+                const float sa = hbits(mA & 0xffffu), sb = hbits(mB & 0xffffu);
+                const float za = hbits(mA >> 16), zb = hbits(mB >> 16);
+#pragma unroll
+                for (int r = 0; r < NH; ++r) {
+                    ph[(gg * 8 + 2 * r) * PHROW + lane] = f16_part(pA[r] * sa, pB[r] * sb, 0);
+                    ph[(gg * 8 + 2 * r + 1) * PHROW + lane] = f16_part(pA[r] * sa, pB[r] * sb, 1);
+                    z[r] = fmaf(pA[r], za, fmaf(pB[r], zb, z[r]));
+                }
+            }
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 const int t = tA + half;
                 const float* pp = half ? pB : pA;
-                if (t >= nv) continue;
+                if (t >= nv || (VMMA && t < nq)) continue;
                 float wt[NH];
                 if (t < nq) {
                     const uint32_t m = vm[t * nvg + gg];
@@ -491,26 +557,53 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
                 for (int r = 0; r < NH; ++r) {
                     const float zs = warp_sum(z[r]);
                     if (gg == gv) corr[r] = zs;
+                    if (VMMA && lane == 0) crr[gg * 4 + r] = zs;
                 }
             }
         }
-        __syncwarp();                               // the weight table is complete
+        __syncwarp();                               // the weight tables are complete
 
-        // ---- o += sum_t w_t v_t over the tile: channels j0 .. j0+3
-        for (int qt = 0; qt < nq / 16; ++qt) {
-            uint32_t cw4[4][4];
+        if constexpr (VMMA) {
+            // ---- o += sum_t w_t v_t, positions in pages: 8 channel tiles x nq/16 k-steps
+            for (int ks = 0; ks < nq / 16; ++ks) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) run_quarter<VB>(vc, j0 + c, qt, cw4[c]);
+                for (int mt = 0; mt < 8; ++mt) {
+                    const int ja = 16 * mt + g8, gvm = (16 * mt) >> lvg;
+                    uint32_t wa[4], wb[4];
+                    vrun_kstep<VB>(vc, ja, ks, wa);
+                    vrun_kstep<VB>(vc, ja + 8, ks, wb);
+                    const uint32_t a4[4] = {vpair_f16<VB, 0>(wa, tig), vpair_f16<VB, 0>(wb, tig),
+                                            vpair_f16<VB, 1>(wa, tig), vpair_f16<VB, 1>(wb, tig)};
+                    const uint32_t* prow = ph + (gvm * 8 + g8) * PHROW + 8 * ks + tig;
+                    mma_f16(ov[mt], a4, prow[0], prow[4]);
+                }
+            }
+            if (nq > 0) {
+                // zero points of the positions in pages, once per (channel, head) in the high part
 #pragma unroll
-            for (int tt = 0; tt < 16; ++tt) {
-                float pq[NH];
-                ld_heads<NH>(pw + ((16 * qt + tt) * nvg + gv) * NH, pq);
-                const int bit = tt * VB;
+                for (int mt = 0; mt < 8; ++mt) {
+                    const float zc = crr[((16 * mt) >> lvg) * 4 + tig];
+                    ov[mt][0] += zc;
+                    ov[mt][2] += zc;
+                }
+            }
+        } else {
+            // ---- o += sum_t w_t v_t over the tile: channels j0 .. j0+3
+            for (int qt = 0; qt < nq / 16; ++qt) {
+                uint32_t cw4[4][4];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float f = code_f<VB>(cw4[c][bit >> 5], bit & 31);
+                for (int c = 0; c < 4; ++c) run_quarter<VB>(vc, j0 + c, qt, cw4[c]);
 #pragma unroll
-                    for (int r = 0; r < NH; ++r) o[r][c] = fmaf(pq[r], f, o[r][c]);
+                for (int tt = 0; tt < 16; ++tt) {
+                    float pq[NH];
+                    ld_heads<NH>(pw + ((16 * qt + tt) * nvg + gv) * NH, pq);
+                    const int bit = tt * VB;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const float f = code_f<VB>(cw4[c][bit >> 5], bit & 31);
+#pragma unroll
+                        for (int r = 0; r < NH; ++r) o[r][c] = fmaf(pq[r], f, o[r][c]);
+                    }
                 }
             }
         }
@@ -525,10 +618,12 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
 #pragma unroll
                 for (int r = 0; r < NH; ++r) o[r][c] = fmaf(pq[r], x[c], o[r][c]);
         }
+        if constexpr (!VMMA) {
 #pragma unroll
-        for (int r = 0; r < NH; ++r)
+            for (int r = 0; r < NH; ++r)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) o[r][c] += corr[r];
+                for (int c = 0; c < 4; ++c) o[r][c] += corr[r];
+        }
         __syncwarp();                               // slot, tables free for the next tiles
         slot ^= 1;
     }
@@ -545,6 +640,17 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
         if (lane == 0) {
             part[(w * NH + r) * PS + PD] = m_run[r];
             part[(w * NH + r) * PS + PD + 1] = l_run[r];
+        }
+    }
+    if constexpr (VMMA) {
+        __syncwarp();                               // the CUDA-core part of the warp's rows first
+        if (tig < g) {
+            float* prt = part + (w * NH + tig) * PS;
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                prt[16 * mt + g8] += ov[mt][0] + ov[mt][1];
+                prt[16 * mt + g8 + 8] += ov[mt][2] + ov[mt][3];
+            }
         }
     }
     __syncthreads();
