@@ -456,7 +456,7 @@ def run_ours(args):
     # kernel, or a split kernel and its combine
     path = kvq.kvq_get_decode_path(lay)
     if w.k_per_channel:
-        launches_per_step, decode_kernel = 3, "kvq_decode_attention (chunked-prefill kernel, one query per sequence)"
+        launches_per_step, decode_kernel = 3, "kvq_decode_attention (per-channel decode kernel: warp-independent tiles, tensor-core scores and weighted values)"
     elif path == kvq.DECODE_TENSOR_CORES:
         launches_per_step, decode_kernel = 2, "kvq_decode_attention (persistent tensor-core kernel, merge fused)"
     else:
