@@ -182,9 +182,11 @@ size_t kvq_decode_workspace_bytes(const kvq_layout* layout, int batch, int max_l
 int kvq_set_decode_path(int path);
 
 /* Decode kernel family the current setting picks for this layout (at batch
- * 1): 2 = persistent tensor-core kernel, 3 = two-phase tcgen05 kernel,
- * 1 = CUDA cores (always for k_per_channel layouts), or a negative KVQ_ERR_*
- * code. */
+ * 1, short sequences): 2 = persistent tensor-core kernel, 3 = two-phase
+ * tcgen05 kernel, 1 = CUDA cores, 4 = the per-channel decode kernel (the
+ * k_per_channel layouts it takes: head_dim 128, unrotated; other
+ * k_per_channel layouts report 1), or a negative KVQ_ERR_* code.  The
+ * setting of kvq_set_decode_path does not apply to k_per_channel layouts. */
 int kvq_get_decode_path(const kvq_layout* layout);
 
 /* Decode diagnostics of the current device, counted by the decode kernels
@@ -236,8 +238,9 @@ int kvq_quantize_append(const kvq_layout* layout, const kvq_cache* cache,
  *           once per allocation, not per call.  Calls that overlap on the GPU
  *           need separate workspaces.
  *           Not read for k_per_channel layouts (may be NULL): those run the
- *           chunked-prefill kernel with one query per sequence, one CTA per
- *           (sequence, kv-head), no split-K.
+ *           per-channel decode kernel, one CTA per (sequence, kv-head) whose
+ *           warps merge their parts in shared memory (head_dim 64 layouts:
+ *           the chunked-prefill kernel with one query per sequence).
  * Returns KVQ_ERR_UNSUPPORTED for batch or num_kv_heads above 65535. */
 int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache,
                          const void* q, int q_dtype, const int32_t* lens, int max_len,

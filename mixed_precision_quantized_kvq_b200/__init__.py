@@ -344,6 +344,7 @@ def kvq_rotate_keys(layout: Layout, k: torch.Tensor, out: torch.Tensor, stream=N
 
 
 DECODE_AUTO, DECODE_CUDA_CORES, DECODE_TENSOR_CORES, DECODE_TCGEN05 = 0, 1, 2, 3
+DECODE_PER_CHANNEL = 4   # reported by kvq_get_decode_path for key groups along positions
 
 
 def kvq_set_decode_path(path: int) -> None:

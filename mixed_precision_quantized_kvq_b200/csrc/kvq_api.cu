@@ -172,8 +172,8 @@ int kvq_set_decode_path(int path) {
 int kvq_get_decode_path(const kvq_layout* layout) {
     int rc = check_layout(layout);
     if (rc) return rc;
-    if (layout->k_per_channel) return 1;
     Params p = make_params(layout, nullptr);
+    if (layout->k_per_channel) return kvq::decode_pc_supported(p, 1) ? 4 : 1;
     const int path = kvq::g_decode_path;
     if (path == 1) return 1;
     if (path == 3) return kvq::tc_supported(p) ? 3 : 1;

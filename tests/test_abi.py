@@ -146,13 +146,14 @@ def test_workspace_size_monotone():
                                              (2, 4, 16, 64, 64, 8), (1, 1, 16, 32, 64, 3)])
 def test_per_channel_sizes_agree_with_oracle(kb, vb, kg, vg, d, w):
     """Key groups along positions: page bytes as the oracle's layout, a ring
-    of window + k_group - 1 slots, no decode workspace, CUDA-core decode."""
+    of window + k_group - 1 slots, no decode workspace; head_dim 128 decodes
+    with the per-channel kernel, head_dim 64 on CUDA cores."""
     lay = L(head_dim=d, k_bits=kb, v_bits=vb, k_group=kg, v_group=vg, window=w, k_per_channel=True)
     olay = oracle.Layout(d, 32, 8, kb, vb, kg, vg, 64, w, k_per_channel=True)
     assert kvq.kvq_page_bytes(lay) == oracle.page_bytes(olay)
     assert kvq.kvq_window_bytes(lay, 16) == 16 * 8 * (w + kg - 1) * d * 2 == 16 * 8 * olay.ring_slots * d * 2
     assert kvq.kvq_decode_workspace_bytes(lay, 16, 4096) == 0
-    assert kvq.kvq_get_decode_path(lay) == kvq.DECODE_CUDA_CORES
+    assert kvq.kvq_get_decode_path(lay) == (kvq.DECODE_PER_CHANNEL if d == 128 else kvq.DECODE_CUDA_CORES)
 
 
 @pytest.mark.parametrize("kw,code", [
