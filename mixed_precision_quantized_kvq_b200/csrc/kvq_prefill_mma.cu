@@ -44,9 +44,9 @@ constexpr int PTHREADS = 256;        // 8 warps x 16 rows
 constexpr unsigned kFull = 0xffffffffu;
 
 // shared memory: keys hi/lo [64 pos][128 ch] bf16, values hi/lo [128 ch][64 pos]
-// bf16, value metadata [64][nvg] words
+// bf16, value (scale 2^vb, zero - scale 2^vb) [64][nvg] float pairs
 constexpr int KBYTES = PTILE * PD * 2;    // 16 KB per array
-constexpr size_t prefill_mma_smem(int nvg) { return 4 * size_t(KBYTES) + size_t(PTILE) * nvg * 4; }
+constexpr size_t prefill_mma_smem(int nvg) { return 4 * size_t(KBYTES) + size_t(PTILE) * nvg * 8; }
 
 __device__ __forceinline__ float bits_bf16(uint32_t b) { return __uint_as_float(b << 16); }
 __device__ __forceinline__ float bits_half(uint32_t b) {
@@ -54,20 +54,22 @@ __device__ __forceinline__ float bits_half(uint32_t b) {
     r.x = uint16_t(b);
     return __half2float(__half(r));
 }
-// x as bf16 (hi, lo): hi = bf16(x), lo = bf16(x - hi)
-__device__ __forceinline__ void split_bf16(float x, uint32_t& hi, uint32_t& lo) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    const __nv_bfloat16 l = __float2bfloat16_rn(x - __bfloat162float(h));
-    hi = __bfloat16_as_ushort(h);
-    lo = __bfloat16_as_ushort(l);
-}
-// two values (first in the low half) as packed bf16 hi and lo words
+// two values (first in the low half) as packed bf16 hi and lo words:
+// hi = bf16(x), lo = bf16(x - hi), two values per conversion
 __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-    uint32_t h0, l0, h1, l1;
-    split_bf16(x0, h0, l0);
-    split_bf16(x1, h1, l1);
-    hi = h0 | (h1 << 16);
-    lo = l0 | (l1 << 16);
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xffff0000u));
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+// code c (BITS wide) at bit sh of x as the float 1 + c 2^-BITS (the code in the
+// top of the mantissa of 1.0f): scale*c + zero = (scale 2^BITS) f + (zero - scale 2^BITS)
+template <int BITS>
+__device__ __forceinline__ float code_f(uint32_t x, int sh) {
+    constexpr int top = 23 - BITS;
+    constexpr uint32_t mask = ((1u << BITS) - 1u) << top;
+    const uint32_t y = sh <= top ? (x << (top - sh)) : (x >> (sh - top));
+    return __uint_as_float((y & mask) | 0x3F800000u);
 }
 // byte offset of 16-byte chunk c of row r in a [rows][chunks_per_row] array swizzled by row
 __device__ __forceinline__ uint32_t swz(int r, int c, int chunks_per_row) {
@@ -78,7 +80,7 @@ template <int KB, int VB>
 __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill::View v) {
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t sKh = smem_u32(smem), sKl = sKh + KBYTES, sVh = sKl + KBYTES, sVl = sVh + KBYTES;
-    uint32_t* sVm = reinterpret_cast<uint32_t*>(smem + 4 * KBYTES);   // [64][nvg]
+    float2* sVf = reinterpret_cast<float2*>(smem + 4 * KBYTES);       // [64][nvg]
     const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g8 = lane >> 2, tig = lane & 3;
     const int g = v.g, QT = PROWS / g, R = QT * g;
@@ -139,10 +141,13 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
             pg = lp < v.max_pages ? v.page_table[size_t(b) * v.max_pages + lp] : -1;
             if (pg >= v.num_pages) pg = -1;
         }
-        // value metadata of the tile's paged positions
+        // value metadata of the tile's paged positions, as (scale 2^VB, zero - scale 2^VB)
         if (paged_tile && pg >= 0)
-            for (int e = tid; e < PTILE * v.nvg; e += PTHREADS)
-                sVm[e] = v.v_meta[((size_t(pg) * v.hkv + blk) * PTILE + e / v.nvg) * v.nvg + e % v.nvg];
+            for (int e = tid; e < PTILE * v.nvg; e += PTHREADS) {
+                const uint32_t m = v.v_meta[((size_t(pg) * v.hkv + blk) * PTILE + e / v.nvg) * v.nvg + e % v.nvg];
+                const float sc = bits_half(m & 0xffffu) * float(1 << VB);
+                sVf[e] = make_float2(sc, bits_half(m >> 16) - sc);
+            }
         __syncthreads();
         // ---- keys: thread = (position, key group of 32 channels), 8 channels at a time
         {
@@ -161,8 +166,8 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
                                                                 byte % v.kch);
                 }
                 const uint32_t m = v.k_meta[((size_t(pg) * v.hkv + blk) * PTILE + t) * v.nkg + grp];
-                sc = bits_half(m & 0xffffu);
-                zr = bits_half(m >> 16);
+                sc = bits_half(m & 0xffffu) * float(1 << KB);
+                zr = bits_half(m >> 16) - sc;
             } else if (kind == 2) {
                 wrow = v.k_win + ((size_t(b) * v.hkv + blk) * v.W + size_t(pos % v.W)) * PD + 32 * grp;
             }
@@ -181,8 +186,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
 #pragma unroll
                             for (int e = 0; e < 2; ++e) {
                                 const int j = 8 * cc + 2 * k + e;
-                                const uint32_t c = (wd[(j * KB) >> 5] >> ((j * KB) & 31)) & ((1u << KB) - 1u);
-                                x2[e] = fmaf(float(c), sc, zr);
+                                x2[e] = fmaf(code_f<KB>(wd[(j * KB) >> 5], (j * KB) & 31), sc, zr);
                             }
                         }
                         split2(x2[0], x2[1], hi[k], lo[k]);
@@ -199,7 +203,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
         }
         // ---- values: thread = (channel, half of the tile's positions), 8 positions at a time
         {
-            const int ch = tid >> 1, half = tid & 1;
+            const int ch = tid >> 1, half = tid & 1, gvc = ch / v.vg;
             uint32_t wd[VB];
             if (pg >= 0) {
                 const uint8_t* vc = v.v_codes + (size_t(pg) * v.hkv + blk) * size_t(PD) * v.vchan_bytes;
@@ -224,9 +228,8 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
                         if (pos <= p_max) {
                             if (pos < Lq) {
                                 if (pg >= 0) {
-                                    const uint32_t c = (wd[(i * VB) >> 5] >> ((i * VB) & 31)) & ((1u << VB) - 1u);
-                                    const uint32_t m = sVm[t * v.nvg + ch / v.vg];
-                                    xv = fmaf(float(c), bits_half(m & 0xffffu), bits_half(m >> 16));
+                                    const float2 sz = sVf[t * v.nvg + gvc];
+                                    xv = fmaf(code_f<VB>(wd[(i * VB) >> 5], (i * VB) & 31), sz.x, sz.y);
                                 }
                             } else {
                                 xv = bits_bf16(vw[((size_t(b) * v.hkv + blk) * v.W + size_t(pos % v.W)) * PD + ch]);
