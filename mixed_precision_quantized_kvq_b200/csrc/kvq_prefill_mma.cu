@@ -44,9 +44,21 @@ constexpr int PTHREADS = 256;        // 8 warps x 16 rows
 constexpr unsigned kFull = 0xffffffffu;
 
 // shared memory: keys hi/lo [64 pos][128 ch] bf16, values hi/lo [128 ch][64 pos]
-// bf16, value (scale 2^vb, zero - scale 2^vb) [64][nvg] float pairs
+// bf16, value (scale 2^vb, zero - scale 2^vb) [64][nvg] float pairs, and two
+// stages of a page's raw blocks (key codes, key metadata, value codes, value
+// metadata), the next tile's copied while the current one is worked on
 constexpr int KBYTES = PTILE * PD * 2;    // 16 KB per array
-constexpr size_t prefill_mma_smem(int nvg) { return 4 * size_t(KBYTES) + size_t(PTILE) * nvg * 8; }
+constexpr int NVG_MAX = 8;                // value groups of 16 channels or more
+__host__ __device__ constexpr int raw_bytes(int kb, int vb, int nvg) {
+    return PTILE * PD * kb / 8 + PTILE * (PD / 32) * 4 + PD * PTILE * vb / 8 + PTILE * nvg * 4;
+}
+constexpr size_t prefill_mma_smem(int kb, int vb, int nvg) {
+    return 4 * size_t(KBYTES) + size_t(PTILE) * nvg * 8 + 2 * size_t(raw_bytes(kb, vb, nvg));
+}
+
+__device__ __forceinline__ void cpa16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
 
 __device__ __forceinline__ float bits_bf16(uint32_t b) { return __uint_as_float(b << 16); }
 __device__ __forceinline__ float bits_half(uint32_t b) {
@@ -81,6 +93,10 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t sKh = smem_u32(smem), sKl = sKh + KBYTES, sVh = sKl + KBYTES, sVl = sVh + KBYTES;
     float2* sVf = reinterpret_cast<float2*>(smem + 4 * KBYTES);       // [64][nvg]
+    // raw page blocks of a tile: [stage][key codes | key metadata | value codes | value metadata]
+    const int KCB = PTILE * PD * KB / 8, KMB = PTILE * (PD / 32) * 4, VCB = PD * PTILE * VB / 8;
+    const int RAWB = raw_bytes(KB, VB, v.nvg);
+    uint8_t* raw0 = smem + 4 * KBYTES + size_t(PTILE) * v.nvg * 8;
     const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g8 = lane >> 2, tig = lane & 3;
     const int g = v.g, QT = PROWS / g, R = QT * g;
@@ -132,19 +148,42 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
     const int warp_pmax = max(p_lo, p_hi);                 // newest position this lane's rows see
 
     const size_t blk = size_t(h);                          // kv-head index inside a page block
-    for (int t0 = 0; t0 <= p_max; t0 += PTILE) {
-        __syncthreads();                                   // the previous tile's readers are done
-        const bool paged_tile = t0 < Lq;
-        int pg = -1;
-        if (paged_tile) {
-            const int lp = t0 / PTILE;
-            pg = lp < v.max_pages ? v.page_table[size_t(b) * v.max_pages + lp] : -1;
-            if (pg >= v.num_pages) pg = -1;
-        }
+    // page of tile index lp (-1: unmapped, or not a paged tile)
+    auto page_of = [&](int lp) -> int {
+        if (lp * PTILE >= Lq || lp * PTILE > p_max || lp >= v.max_pages) return -1;
+        const int pg = v.page_table[size_t(b) * v.max_pages + lp];
+        return pg >= v.num_pages ? -1 : pg;
+    };
+    // this thread's 16-byte pieces of the raw blocks of page pg into stage st
+    auto issue = [&](int pg, int st) {
+        if (pg < 0) return;
+        const uint32_t d0 = smem_u32(raw0 + size_t(st) * RAWB);
+        const size_t bk = size_t(pg) * v.hkv + blk;
+        const uint8_t* kc = v.k_codes + bk * size_t(KCB);
+        const uint8_t* km = reinterpret_cast<const uint8_t*>(v.k_meta) + bk * size_t(KMB);
+        const uint8_t* vc = v.v_codes + bk * size_t(VCB);
+        const uint8_t* vm = reinterpret_cast<const uint8_t*>(v.v_meta) + bk * size_t(PTILE * v.nvg * 4);
+        for (int c = tid; c < KCB / 16; c += PTHREADS) cpa16(d0 + 16 * c, kc + 16 * c);
+        for (int c = tid; c < KMB / 16; c += PTHREADS) cpa16(d0 + KCB + 16 * c, km + 16 * c);
+        for (int c = tid; c < VCB / 16; c += PTHREADS) cpa16(d0 + KCB + KMB + 16 * c, vc + 16 * c);
+        for (int c = tid; c < PTILE * v.nvg * 4 / 16; c += PTHREADS) cpa16(d0 + KCB + KMB + VCB + 16 * c, vm + 16 * c);
+    };
+    int pg = page_of(0), pg_next = page_of(1), pg_after = page_of(2);
+    issue(pg, 0);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    for (int t0 = 0, st = 0; t0 <= p_max; t0 += PTILE, st ^= 1) {
+        // the next tile's copies go to the other stage, free since the last
+        // tile's reconstruction (before the barrier that preceded its products)
+        issue(pg_next, st ^ 1);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        const int pg_later = page_of(t0 / PTILE + 3);
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+        __syncthreads();                                   // this tile's pieces have landed; the previous tile's readers are done
+        const uint8_t* raw = raw0 + size_t(st) * RAWB;
         // value metadata of the tile's paged positions, as (scale 2^VB, zero - scale 2^VB)
-        if (paged_tile && pg >= 0)
+        if (pg >= 0)
             for (int e = tid; e < PTILE * v.nvg; e += PTHREADS) {
-                const uint32_t m = v.v_meta[((size_t(pg) * v.hkv + blk) * PTILE + e / v.nvg) * v.nvg + e % v.nvg];
+                const uint32_t m = reinterpret_cast<const uint32_t*>(raw + KCB + KMB + VCB)[e];
                 const float sc = bits_half(m & 0xffffu) * float(1 << VB);
                 sVf[e] = make_float2(sc, bits_half(m >> 16) - sc);
             }
@@ -158,14 +197,13 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
             float sc = 0.0f, zr = 0.0f;
             const uint16_t* wrow = nullptr;
             if (kind == 1) {
-                const uint8_t* kc = v.k_codes + (size_t(pg) * v.hkv + blk) * size_t(PTILE) * v.krow_bytes;
+                constexpr int kch = PD * KB / 8 < 16 ? PD * KB / 8 : 16;
 #pragma unroll
                 for (int i = 0; i < KB; ++i) {
                     const int byte = grp * 4 * KB + 4 * i;
-                    wd[i] = *reinterpret_cast<const uint32_t*>(kc + (byte / v.kch) * (PTILE * v.kch) + t * v.kch +
-                                                                byte % v.kch);
+                    wd[i] = *reinterpret_cast<const uint32_t*>(raw + (byte / kch) * (PTILE * kch) + t * kch + byte % kch);
                 }
-                const uint32_t m = v.k_meta[((size_t(pg) * v.hkv + blk) * PTILE + t) * v.nkg + grp];
+                const uint32_t m = reinterpret_cast<const uint32_t*>(raw + KCB)[t * (PD / 32) + grp];
                 sc = bits_half(m & 0xffffu) * float(1 << KB);
                 zr = bits_half(m >> 16) - sc;
             } else if (kind == 2) {
@@ -206,12 +244,12 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
             const int ch = tid >> 1, half = tid & 1, gvc = ch / v.vg;
             uint32_t wd[VB];
             if (pg >= 0) {
-                const uint8_t* vc = v.v_codes + (size_t(pg) * v.hkv + blk) * size_t(PD) * v.vchan_bytes;
+                constexpr int vch = PTILE * VB / 8 < 16 ? PTILE * VB / 8 : 16;
+                const uint8_t* vc = raw + KCB + KMB;
 #pragma unroll
                 for (int i = 0; i < VB; ++i) {
                     const int byte = half * 4 * VB + 4 * i;
-                    wd[i] = *reinterpret_cast<const uint32_t*>(vc + (byte / v.vch) * (PD * v.vch) + ch * v.vch +
-                                                                byte % v.vch);
+                    wd[i] = *reinterpret_cast<const uint32_t*>(vc + (byte / vch) * (PD * vch) + ch * vch + byte % vch);
                 }
             }
             const uint16_t* vw = reinterpret_cast<const uint16_t*>(v.v_win);
@@ -249,6 +287,9 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
             }
         }
         __syncthreads();
+        pg = pg_next;
+        pg_next = pg_after;
+        pg_after = pg_later;
         // no row of this warp sees the tile (every lane takes the vote)
         const bool skip = __all_sync(kFull, warp_pmax < t0);
         if (skip) continue;
@@ -329,6 +370,8 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
         }
     }
 
+    asm volatile("cp.async.wait_group 0;" ::: "memory");   // nothing in flight when the CTA exits
+
     // ---- o / l and lse = (m + log2 l) ln 2
     l_lo += __shfl_xor_sync(kFull, l_lo, 1);
     l_lo += __shfl_xor_sync(kFull, l_lo, 2);
@@ -358,13 +401,13 @@ cudaError_t launch_kv(const prefill::View& v, cudaStream_t s) {
     if (!configured[dev]) {
         const cudaError_t e = cudaFuncSetAttribute(prefill_mma_kernel<KB, VB>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   int(prefill_mma_smem(PD)));   // up to 128 value groups
+                                                   int(prefill_mma_smem(KB, VB, NVG_MAX)));
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
     const int qpc = PROWS / v.g;
     dim3 grid((v.max_q + qpc - 1) / qpc, v.hkv, v.batch);
-    prefill_mma_kernel<KB, VB><<<grid, PTHREADS, prefill_mma_smem(v.nvg), s>>>(v);
+    prefill_mma_kernel<KB, VB><<<grid, PTHREADS, prefill_mma_smem(KB, VB, v.nvg), s>>>(v);
     return cudaGetLastError();
 }
 
@@ -382,7 +425,7 @@ cudaError_t launch_k(const prefill::View& v, cudaStream_t s) {
 
 bool prefill_mma_supported(const prefill::View& v) {
     return v.d == PD && !v.kpc && !v.rotate && !v.one_query && v.kg == 32 && v.g >= 1 && v.g <= 8 &&
-           PD % v.vg == 0 && v.vg >= 1 && (v.kb == 1 || v.kb == 2 || v.kb == 4 || v.kb == 8) &&
+           PD % v.vg == 0 && v.vg >= 16 && (v.kb == 1 || v.kb == 2 || v.kb == 4 || v.kb == 8) &&
            (v.vb == 1 || v.vb == 2 || v.vb == 4 || v.vb == 8);
 }
 
