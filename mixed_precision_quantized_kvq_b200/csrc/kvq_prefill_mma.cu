@@ -56,6 +56,29 @@ constexpr size_t prefill_mma_smem(int kb, int vb, int nvg) {
     return 4 * size_t(KBYTES) + size_t(PTILE) * nvg * 8 + 2 * size_t(raw_bytes(kb, vb, nvg));
 }
 
+// the N words of bytes [4 N k, 4 N (k + 1)) of row r of a chunk-major block
+// [chunk][rows][cw] of ROWB-byte rows (cw = min(16, ROWB)), as vector loads
+template <int N, int ROWB>
+__device__ __forceinline__ void row_words(const uint8_t* blk, int rows, int r, int k, uint32_t (&w)[N]) {
+    constexpr int cw = ROWB < 16 ? ROWB : 16;
+    static_assert(4 * N <= cw || 4 * N % cw == 0, "a word group is inside one chunk or whole chunks");
+    const int byte = 4 * N * k;
+    const uint8_t* a = blk + (byte / cw) * (rows * cw) + r * cw + (byte % cw);
+    if constexpr (N == 1) {
+        w[0] = *reinterpret_cast<const uint32_t*>(a);
+    } else if constexpr (N == 2) {
+        const uint2 u = *reinterpret_cast<const uint2*>(a);
+        w[0] = u.x, w[1] = u.y;
+    } else if constexpr (N == 4) {
+        const uint4 u = *reinterpret_cast<const uint4*>(a);
+        w[0] = u.x, w[1] = u.y, w[2] = u.z, w[3] = u.w;
+    } else {
+        const uint4 u = *reinterpret_cast<const uint4*>(a);
+        const uint4 u2 = *reinterpret_cast<const uint4*>(a + rows * cw);
+        w[0] = u.x, w[1] = u.y, w[2] = u.z, w[3] = u.w, w[4] = u2.x, w[5] = u2.y, w[6] = u2.z, w[7] = u2.w;
+    }
+}
+
 __device__ __forceinline__ void cpa16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -190,19 +213,15 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
         __syncthreads();
         // ---- keys: thread = (position, key group of 32 channels), 8 channels at a time
         {
-            const int t = tid >> 2, grp = tid & 3, pos = t0 + t;
+            // a warp: 32 consecutive positions of one key group (conflict-free row reads)
+            const int t = tid & (PTILE - 1), grp = tid / PTILE, pos = t0 + t;
             // 0: zeros (past every row, or an unmapped page), 1: page codes, 2: window row
             const int kind = pos > p_max ? 0 : (pos < Lq ? (pg >= 0 ? 1 : 0) : 2);
             uint32_t wd[KB];
             float sc = 0.0f, zr = 0.0f;
             const uint16_t* wrow = nullptr;
             if (kind == 1) {
-                constexpr int kch = PD * KB / 8 < 16 ? PD * KB / 8 : 16;
-#pragma unroll
-                for (int i = 0; i < KB; ++i) {
-                    const int byte = grp * 4 * KB + 4 * i;
-                    wd[i] = *reinterpret_cast<const uint32_t*>(raw + (byte / kch) * (PTILE * kch) + t * kch + byte % kch);
-                }
+                row_words<KB, PD * KB / 8>(raw, PTILE, t, grp, wd);      // 32 channels of KB bits: KB words
                 const uint32_t m = reinterpret_cast<const uint32_t*>(raw + KCB)[t * (PD / 32) + grp];
                 sc = bits_half(m & 0xffffu) * float(1 << KB);
                 zr = bits_half(m >> 16) - sc;
@@ -244,13 +263,7 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
             const int ch = tid >> 1, half = tid & 1, gvc = ch / v.vg;
             uint32_t wd[VB];
             if (pg >= 0) {
-                constexpr int vch = PTILE * VB / 8 < 16 ? PTILE * VB / 8 : 16;
-                const uint8_t* vc = raw + KCB + KMB;
-#pragma unroll
-                for (int i = 0; i < VB; ++i) {
-                    const int byte = half * 4 * VB + 4 * i;
-                    wd[i] = *reinterpret_cast<const uint32_t*>(vc + (byte / vch) * (PD * vch) + ch * vch + byte % vch);
-                }
+                row_words<VB, PTILE * VB / 8>(raw + KCB + KMB, PD, ch, half, wd);   // 32 positions: VB words
             }
             const uint16_t* vw = reinterpret_cast<const uint16_t*>(v.v_win);
 #pragma unroll
