@@ -27,6 +27,7 @@ struct ChanCtx {
     __device__ float div_ru(float a, float b) const { return __fdiv_ru(a, b); }
     __device__ float sub_rn(float a, float b) const { return __fsub_rn(a, b); }
     __device__ float div_rn(float a, float b) const { return __fdiv_rn(a, b); }
+    __device__ float mul_rn(float a, float b) const { return __fmul_rn(a, b); }
     __device__ uint16_t f2bf_rn(float x) const { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
     __device__ void atomic_and(uint32_t* p, uint32_t v) const { atomicAnd(p, v); }
     __device__ void atomic_or(uint32_t* p, uint32_t v) const { atomicOr(p, v); }

@@ -138,12 +138,26 @@ KVQ_HD uint32_t span_meta(const Ctx& cx, float mn, float mx, int bits, float& zf
     if (sf == 0.0f) sh = 0;
     return uint32_t(sh) | (uint32_t(zh) << 16);
 }
+// codes of n values with the group's fp32 zero zf and scale sf:
+// rint((x - zf) / sf) clamped to [0, 2^bits - 1], the quotient correctly
+// rounded.  The quotient is formed as (x - zf) * (1 / sf), both correctly
+// rounded, which is within 2^-22 |q| of the exact quotient; the two can round
+// to different integers only when a half-integer lies that close to the
+// product, and then the division is carried out (the codes are the same as
+// with a division per value).
 template <class Ctx>
-KVQ_HD void span_codes(const Ctx& cx, const float* x, int stride, int n, float zf, float sf, int bits, uint8_t* c) {
+KVQ_HD void span_codes(const Ctx& cx, const float* x, int stride, int n, float zf, float sf, float rs, int bits,
+                       uint8_t* c) {
     const float qmax = float((1 << bits) - 1);
     for (int i = 0; i < n; ++i) {
         float code = 0.0f;
-        if (sf != 0.0f) code = fminf(fmaxf(rintf(cx.div_rn(cx.sub_rn(x[size_t(i) * stride], zf), sf)), 0.0f), qmax);
+        if (sf != 0.0f) {
+            const float a = cx.sub_rn(x[size_t(i) * stride], zf);
+            float q = cx.mul_rn(a, rs);
+            const float fq = floorf(q);
+            if (fabsf(q - fq - 0.5f) <= fabsf(q) * 0x1p-20f) q = cx.div_rn(a, sf);
+            code = fminf(fmaxf(rintf(q), 0.0f), qmax);
+        }
         c[i] = uint8_t(code);
     }
 }
@@ -183,10 +197,10 @@ constexpr int kParts = 4;
 
 // shared memory of one append CTA (bytes): keys and values as fp32 rows of
 // d + 1 floats (the padding puts rows that different threads walk in
-// different banks), the parts' extremes, key codes [d][kg], value codes as
-// rows of d + 4 bytes
+// different banks), the parts' extremes, per group (zero, scale, 1/scale),
+// key codes [d][kg], value codes as rows of d + 4 bytes
 KVQ_HD size_t append_smem_bytes(int d, int kg, int nvg) {
-    return size_t(kg) * size_t(d + 1) * 8 + size_t(d + kg * nvg) * kParts * 8 + size_t(d) * kg +
+    return size_t(kg) * size_t(d + 1) * 8 + size_t(d + kg * nvg) * (kParts * 8 + 12) + size_t(d) * kg +
            size_t(kg) * size_t(d + 4);
 }
 
@@ -200,8 +214,8 @@ struct alignas(16) Words4 {
 // quantized into their page.  Must run before part 2 rewrites ring slots.
 // The CTA's groups (d key groups along positions, kg * nvg value groups
 // along channels) are split into kParts parts each: the parts' extremes,
-// then each part's codes from its group's metadata, then the codes packed
-// into the channel runs.
+// then each group's metadata (one thread per group), then each part's codes,
+// then the codes packed into the channel runs.
 #ifdef __CUDACC__
 #pragma nv_exec_check_disable
 #endif
@@ -222,7 +236,8 @@ KVQ_HD void append_groups_body(Ctx& cx, const View& v) {
     float* sK = cx.smem();
     float* sV = sK + G * dp;
     float* sX = sV + G * dp;                                  // [T][kParts] {min, max}
-    uint8_t* sKC = reinterpret_cast<uint8_t*>(sX + 2 * T * kParts);   // key codes [d][G]
+    float* sQ = sX + 2 * T * kParts;                          // [T] {zero, scale, 1/scale}
+    uint8_t* sKC = reinterpret_cast<uint8_t*>(sQ + 3 * T);    // key codes [d][G]
     uint8_t* sC = sKC + d * G;                                // value codes [G][d + 4]
 
     // positions still in the ring: 16-byte loads of 8 channels, every load of a
@@ -286,8 +301,8 @@ KVQ_HD void append_groups_body(Ctx& cx, const View& v) {
         span_extremes(x, stride, m, sX[2 * e], sX[2 * e + 1]);
     }
     cx.sync();
-    for (int e = tid; e < T * kParts; e += NT) {
-        const int grp = e / kParts, k = e % kParts;
+    // each group's metadata once, from its parts' extremes
+    for (int grp = tid; grp < T; grp += NT) {
         const float* ex = sX + 2 * grp * kParts;
         float mn = ex[0], mx = ex[1];
         for (int i = 1; i < kParts; ++i) {
@@ -297,16 +312,28 @@ KVQ_HD void append_groups_body(Ctx& cx, const View& v) {
         float zf, sf;
         const bool key = grp < d;
         const uint32_t meta = span_meta(cx, mn, mx, key ? v.kb : v.vb, zf, sf);
+        if (key) {
+            *k_meta_at(v, pg, h, slot0, grp) = meta;
+        } else {
+            const int t = (grp - d) / v.nvg, cg = (grp - d) % v.nvg;
+            *v_meta_at(v, pg, h, slot0 + t, cg) = meta;
+        }
+        sQ[3 * grp] = zf;
+        sQ[3 * grp + 1] = sf;
+        sQ[3 * grp + 2] = sf != 0.0f ? cx.div_rn(1.0f, sf) : 0.0f;
+    }
+    cx.sync();
+    for (int e = tid; e < T * kParts; e += NT) {
+        const int grp = e / kParts, k = e % kParts;
+        const float zf = sQ[3 * grp], sf = sQ[3 * grp + 1], rs = sQ[3 * grp + 2];
         const float* x;
         int stride, m;
         part(e, x, stride, m);
-        if (key) {
-            if (k == 0) *k_meta_at(v, pg, h, slot0, grp) = meta;
-            span_codes(cx, x, stride, m, zf, sf, v.kb, sKC + grp * G + k * m);
+        if (grp < d) {
+            span_codes(cx, x, stride, m, zf, sf, rs, v.kb, sKC + grp * G + k * m);
         } else {
             const int t = (grp - d) / v.nvg, cg = (grp - d) % v.nvg;
-            if (k == 0) *v_meta_at(v, pg, h, slot0 + t, cg) = meta;
-            span_codes(cx, x, stride, m, zf, sf, v.vb, sC + t * cp + cg * v.vg + k * m);
+            span_codes(cx, x, stride, m, zf, sf, rs, v.vb, sC + t * cp + cg * v.vg + k * m);
         }
     }
     cx.sync();

@@ -86,6 +86,10 @@ struct Ctx {
         volatile float va = a, vb = b;
         return va / vb;
     }
+    float mul_rn(float a, float b) const {
+        volatile float va = a, vb = b;
+        return va * vb;
+    }
     uint16_t f2bf_rn(float x) const { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
     void atomic_and(uint32_t* p, uint32_t v) const { std::atomic_ref<uint32_t>(*p).fetch_and(v); }
     void atomic_or(uint32_t* p, uint32_t v) const { std::atomic_ref<uint32_t>(*p).fetch_or(v); }
