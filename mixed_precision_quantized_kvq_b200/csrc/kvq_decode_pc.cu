@@ -163,17 +163,28 @@ __device__ __forceinline__ uint32_t codes_f16(uint32_t y) {
     return h2bits(r);
 }
 
-// the codes of positions 2 tig + 8 hf and the next one (a pair never
-// straddles a word) of a k-step's words, as an fp16 pair, the first in the
-// low half; the word is chosen without indexing the array at run time
+// The weighted-value MMA's k slots (2 tig, 2 tig + 1) of register a0 hold the
+// k-step's positions tig and tig + 8, those of a2 positions tig + 4 and
+// tig + 12 (any order of k works when A and B agree; the weight table pairs
+// the same positions).  A position p + 8 sits 8*BITS bits above p, so for
+// 2-bit codes both halves come from one shift and one mask.  The codes of
+// positions tig + 4 hf and tig + 4 hf + 8 of a k-step's words, as an fp16
+// pair, the first in the low half.
 template <int BITS, int HF>
 __device__ __forceinline__ uint32_t vpair_f16(const uint32_t (&w)[4], int tig) {
-    const int pos = (2 * tig + 8 * HF) * BITS;
-    uint32_t x;
-    if constexpr (BITS == 8) x = (tig >> 1) ? w[2 * HF + 1] : w[2 * HF];
-    else x = w[(8 * HF * BITS) >> 5];
-    x >>= pos & 31;
-    return codes_f16<BITS>((x & ((1u << BITS) - 1u)) | ((x << (16 - BITS)) & (((1u << BITS) - 1u) << 16)));
+    constexpr uint32_t m = (1u << BITS) - 1u;
+    const int p = tig + 4 * HF;
+    if constexpr (BITS == 1) {                      // bits p and p + 8 of the 16-bit word
+        const uint32_t x = w[0] >> p;
+        return codes_f16<1>((x & m) | ((x << 8) & (m << 16)));
+    } else if constexpr (BITS == 2) {               // bits 2p and 2p + 16 of the word
+        return codes_f16<2>(w[0] >> (2 * p));
+    } else if constexpr (BITS == 4) {               // the same nibble of words 0 and 1
+        return codes_f16<4>(__byte_perm(w[0] >> (4 * p), w[1] >> (4 * p), 0x5410));
+    } else {                                        // byte p % 4 of word p / 4 and of word p / 4 + 2
+        const uint32_t lo = (p >> 2) ? w[1] : w[0], hi = (p >> 2) ? w[3] : w[2];
+        return codes_f16<8>(__byte_perm(lo, hi, uint32_t(p & 3) | (uint32_t((p & 3) + 4) << 8)));
+    }
 }
 // the codes of positions 16 ks .. 16 ks + 15 of channel j's value run (2*BITS bytes)
 template <int BITS>
@@ -332,7 +343,9 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
     float ov[VMMA ? 8 : 1][4];
 #pragma unroll
     for (int mt = 0; mt < (VMMA ? 8 : 1); ++mt) ov[mt][0] = ov[mt][1] = ov[mt][2] = ov[mt][3] = 0.0f;
-    const int tA = 2 * lane, tB = tA + 1;           // score positions of this lane (in the tile)
+    // positions of this lane in the tile (scores, softmax, weight table): p and
+    // p + 8 of the lane's 16-position block, the pairs the value MMA's k slots take
+    const int tA = 16 * (lane >> 3) + (lane & 7), tB = tA + 8;
     const int j0 = 4 * lane;                        // value channels of this lane
     const int gv = j0 / p.vg;                       // their value group
 
@@ -509,7 +522,7 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
         // positions in pages p*scale*2^VB, ring positions p; per value group the
         // zero points and the mantissa offsets: sum_t p (zero - scale 2^VB).
         // Four heads: positions in pages as fp16 parts of p*scale, [group][(head,
-        // part)][t/2] (lane l writes word l: positions 2l, 2l+1), and the zero
+        // part)][word] (lane l writes word l: its positions tA, tB), and the zero
         // sums sum_t p zero per group; ring positions p in the float table.
         float corr[NH];
 #pragma unroll
@@ -531,7 +544,7 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
             }
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                const int t = tA + half;
+                const int t = half ? tB : tA;
                 const float* pp = half ? pB : pA;
                 if (t >= nv || (VMMA && t < nq)) continue;
                 float wt[NH];
