@@ -164,7 +164,9 @@ int kvq_window_bytes(const kvq_layout* layout, int batch, size_t* bytes);
 
 /* Workspace that kvq_decode_attention needs for this batch and bound on
  * lengths on the current device (split partials); 0 on invalid input, and
- * 0 for k_per_channel layouts (no split partials: workspace may be NULL). */
+ * for k_per_channel layouts the bytes that let the decode split each (sequence,
+ * kv-head) between CTAs when the pairs leave SMs idle, else 0; for these
+ * layouts the workspace is optional (NULL, or smaller: one CTA per pair). */
 size_t kvq_decode_workspace_bytes(const kvq_layout* layout, int batch, int max_len);
 
 /* Select the decode kernel family for subsequent kvq_decode_attention and
@@ -237,10 +239,13 @@ int kvq_quantize_append(const kvq_layout* layout, const kvq_cache* cache,
  *           call leaves the tickets at zero again, so the zero fill is needed
  *           once per allocation, not per call.  Calls that overlap on the GPU
  *           need separate workspaces.
- *           Not read for k_per_channel layouts (may be NULL): those run the
+ *           Optional for k_per_channel layouts (may be NULL): those run the
  *           per-channel decode kernel, one CTA per (sequence, kv-head) whose
- *           warps merge their parts in shared memory (head_dim 64 layouts:
- *           the chunked-prefill kernel with one query per sequence).
+ *           warps merge their parts in shared memory, or, when the workspace
+ *           holds kvq_decode_workspace_bytes (zero-filled before its first
+ *           use, like the others), several CTAs per pair merged through it
+ *           by the last one to finish (head_dim 64 layouts: the
+ *           chunked-prefill kernel with one query per sequence).
  * Returns KVQ_ERR_UNSUPPORTED for batch or num_kv_heads above 65535. */
 int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache,
                          const void* q, int q_dtype, const int32_t* lens, int max_len,

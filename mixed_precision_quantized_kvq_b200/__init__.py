@@ -245,6 +245,20 @@ def kvq_quantize_append(layout: Layout, cache: PagedCache, k_new: torch.Tensor, 
           _dtype_code(k_new), _ptr(cu_new), _ptr(lens), int(max_new), _stream(stream))
 
 
+def _nbytes(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def _check_workspace(layout, cache, max_len, workspace):
+    """At least kvq_decode_workspace_bytes; optional for key groups along
+    positions (without it, or with less, the pairs are not split between CTAs)."""
+    if layout.k_per_channel:
+        _check(workspace, "workspace", (torch.uint8,), optional=True)
+    else:
+        _check(workspace, "workspace", (torch.uint8,), kvq_decode_workspace_bytes(layout, cache.batch, max_len),
+               at_least=True)
+
+
 def _check_decode_args(layout, cache, q, lens, out, lse):
     B, Hq, d = cache.batch, layout.num_q_heads, layout.head_dim
     _check(q, "q", _FLOAT_IN, B * Hq * d)
@@ -258,11 +272,10 @@ def kvq_decode_attention(layout: Layout, cache: PagedCache, q: torch.Tensor, len
                          lse: Optional[torch.Tensor], workspace: torch.Tensor, stream=None) -> None:
     """kvq.h kvq_decode_attention: q [B][Hq][d] -> out fp32 [B][Hq][d], lse fp32 [B][Hq]."""
     _check_decode_args(layout, cache, q, lens, out, lse)
-    _check(workspace, "workspace", (torch.uint8,), kvq_decode_workspace_bytes(layout, cache.batch, max_len),
-           at_least=True)
+    _check_workspace(layout, cache, max_len, workspace)
     _call("kvq_decode_attention", C.byref(layout.c()), C.byref(cache.c()), _ptr(q), _dtype_code(q),
           _ptr(lens), int(max_len), C.c_float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace),
-          C.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
+          C.c_size_t(_nbytes(workspace)), _stream(stream))
 
 
 def kvq_append_decode(layout: Layout, cache: PagedCache, k_new: torch.Tensor, v_new: torch.Tensor,
@@ -281,12 +294,11 @@ def kvq_append_decode(layout: Layout, cache: PagedCache, k_new: torch.Tensor, v_
     _check(cu_new, "cu_new", _I32, B + 1)
     _check(lens_old, "lens_old", _I32, B)
     _check_decode_args(layout, cache, q, lens, out, lse)
-    _check(workspace, "workspace", (torch.uint8,), kvq_decode_workspace_bytes(layout, cache.batch, max_len),
-           at_least=True)
+    _check_workspace(layout, cache, max_len, workspace)
     _call("kvq_append_decode", C.byref(layout.c()), C.byref(cache.c()), _ptr(k_new), _ptr(v_new),
           _dtype_code(k_new), _ptr(cu_new), _ptr(lens_old), int(max_new), _ptr(q), _dtype_code(q), _ptr(lens),
           int(max_len), C.c_float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace),
-          C.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
+          C.c_size_t(_nbytes(workspace)), _stream(stream))
 
 
 def kvq_decode_attention_static_scratch(layout: Layout, cache: PagedCache, q: torch.Tensor,

@@ -157,8 +157,12 @@ int kvq_window_bytes(const kvq_layout* layout, int batch, size_t* bytes) {
 
 size_t kvq_decode_workspace_bytes(const kvq_layout* layout, int batch, int max_len) {
     if (check_layout(layout) || batch < 0 || max_len < 0) return 0;
-    if (layout->k_per_channel) return 0;   // one pass per (sequence, kv-head), no partials
     Params p = make_params(layout, nullptr);
+    if (layout->k_per_channel) {   // partials only when the pairs are split between CTAs
+        if (!kvq::decode_pc_supported(p, max_len)) return 0;
+        const int splits = kvq::pc_splits(p, batch, max_len, device_sm_count());
+        return splits > 1 ? kvq::pc_workspace_bytes(p, batch, splits) : 0;
+    }
     kvq::DecodePlan pl = kvq::plan_decode(p, batch, max_len, device_sm_count());
     return kvq::decode_workspace_bytes(p, batch, pl);
 }
@@ -184,14 +188,21 @@ int kvq_decode_status(unsigned int* wait_timeouts, unsigned int* bad_tickets, in
     return cuda_status(kvq::decode_status(wait_timeouts, bad_tickets, clear != 0));
 }
 
-// decode for key groups along positions: the per-channel decode kernel, or the
+// decode for key groups along positions: the per-channel decode kernel (its
+// pairs split between CTAs when the workspace holds the partials), or the
 // chunked-prefill kernel with one query per sequence for the shapes it does not take
 static int decode_per_channel(const Params& p, const void* q, int q_dtype, const int32_t* lens, int max_len,
-                              float sm_scale, float* out, float* lse, kvq_stream_t stream) {
+                              float sm_scale, float* out, float* lse, void* ws, size_t ws_bytes,
+                              kvq_stream_t stream) {
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (kvq::decode_pc_supported(p, max_len))
+    if (kvq::decode_pc_supported(p, max_len)) {
+        int splits = kvq::pc_splits(p, p.batch, max_len, device_sm_count());
+        if (splits > 1 && (!ws || ws_bytes < kvq::pc_workspace_bytes(p, p.batch, splits) ||
+                           (reinterpret_cast<uintptr_t>(ws) & 255u)))
+            splits = 1;   // no room for the partials: one CTA per pair
         return cuda_status(kvq::launch_decode_per_channel(p, q, q_dtype == KVQ_BF16, lens, max_len, sm_scale, out, lse,
-                                                          s));
+                                                          ws, splits, s));
+    }
     return cuda_status(kvq::launch_prefill_attention(p, 1, 1, q, q_dtype == KVQ_BF16, nullptr, lens, max_len, 1,
                                                      sm_scale, out, lse, s));
 }
@@ -226,8 +237,9 @@ int kvq_decode_attention(const kvq_layout* layout, const kvq_cache* cache, const
     if (cache->batch == 0) return KVQ_OK;
     if (cache->batch > 65535 || layout->num_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
     Params p = make_params(layout, cache);
-    if (layout->k_per_channel)   // needs no workspace
-        return decode_per_channel(p, q, q_dtype, lens, max_len, sm_scale, out, lse, stream);
+    if (layout->k_per_channel)   // the workspace is optional (used for split pairs when it is large enough)
+        return decode_per_channel(p, q, q_dtype, lens, max_len, sm_scale, out, lse, workspace, workspace_bytes,
+                                  stream);
     kvq::DecodePlan pl = kvq::plan_decode(p, cache->batch, max_len, device_sm_count());
     const size_t need = kvq::decode_workspace_bytes(p, cache->batch, pl);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -362,8 +374,12 @@ extern "C" int kvq_decode_attention_static_scratch(const kvq_layout* layout, con
     if (cache->batch == 0) return KVQ_OK;
     if (cache->batch > 65535 || layout->num_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
     Params p = make_params(layout, cache);
-    if (layout->k_per_channel)   // needs no scratch
-        return decode_per_channel(p, q, q_dtype, lens, max_len, sm_scale, out, lse, stream);
+    if (layout->k_per_channel) {   // the static scratch holds the partials of split pairs when large enough
+        void* scratch = nullptr;
+        if ((rc = static_scratch(&scratch))) return rc;
+        return decode_per_channel(p, q, q_dtype, lens, max_len, sm_scale, out, lse, scratch, KVQ_STATIC_SCRATCH_BYTES,
+                                  stream);
+    }
     kvq::DecodePlan pl = kvq::plan_decode(p, cache->batch, max_len, device_sm_count());
     if (kvq::decode_workspace_bytes(p, cache->batch, pl) > KVQ_STATIC_SCRATCH_BYTES) return KVQ_ERR_WORKSPACE;
     void* scratch = nullptr;

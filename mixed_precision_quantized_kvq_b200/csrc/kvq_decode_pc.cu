@@ -54,7 +54,7 @@ constexpr int GMAX = 8;             // query heads per kv-head (kernels for up t
 // warps per CTA at most (about 200 registers per thread)
 __host__ __device__ constexpr int nw_max(int nh) { return 8; }
 constexpr int PHROW = 36;           // words per row of the fp16 weight table (32 used; the rest spreads banks)
-constexpr int SMEM_MAX = 227 * 1024;
+constexpr int SMEM_MAX = 227 * 1024 - 256;   // dynamic bytes; the merge ticket is static
 constexpr unsigned FULLM = 0xffffffffu;
 
 // shared-memory geometry of one launch (bytes)
@@ -71,6 +71,12 @@ struct PcGeom {
 };
 
 __host__ __device__ inline int round_up(int x, int a) { return (x + a - 1) / a * a; }
+
+constexpr int PSW = PD + 4;         // floats per (head) row of a part: PD outputs, maximum, weight sum, pad
+// bytes of the split partials [pairs][splits][GMAX heads][PSW] (256-aligned)
+inline size_t pc_part_bytes(int batch, int hkv, int splits) {
+    return (size_t(batch) * hkv * splits * GMAX * PSW * 4 + 255) & ~size_t(255);
+}
 
 PcGeom pc_geometry(const Params& p, int max_len, int nh) {
     PcGeom g{};
@@ -214,6 +220,17 @@ __device__ __forceinline__ void ld_heads(const float* a, float (&x)[NH]) {
     }
 }
 
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* a, unsigned v) {
+    unsigned old;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(a), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ float ld_relaxed_gpu(const float* a) {
+    float v;
+    asm volatile("ld.relaxed.gpu.f32 %0, [%1];" : "=f"(v) : "l"(a) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULLM, v, o);
@@ -230,14 +247,17 @@ template <int KB, int VB, int NH>
 __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Params p, const void* __restrict__ qv,
                                                                   int q_bf16, const int32_t* __restrict__ lens,
                                                                   int max_len, float sl2, float* __restrict__ out,
-                                                                  float* __restrict__ lse, const PcGeom geo) {
+                                                                  float* __restrict__ lse, const PcGeom geo,
+                                                                  float* __restrict__ wpart, unsigned* tickets,
+                                                                  const int S) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    const int h = blockIdx.x, b = blockIdx.y;
+    const int h = blockIdx.x, b = blockIdx.y, split = blockIdx.z;   // split `split` of S of the pair's tiles
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, NW = blockDim.x >> 5;
     const int g = p.g, kg = p.kg, nvg = p.nvg;
     const int L = max(0, min(lens[b], max_len));
     const size_t orow0 = size_t(b) * p.hq + size_t(h) * g;
-    if (L == 0) {                                   // an empty sequence: o = 0, lse = -inf
+    if (L == 0) {                                   // an empty sequence: o = 0, lse = -inf (no split takes a ticket)
+        if (split == 0)
         for (int e = tid; e < g * PD; e += blockDim.x) {
             out[(orow0 + e / PD) * PD + e % PD] = 0.0f;
             if (lse && e % PD == 0) lse[orow0 + e / PD] = -INFINITY;
@@ -249,7 +269,9 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
     uint8_t* areas = smem_raw + geo.OFF_AREAS;
     const int R = p.W + kg - 1;                     // ring slots
     const int Q = L - p.W > 0 ? ((L - p.W) / kg) * kg : 0;   // positions below Q live in pages
-    const int ntiles = (L + PT - 1) / PT, npq = (Q + PT - 1) / PT;
+    const int ntiles_all = (L + PT - 1) / PT, npq = (Q + PT - 1) / PT;
+    // this CTA's tiles [tile0, ntiles) of the pair's ntiles_all
+    const int tile0 = int((long(ntiles_all) * split) / S), ntiles = int((long(ntiles_all) * (split + 1)) / S);
     const size_t prow = size_t(b) * p.hkv + h;      // (sequence, kv-head) row of the ring
 
     for (int e = tid; e < NH * PD; e += blockDim.x) {
@@ -360,9 +382,9 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
     }
 
     int slot = 0;
-    issue(w, 0);
+    issue(tile0 + w, 0);
     cpa_commit();
-    for (int i = w; i < ntiles; i += NW) {
+    for (int i = tile0 + w; i < ntiles; i += NW) {
         issue(i + NW, slot ^ 1);
         cpa_commit();
         cpa_wait_1();
@@ -667,6 +689,11 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
         }
     }
     __syncthreads();
+    // a pair split between CTAs: this CTA's merged part goes to the workspace,
+    // [pair][split][head][PS]: the unnormalized output, the maximum (log2
+    // domain) and the weight sum
+    const size_t pair = size_t(b) * p.hkv + h;
+    float* wp = S > 1 ? wpart + (pair * S + split) * size_t(GMAX * PS) : nullptr;
     for (int e = tid; e < g * PD; e += blockDim.x) {
         const int r = e / PD, j = e % PD;
         float M = -INFINITY;
@@ -679,20 +706,59 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
             num = fmaf(part[(ww * NH + r) * PS + j], f, num);
             den = fmaf(part[(ww * NH + r) * PS + PD + 1], f, den);
         }
+        if (S == 1) {
+            out[(orow0 + r) * PD + j] = num / den;
+            if (lse && j == 0) lse[orow0 + r] = (M + log2f(den)) * 0.693147180559945309f;
+        } else {
+            wp[r * PS + j] = num;
+            if (j == 0) {
+                wp[r * PS + PD] = M;
+                wp[r * PS + PD + 1] = den;
+            }
+        }
+    }
+    if (S == 1) return;
+    // every thread's part, then the ticket (release); the CTA that takes the
+    // pair's last ticket (acquire) merges every split's part in split order,
+    // so that the result does not depend on which CTA finished last, and
+    // resets the ticket for the next call.  No CTA waits for another.
+    __shared__ unsigned ticket;
+    __syncthreads();
+    if (tid == 0) ticket = atom_add_acq_rel_gpu(tickets + pair, 1u);
+    __syncthreads();
+    if (ticket != unsigned(S - 1)) return;
+    const float* wq = wpart + pair * S * size_t(GMAX * PS);
+    for (int e = tid; e < g * PD; e += blockDim.x) {
+        const int r = e / PD, j = e % PD;
+        float M = -INFINITY;
+        for (int sp = 0; sp < S; ++sp) M = fmaxf(M, ld_relaxed_gpu(wq + (size_t(sp) * GMAX + r) * PS + PD));
+        float num = 0.0f, den = 0.0f;
+        for (int sp = 0; sp < S; ++sp) {
+            const float* q2 = wq + (size_t(sp) * GMAX + r) * PS;
+            const float ms = ld_relaxed_gpu(q2 + PD);
+            if (ms == -INFINITY) continue;          // a split without positions
+            const float f = ex2(ms - M);
+            num = fmaf(ld_relaxed_gpu(q2 + j), f, num);
+            den = fmaf(ld_relaxed_gpu(q2 + PD + 1), f, den);
+        }
         out[(orow0 + r) * PD + j] = num / den;
         if (lse && j == 0) lse[orow0 + r] = (M + log2f(den)) * 0.693147180559945309f;
     }
+    if (tid == 0) tickets[pair] = 0u;               // ready for the next call
 }
 
 template <int KB, int NH>
 cudaError_t launch_nh_pc(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len, float sl2,
-                         float* out, float* lse, cudaStream_t s) {
+                         float* out, float* lse, void* ws, int S, cudaStream_t s) {
     const PcGeom geo = pc_geometry(p, max_len, NH);
-    const dim3 grid(p.hkv, p.batch);
+    const dim3 grid(p.hkv, p.batch, S);
+    float* wpart = S > 1 ? static_cast<float*>(ws) : nullptr;
+    unsigned* tickets = S > 1 ? reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + pc_part_bytes(p.batch, p.hkv, S))
+                              : nullptr;
     auto go = [&](auto kern) -> cudaError_t {
         const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, geo.bytes);
         if (e != cudaSuccess) return e;
-        kern<<<grid, geo.NW * 32, geo.bytes, s>>>(p, q, q_bf16, lens, max_len, sl2, out, lse, geo);
+        kern<<<grid, geo.NW * 32, geo.bytes, s>>>(p, q, q_bf16, lens, max_len, sl2, out, lse, geo, wpart, tickets, S);
         return cudaGetLastError();
     };
     switch (p.vb) {
@@ -705,9 +771,9 @@ cudaError_t launch_nh_pc(const Params& p, const void* q, int q_bf16, const int32
 
 template <int KB>
 cudaError_t launch_kb_pc(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len, float sl2,
-                         float* out, float* lse, cudaStream_t s) {
-    if (p.g <= 4) return launch_nh_pc<KB, 4>(p, q, q_bf16, lens, max_len, sl2, out, lse, s);
-    return launch_nh_pc<KB, 8>(p, q, q_bf16, lens, max_len, sl2, out, lse, s);
+                         float* out, float* lse, void* ws, int S, cudaStream_t s) {
+    if (p.g <= 4) return launch_nh_pc<KB, 4>(p, q, q_bf16, lens, max_len, sl2, out, lse, ws, S, s);
+    return launch_nh_pc<KB, 8>(p, q, q_bf16, lens, max_len, sl2, out, lse, ws, S, s);
 }
 
 }  // namespace
@@ -720,14 +786,29 @@ bool decode_pc_supported(const Params& p, int max_len) {
     return pc_geometry(p, max_len, p.g <= 4 ? 4 : 8).NW >= 2;
 }
 
+int pc_splits(const Params& p, int batch, int max_len, int sms) {
+    const long pairs = long(batch) * p.hkv;
+    if (pairs <= 0) return 1;
+    long S = sms / pairs;                           // every CTA in one wave (one CTA per SM)
+    const long by_len = (long(max_len) + PT - 1) / PT / nw_max(8);   // eight tiles per CTA at least
+    if (S > by_len) S = by_len;
+    if (S > 8) S = 8;
+    return S < 1 ? 1 : int(S);
+}
+
+size_t pc_workspace_bytes(const Params& p, int batch, int splits) {
+    return pc_part_bytes(batch, p.hkv, splits) + size_t(batch) * p.hkv * 4;
+}
+
 cudaError_t launch_decode_per_channel(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len,
-                                      float sm_scale, float* out, float* lse, cudaStream_t s) {
+                                      float sm_scale, float* out, float* lse, void* ws, int splits, cudaStream_t s) {
     const float sl2 = sm_scale * 1.4426950408889634f;
+    const int S = splits > 1 && ws ? splits : 1;
     switch (p.kb) {
-        case 1: return launch_kb_pc<1>(p, q, q_bf16, lens, max_len, sl2, out, lse, s);
-        case 2: return launch_kb_pc<2>(p, q, q_bf16, lens, max_len, sl2, out, lse, s);
-        case 4: return launch_kb_pc<4>(p, q, q_bf16, lens, max_len, sl2, out, lse, s);
-        default: return launch_kb_pc<8>(p, q, q_bf16, lens, max_len, sl2, out, lse, s);
+        case 1: return launch_kb_pc<1>(p, q, q_bf16, lens, max_len, sl2, out, lse, ws, S, s);
+        case 2: return launch_kb_pc<2>(p, q, q_bf16, lens, max_len, sl2, out, lse, ws, S, s);
+        case 4: return launch_kb_pc<4>(p, q, q_bf16, lens, max_len, sl2, out, lse, ws, S, s);
+        default: return launch_kb_pc<8>(p, q, q_bf16, lens, max_len, sl2, out, lse, ws, S, s);
     }
 }
 

@@ -158,8 +158,15 @@ size_t decode_workspace_bytes(const Params& p, int batch, const DecodePlan& plan
 // decode for key groups along positions (kvq_decode_pc.cu): head_dim 128, up
 // to 8 query heads per kv-head, key groups of 16/32/64 positions, unrotated
 bool decode_pc_supported(const Params& p, int max_len);
+// CTAs per (sequence, kv-head) of the per-channel decode: more than one only
+// when the pairs leave SMs without a CTA (all CTAs in one wave), at most 8,
+// and at least eight 64-position tiles per CTA at max_len
+int pc_splits(const Params& p, int batch, int max_len, int sms);
+// workspace of a split per-channel decode: partials [pairs][splits][8 heads][132]
+// floats, then one merge ticket per pair (zero-filled once)
+size_t pc_workspace_bytes(const Params& p, int batch, int splits);
 cudaError_t launch_decode_per_channel(const Params& p, const void* q, int q_bf16, const int32_t* lens, int max_len,
-                                      float sm_scale, float* out, float* lse, cudaStream_t s);
+                                      float sm_scale, float* out, float* lse, void* ws, int splits, cudaStream_t s);
 // the append of max_new tokens per sequence is one launch of the small-append
 // kernel (which lets a programmatic dependent start early)
 bool append_is_one_launch(const Params& p, int max_new);

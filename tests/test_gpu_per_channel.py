@@ -109,3 +109,32 @@ def test_empty_sequences_and_static_scratch_entry():
     torch.cuda.synchronize()
     assert torch.equal(o2.cpu(), torch.from_numpy(np.asarray(out, np.float32)))
     assert torch.all(o2[1] == 0) and torch.all(torch.isinf(l2[1]))
+
+
+def test_split_pairs():
+    """Few (sequence, kv-head) pairs with long sequences: each pair's tiles
+    are split between CTAs that merge through the workspace (the last CTA to
+    finish merges every split in split order).  Against the oracle, with an
+    empty sequence; the static-scratch entry point gives the same bits; the
+    call without a workspace (one CTA per pair) agrees within tolerance."""
+    w = pc(batch=2, num_kv_heads=2, num_q_heads=8, ragged=(2500, 4200), window=64, k_group=64, v_group=64)
+    lens = wl.lengths(w)
+    lens[1] = 0
+    lens[0] = max(int(lens[0]), 3000)
+    pair = Pair(w, lens)
+    pair.prefill(with_f32=False)
+    max_len = int(lens.max())
+    assert kvq.kvq_decode_workspace_bytes(pair.glay, w.batch, max_len) > 0   # the split is taken
+    out, ref = pair.check_decode(step=2)
+    q = torch_raw(wl.query(w, 2)[0])
+    sc = 1.0 / np.sqrt(w.head_dim)
+    o2 = torch.empty((w.batch, w.num_q_heads, w.head_dim), device="cuda")
+    l2 = torch.empty((w.batch, w.num_q_heads), device="cuda")
+    kvq.kvq_decode_attention_static_scratch(pair.glay, pair.gcache, q, pair.glens, max_len, sc, o2, l2)
+    o3 = torch.empty_like(o2)
+    l3 = torch.empty_like(l2)
+    kvq.kvq_decode_attention(pair.glay, pair.gcache, q, pair.glens, max_len, sc, o3, l3, None)
+    torch.cuda.synchronize()
+    assert torch.equal(o2.cpu(), torch.from_numpy(np.asarray(out, np.float32)))
+    check_close(o3.cpu().numpy(), ref, "out without a workspace")
+    assert torch.all(o2[1] == 0) and torch.all(torch.isinf(l2[1]))
