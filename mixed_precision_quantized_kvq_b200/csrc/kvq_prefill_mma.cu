@@ -52,8 +52,10 @@ constexpr int NVG_MAX = 8;                // value groups of 16 channels or more
 __host__ __device__ constexpr int raw_bytes(int kb, int vb, int nvg) {
     return PTILE * PD * kb / 8 + PTILE * (PD / 32) * 4 + PD * PTILE * vb / 8 + PTILE * nvg * 4;
 }
+constexpr int QFRAG_BYTES = 8 * 2 * 32 * 16;   // per warp: the query's A fragments [k-step][hi/lo][lane]
 constexpr size_t prefill_mma_smem(int kb, int vb, int nvg) {
-    return 4 * size_t(KBYTES) + size_t(PTILE) * nvg * 8 + 2 * size_t(raw_bytes(kb, vb, nvg));
+    return 4 * size_t(KBYTES) + size_t(PTILE) * nvg * 8 + 2 * size_t(raw_bytes(kb, vb, nvg)) +
+           size_t(PTHREADS / 32) * QFRAG_BYTES;
 }
 
 // the N words of bytes [4 N k, 4 N (k + 1)) of row r of a chunk-major block
@@ -138,7 +140,9 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
     auto row_valid = [&](int r) { return r < R && r / g < nq; };
     auto row_pos = [&](int r) { return row_valid(r) ? base + i0 + r / g : -1; };
     const int p_lo = row_pos(r_lo), p_hi = row_pos(r_hi);
-    uint32_t qh[8][4], ql[8][4];
+    // the query's A fragments (bf16 hi and lo parts) in shared memory, each lane's
+    // own in register order, read back per k-step (registers for the tiles' work)
+    uint4* sQ = reinterpret_cast<uint4*>(raw0 + 2 * size_t(RAWB)) + size_t(warp) * (QFRAG_BYTES / 16);
     {
         auto qpair = [&](int r, int ch, uint32_t& hi, uint32_t& lo) {
             float x0 = 0.0f, x1 = 0.0f;
@@ -156,12 +160,15 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
             }
             split2(x0 * v.scale_log2, x1 * v.scale_log2, hi, lo);
         };
-#pragma unroll
+#pragma unroll 2
         for (int kk = 0; kk < 8; ++kk) {
-            qpair(r_lo, 16 * kk + 2 * tig, qh[kk][0], ql[kk][0]);
-            qpair(r_hi, 16 * kk + 2 * tig, qh[kk][1], ql[kk][1]);
-            qpair(r_lo, 16 * kk + 8 + 2 * tig, qh[kk][2], ql[kk][2]);
-            qpair(r_hi, 16 * kk + 8 + 2 * tig, qh[kk][3], ql[kk][3]);
+            uint32_t hq[4], lq[4];
+            qpair(r_lo, 16 * kk + 2 * tig, hq[0], lq[0]);
+            qpair(r_hi, 16 * kk + 2 * tig, hq[1], lq[1]);
+            qpair(r_lo, 16 * kk + 8 + 2 * tig, hq[2], lq[2]);
+            qpair(r_hi, 16 * kk + 8 + 2 * tig, hq[3], lq[3]);
+            sQ[(2 * kk) * 32 + lane] = make_uint4(hq[0], hq[1], hq[2], hq[3]);
+            sQ[(2 * kk + 1) * 32 + lane] = make_uint4(lq[0], lq[1], lq[2], lq[3]);
         }
     }
     float o[16][4];
@@ -315,13 +322,15 @@ __global__ void __launch_bounds__(PTHREADS, 1) prefill_mma_kernel(const prefill:
         for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0f;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
+            const uint4 a = sQ[(2 * kk) * 32 + lane], c = sQ[(2 * kk + 1) * 32 + lane];
+            const uint32_t qh[4] = {a.x, a.y, a.z, a.w}, ql[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 uint32_t f[4];      // Kh k0-7, Kh k8-15, Kl k0-7, Kl k8-15 of positions 8j .. 8j+7
                 ldsm_x4(f, (mi < 2 ? sKh : sKl) + swz(8 * j + rr, 2 * kk + (mi & 1), 16));
-                mma_bf16(s[j], qh[kk], f[0], f[1]);
-                mma_bf16(s[j], qh[kk], f[2], f[3]);
-                mma_bf16(s[j], ql[kk], f[0], f[1]);
+                mma_bf16(s[j], qh, f[0], f[1]);
+                mma_bf16(s[j], qh, f[2], f[3]);
+                mma_bf16(s[j], ql, f[0], f[1]);
             }
         }
         // ---- causal mask, online softmax (rows r_lo: s[][0..1], r_hi: s[][2..3])
