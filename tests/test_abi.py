@@ -175,3 +175,22 @@ def test_per_channel_ring_required_without_window():
     buf = C.create_string_buffer(1024)
     p = C.c_void_p((C.addressof(buf) + 255) & ~255)
     assert lib.kvq_quantize_append(C.byref(lay.c()), C.byref(c), p, p, 1, p, p, 4, None) == kvq.KVQ_ERR_INVALID_ARG
+
+
+def test_per_channel_split_workspace_rule():
+    """Key groups along positions: the decode splits pairs between CTAs only
+    when the pairs leave SMs idle (148 SMs without a device) and the sequences
+    hold eight 64-position tiles per CTA; the workspace then holds a part of
+    8 heads x 132 floats per (pair, split), 256-byte aligned, and a ticket per
+    pair."""
+    lay = L(k_group=64, v_group=64, window=0, k_per_channel=True)
+    assert kvq.kvq_decode_workspace_bytes(lay, 16, 4096) == 0        # 128 pairs: one CTA each
+    assert kvq.kvq_decode_workspace_bytes(lay, 8, 511) == 0          # too short to split
+    pairs = 8 * 8                                                    # B8: 64 pairs, two CTAs each
+    part = (pairs * 2 * 8 * 132 * 4 + 255) // 256 * 256
+    assert kvq.kvq_decode_workspace_bytes(lay, 8, 16384) == part + pairs * 4
+    pairs = 1 * 8                                                    # B1: 8 pairs, eight CTAs each
+    part = (pairs * 8 * 8 * 132 * 4 + 255) // 256 * 256
+    assert kvq.kvq_decode_workspace_bytes(lay, 1, 16384) == part + pairs * 4
+    assert kvq.kvq_decode_workspace_bytes(L(head_dim=64, k_group=64, v_group=64, window=0, k_per_channel=True),
+                                          1, 16384) == 0             # head_dim 64: the chunked-prefill path
