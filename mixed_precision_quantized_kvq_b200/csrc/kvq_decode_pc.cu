@@ -153,6 +153,13 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 __device__ __forceinline__ uint32_t h2bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+// both parts of the pair (x, y): the fp16 rounding, and the fp16 rounding of the rest
+__device__ __forceinline__ void f16_parts(float x, float y, uint32_t& hi, uint32_t& lo) {
+    const __half2 h = __floats2half2_rn(x, y);
+    const float2 f = __half22float2(h);
+    hi = h2bits(h);
+    lo = h2bits(__floats2half2_rn(x - f.x, y - f.y));
+}
 // part `limb` (0: the fp16 rounding, 1: the fp16 rounding of the rest) of the pair (x, y)
 __device__ __forceinline__ uint32_t f16_part(float x, float y, int limb) {
     const __half2 hi = __floats2half2_rn(x, y);
@@ -559,8 +566,10 @@ __global__ void __launch_bounds__(nw_max(NH) * 32, 1) decode_pc_kernel(const Par
                 const float za = hbits(mA >> 16), zb = hbits(mB >> 16);
 #pragma unroll
                 for (int r = 0; r < NH; ++r) {
-                    ph[(gg * 8 + 2 * r) * PHROW + lane] = f16_part(pA[r] * sa, pB[r] * sb, 0);
-                    ph[(gg * 8 + 2 * r + 1) * PHROW + lane] = f16_part(pA[r] * sa, pB[r] * sb, 1);
+                    uint32_t hi, lo;
+                    f16_parts(pA[r] * sa, pB[r] * sb, hi, lo);
+                    ph[(gg * 8 + 2 * r) * PHROW + lane] = hi;
+                    ph[(gg * 8 + 2 * r + 1) * PHROW + lane] = lo;
                     z[r] = fmaf(pA[r], za, fmaf(pB[r], zb, z[r]));
                 }
             }
