@@ -116,11 +116,14 @@ def test_split_pairs():
     are split between CTAs that merge through the workspace (the last CTA to
     finish merges every split in split order).  Against the oracle, with an
     empty sequence; the static-scratch entry point gives the same bits; the
-    call without a workspace (one CTA per pair) agrees within tolerance."""
-    w = pc(batch=2, num_kv_heads=2, num_q_heads=8, ragged=(2500, 4200), window=64, k_group=64, v_group=64)
+    call without a workspace (one CTA per pair) agrees within tolerance.  The
+    third sequence holds two tiles, so most of its splits have none and store
+    empty parts."""
+    w = pc(batch=3, num_kv_heads=2, num_q_heads=8, ragged=(2500, 4200), window=64, k_group=64, v_group=64)
     lens = wl.lengths(w)
     lens[1] = 0
     lens[0] = max(int(lens[0]), 3000)
+    lens[2] = 100
     pair = Pair(w, lens)
     pair.prefill(with_f32=False)
     max_len = int(lens.max())
