@@ -46,6 +46,9 @@ WORKLOADS = {"llama8b": wl.LLAMA8B, "ragged": wl.RAGGED,
              # the memory-budget planner's pick at 116 B per token-head: key groups of 64 positions
              "per_channel_llama8b": wl.LLAMA8B.with_(name="llama3_8b_layer_b16_l4096_k4pc64v2g64_w128",
                                                      k_group=64, v_group=64, k_per_channel=True),
+             # eight query heads per kv-head (the decode kernel's eight-head build), 64 of them
+             "per_channel_gqa8": wl.LLAMA8B.with_(name="b16_l4096_q64kv8_k4pc64v2g64_w128", num_q_heads=64,
+                                                  k_group=64, v_group=64, k_per_channel=True),
              # the same layout at long context, few pairs (8 x 8): each pair split between CTAs
              "per_channel_sweep": wl.SWEEP.with_(name="sweep_b8_l16384_k4pc64v2g64_w0", k_bits=4, v_bits=2,
                                                  k_group=64, v_group=64, k_per_channel=True)}
