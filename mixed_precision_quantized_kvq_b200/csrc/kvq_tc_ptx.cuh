@@ -1,7 +1,7 @@
-// Thin wrappers over the sm_100a PTX used by the tensor-core decode kernel:
-// mbarriers, 1-D bulk copies (TMA engine, no multicast), tcgen05 tensor
-// memory allocation / load / store, tcgen05.mma with the A operand in tensor
-// memory, and the shared-memory matrix descriptor.
+// Thin wrappers over the sm_100a PTX used by the tensor-core decode kernels:
+// mbarriers, the async-proxy fence, tcgen05 tensor memory allocation / load /
+// store, tcgen05.mma with the A operand in tensor memory, and the
+// shared-memory matrix descriptor.
 #pragma once
 
 #include <stdint.h>
@@ -55,16 +55,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
     }
 }
 
-// ---------------------------------------------------------------- bulk copy
-// 1-D global -> shared copy on the TMA engine; completion is signalled on
-// `bar` as transaction bytes.  dst, src 16-byte aligned; bytes % 16 == 0.
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
 // order this thread's generic-proxy shared-memory accesses before later
 // async-proxy (bulk copy / tensor core) accesses
 __device__ __forceinline__ void fence_proxy_async() {
